@@ -1,0 +1,174 @@
+"""Thin Python binding of the C ABI in ``include/nvq.h`` (ctypes).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libnvq.so``.  PyTorch provides device memory and streams.  If
+the library has not been built, importing this module raises ImportError: no
+entry point has a CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libnvq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m bit_weight_quantized_nvq_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_c_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+
+#: every symbol the C header declares, with (restype, argtypes)
+SIGNATURES = {
+    "nvq_version": (ctypes.c_int, []),
+    "nvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "nvq_last_cuda_error": (ctypes.c_char_p, []),
+    "nvq_pack_nvfp4": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp]),
+    "nvq_quantize_act_q8_0": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp]),
+    "nvq_gemv": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
+                                _c_i64, _vp, _vp]),
+    "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
+    "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
+                                _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
+    "nvq_debug_subblock_sums": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _vp,
+                                               _vp]),
+}
+
+for _name, (_res, _args) in SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+NVQ_OK = 0
+NVQ_ERR_INVALID_ARG = 1
+NVQ_ERR_BAD_SHAPE = 2
+NVQ_ERR_MISALIGNED = 3
+NVQ_ERR_CUDA = 4
+NVQ_ERR_UNSUPPORTED_DEVICE = 5
+NVQ_ERR_WORKSPACE = 6
+
+
+class NVQError(RuntimeError):
+    """A non-OK status returned by the library."""
+
+    def __init__(self, func: str, status: int):
+        self.status = status
+        msg = _lib.nvq_status_string(status).decode()
+        if status == NVQ_ERR_CUDA:
+            msg += f" [{_lib.nvq_last_cuda_error().decode()}]"
+        super().__init__(f"{func}: status {status}: {msg}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libnvq.so`` (raw C entry points)."""
+    return _lib
+
+
+def _check(func: str, status: int) -> None:
+    if status != NVQ_OK:
+        raise NVQError(func, status)
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return int(t)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def version() -> int:
+    return _lib.nvq_version()
+
+
+# ---------------------------------------------------------------------------
+
+def pack_nvfp4(w: np.ndarray):
+    """Host NVFP4 packer: fp32 W[N, K] -> (codes uint8 [N, K/2], scales uint8
+    [N, K/16], g float)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K // 2), np.uint8)
+    scales = np.empty((N, K // 16), np.uint8)
+    g = ctypes.c_float(0.0)
+    _check("nvq_pack_nvfp4", _lib.nvq_pack_nvfp4(
+        _ptr(w), N, K, _ptr(codes), _ptr(scales), ctypes.addressof(g)))
+    return codes, scales, g.value
+
+
+def quantize_act_q8_0(x: torch.Tensor, q: torch.Tensor | None = None,
+                      d: torch.Tensor | None = None, stream=None):
+    """Q8_0 of device fp32 x[M, K] -> (q int8 [M, K], d float16 [M, K/32])."""
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if d is None:
+        d = torch.empty((M, K // 32), dtype=torch.float16, device=x.device)
+    _check("nvq_quantize_act_q8_0", _lib.nvq_quantize_act_q8_0(
+        _ptr(x), M, K, _ptr(q), _ptr(d), _stream(stream)))
+    return q, d
+
+
+def gemv(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
+         d: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode GEMV (M = 1..16): y[M, N] fp32."""
+    N = codes.shape[0]
+    M, K = q.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=q.device)
+    _check("nvq_gemv", _lib.nvq_gemv(
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y),
+        _stream(stream)))
+    return y
+
+
+def gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.nvq_gemm_workspace_size(M, N, K))
+
+
+def gemm(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
+         d: torch.Tensor, y: torch.Tensor | None = None,
+         workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Prefill GEMM (tcgen05): y[M, N] fp32."""
+    N = codes.shape[0]
+    M, K = q.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=q.device)
+    ws_bytes = gemm_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    _check("nvq_gemm", _lib.nvq_gemm(
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y),
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return y
+
+
+def debug_subblock_sums(codes: torch.Tensor, q: torch.Tensor,
+                        isum: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Integer per-16 subblock sums of the GEMV: int32 [M, N, K/16]."""
+    N = codes.shape[0]
+    M, K = q.shape
+    if isum is None:
+        isum = torch.empty((M, N, K // 16), dtype=torch.int32, device=q.device)
+    _check("nvq_debug_subblock_sums", _lib.nvq_debug_subblock_sums(
+        _ptr(codes), N, K, _ptr(q), M, _ptr(isum), _stream(stream)))
+    return isum

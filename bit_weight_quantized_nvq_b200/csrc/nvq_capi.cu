@@ -1,0 +1,174 @@
+// C ABI of the library: host-side argument validation, device checks and
+// dispatch to the kernel launchers.  Nothing here allocates device memory.
+#include <atomic>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/nvq.h"
+#include "nvq_internal.h"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kMaxDevices = 64;
+
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+// 0 = not yet checked, 1 = sm_100, 2 = other architecture.
+std::atomic<int> g_device_ok[kMaxDevices];
+std::atomic<int> g_device_sms[kMaxDevices];
+
+bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+nvq_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return NVQ_OK;
+  t_last_cuda_error = e;
+  return NVQ_ERR_CUDA;
+}
+
+// The current device must be compute capability 10.0 (B200, sm_100a).
+nvq_status check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  if (dev < 0 || dev >= kMaxDevices) return NVQ_ERR_UNSUPPORTED_DEVICE;
+  int state = g_device_ok[dev].load(std::memory_order_relaxed);
+  if (state == 0) {
+    int major = 0, minor = 0, sms = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_status(e);
+    }
+    state = (major == 10 && minor == 0) ? 1 : 2;
+    g_device_sms[dev].store(sms, std::memory_order_relaxed);
+    g_device_ok[dev].store(state, std::memory_order_relaxed);
+  }
+  return state == 1 ? NVQ_OK : NVQ_ERR_UNSUPPORTED_DEVICE;
+}
+
+// Shapes and pointers shared by the weight x activation entry points:
+// K a positive multiple of 64, M within [m_min, m_max] (or 0), every pointer
+// non-NULL and 16-byte aligned unless the product is empty (M == 0 or
+// N == 0).  `need_scales` is false for the integer-sum export, which reads
+// neither the weight scales nor the activation scales.
+nvq_status check_dot_args(const void* codes, const void* scales, int64_t N,
+                          int64_t K, const void* q, const void* d, int64_t M,
+                          const void* y, int64_t m_min, int64_t m_max,
+                          bool need_scales) {
+  if (N < 0 || K < 0 || M < 0) return NVQ_ERR_INVALID_ARG;
+  if (K == 0 || K % 64 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (K > (int64_t{1} << 30) || N > (int64_t{1} << 30)) return NVQ_ERR_BAD_SHAPE;
+  if (M != 0 && (M < m_min || M > m_max)) return NVQ_ERR_BAD_SHAPE;
+  if (N == 0 || M == 0) return NVQ_OK;
+  if (!codes || !q || !y) return NVQ_ERR_INVALID_ARG;
+  if (need_scales && (!scales || !d)) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(q) || !aligned16(y)) return NVQ_ERR_MISALIGNED;
+  if (need_scales && (!aligned16(scales) || !aligned16(d))) return NVQ_ERR_MISALIGNED;
+  return NVQ_OK;
+}
+
+}  // namespace
+
+namespace nvq {
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int sms = g_device_sms[dev].load(std::memory_order_relaxed);
+  return sms > 0 ? sms : 148;
+}
+}  // namespace nvq
+
+extern "C" {
+
+int nvq_version(void) { return kVersion; }
+
+const char* nvq_status_string(nvq_status status) {
+  switch (status) {
+    case NVQ_OK: return "ok";
+    case NVQ_ERR_INVALID_ARG: return "invalid argument (NULL pointer, negative size or bad value)";
+    case NVQ_ERR_BAD_SHAPE: return "unsupported shape (K must be a multiple of 64; M within the entry point's range)";
+    case NVQ_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case NVQ_ERR_CUDA: return "CUDA runtime error (see nvq_last_cuda_error)";
+    case NVQ_ERR_UNSUPPORTED_DEVICE: return "current device is not an sm_100 (B200) GPU";
+    case NVQ_ERR_WORKSPACE: return "workspace missing or smaller than nvq_gemm_workspace_size";
+    default: return "unknown status";
+  }
+}
+
+const char* nvq_last_cuda_error(void) { return cudaGetErrorName(t_last_cuda_error); }
+
+nvq_status nvq_quantize_act_q8_0(const float* x, int64_t M, int64_t K,
+                                 int8_t* q, uint16_t* d, void* stream) {
+  if (M < 0 || K < 0) return NVQ_ERR_INVALID_ARG;
+  if (K % 32 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (M == 0 || K == 0) return NVQ_OK;
+  if (M * K > (int64_t{1} << 40)) return NVQ_ERR_BAD_SHAPE;
+  if (!x || !q || !d) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(d)) return NVQ_ERR_MISALIGNED;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_quantize_q8_0(x, M, K, q, d,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                    int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                    int64_t M, float* y, void* stream) {
+  nvq_status st = check_dot_args(codes, scales, N, K, q, d, M, y, 1, 16, true);
+  if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;  // NaN scale
+  if (N == 0 || M == 0) return NVQ_OK;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_gemv(codes, scales, g, N, K, q, d, M, y,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || K <= 0 || N < 0) return 0;
+  return nvq::gemm_workspace_size(M, N, K);
+}
+
+nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
+                    int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                    int64_t M, float* y, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  nvq_status st = check_dot_args(codes, scales, N, K, q, d, M, y, 1,
+                                 int64_t{1} << 24, true);
+  if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
+  if (N == 0 || M == 0) return NVQ_OK;
+  if (!workspace || workspace_bytes < nvq::gemm_workspace_size(M, N, K))
+    return NVQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return NVQ_ERR_MISALIGNED;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_gemm(codes, scales, g, N, K, q, d, M, y, workspace,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+nvq_status nvq_debug_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
+                                   const int8_t* q, int64_t M, int32_t* isum,
+                                   void* stream) {
+  nvq_status st = check_dot_args(codes, nullptr, N, K, q, nullptr, M, isum, 1, 16,
+                                 false);
+  if (st != NVQ_OK) return st;
+  if (N == 0 || M == 0) return NVQ_OK;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_subblock_sums(codes, N, K, q, M, isum,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Device helpers for the NVFP4 x Q8_0 kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace nvq {
+namespace dev {
+
+// Integer LUT c = 2*E2M1(code), as packed signed bytes.  E2M1 (OCP MX):
+// codes 0..7 are 0, .5, 1, 1.5, 2, 3, 4, 6 and bit 3 is the sign, so c runs
+// over 0, 1, 2, 3, 4, 6, 8, 12 and their negatives ("HANDOFF: flint CPU
+// optimization (Q4_1 + NVFP4)", section 3, "Bias trick": the integer codes
+// lie in -12..12).  Byte j of the pair (lo, hi) is the value of index j.
+constexpr uint32_t kLutPosLo = 0x03020100u;  // codes 0..3   ->  0,  1,  2,  3
+constexpr uint32_t kLutPosHi = 0x0C080604u;  // codes 4..7   ->  4,  6,  8, 12
+constexpr uint32_t kLutNegLo = 0xFDFEFF00u;  // codes 8..11  ->  0, -1, -2, -3
+constexpr uint32_t kLutNegHi = 0xF4F8FAFCu;  // codes 12..15 -> -4, -6, -8,-12
+
+// Decode the eight E2M1 codes of one 32-bit word (nibble i = element i) into
+// two words of four signed bytes c = 2*E2M1: `lo` holds elements 0..3 and
+// `hi` elements 4..7.  Each byte is looked up twice with a byte permute
+// (positive and negative halves of the table, indexed by the code's low
+// three bits) and the sign bit picks between the two.
+__device__ __forceinline__ void decode_e2m1x8(uint32_t w, uint32_t& lo,
+                                              uint32_t& hi) {
+  const uint32_t idx = w & 0x77777777u;
+  // selector of the final permute: byte i from p (i) or from n (4 + i)
+  const uint32_t pick = ((w >> 1) & 0x44444444u) | 0x32103210u;
+  const uint32_t idx_hi = idx >> 16;
+  const uint32_t pick_hi = pick >> 16;
+  const uint32_t p0 = __byte_perm(kLutPosLo, kLutPosHi, idx);
+  const uint32_t n0 = __byte_perm(kLutNegLo, kLutNegHi, idx);
+  const uint32_t p1 = __byte_perm(kLutPosLo, kLutPosHi, idx_hi);
+  const uint32_t n1 = __byte_perm(kLutNegLo, kLutNegHi, idx_hi);
+  lo = __byte_perm(p0, n0, pick);
+  hi = __byte_perm(p1, n1, pick_hi);
+}
+
+// Two UE4M3 scale bytes (low byte = first subblock) to fp32, exactly.  UE4M3
+// is E4M3 with the sign bit 0, so the hardware E4M3 -> f16 conversion
+// applies; every UE4M3 value (2^-9 .. 448) is exact in fp16.
+__device__ __forceinline__ float2 ue4m3x2_to_float2(uint32_t two_bytes) {
+  uint32_t h2;
+  const uint16_t in = static_cast<uint16_t>(two_bytes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  __half2 h = *reinterpret_cast<__half2*>(&h2);
+  return __half22float2(h);
+}
+
+__device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) {
+  return __dp4a(static_cast<int>(a), static_cast<int>(b), c);
+}
+
+// 128-bit streaming load: read-only path, no L1 allocation (each weight
+// byte is used once), 256-byte L2 prefetch.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace dev
+}  // namespace nvq

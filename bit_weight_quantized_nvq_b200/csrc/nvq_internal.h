@@ -1,0 +1,37 @@
+// Internal declarations shared by the library's translation units.
+// Launchers assume validated arguments (the C ABI layer checks them).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace nvq {
+
+// Q8_0 activation quantiser over M*K/32 blocks.
+cudaError_t launch_quantize_q8_0(const float* x, int64_t M, int64_t K,
+                                 int8_t* q, uint16_t* d, cudaStream_t stream);
+
+// Decode GEMV for M = 1..16.
+cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                        int64_t N, int64_t K, const int8_t* q,
+                        const uint16_t* d, int64_t M, float* y,
+                        cudaStream_t stream);
+
+// Integer per-16 subblock sums through the GEMV's decode/dot code.
+cudaError_t launch_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
+                                 const int8_t* q, int64_t M, int32_t* isum,
+                                 cudaStream_t stream);
+
+// Prefill GEMM (tcgen05) and the size of its activation workspace.
+size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm(const uint8_t* codes, const uint8_t* scales, float g,
+                        int64_t N, int64_t K, const int8_t* q,
+                        const uint16_t* d, int64_t M, float* y,
+                        void* workspace, cudaStream_t stream);
+
+// Number of streaming multiprocessors of the current device (cached).
+int device_sm_count();
+
+}  // namespace nvq

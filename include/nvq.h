@@ -1,0 +1,178 @@
+/*
+ * nvq.h - C ABI of the NVFP4 x Q8_0 dequantise-and-dot library (B200, sm_100a).
+ *
+ * The library computes the fused dequantise-and-dot product used in
+ * quantised LLM inference: 4-bit block-scaled weights (NVFP4) times 8-bit
+ * block-quantised activations (Q8_0), for decode (matrix-vector, M = 1..16)
+ * and prefill (GEMM, M up to thousands of tokens).
+ *
+ * Sources of the operations (web pages, cited by title and section):
+ *  - "HANDOFF: flint CPU optimization (Q4_1 + NVFP4)", section 3 "Code map
+ *    (NVFP4 work)": the NVFP4-weight x Q8_0-activation row dot
+ *    (ggml_vec_dot_nvfp4_q8_0), weights handled in 64-element blocks with one
+ *    scale per 16 elements; the tiled prefill kernels on the same operands;
+ *    and the "Bias trick" paragraph: integer weight codes 2*E2M1 (-12..12)
+ *    and sum(w*a) = sum((w+12)*a) - 12*bsum16.
+ *  - The spke.com tutorial on 2-bit GGUF builds of a 27B model, GGML type
+ *    table (download step): Q8_0 = 32 int8 values + one fp16 scale, 34 bytes.
+ *  - "TKintegers K5: 3.21x prefill and 3.10x decode throughput vs TorchAO
+ *    FP8 on NVIDIA L4": compact weight tiles expanded to FP16 tensor-core
+ *    operands with FP32 accumulation (the prefill GEMM's design).
+ *
+ * Data formats (all planar, row-major, owned by the caller):
+ *  - NVFP4 weights W[N, K]:
+ *      codes  uint8 [N, K/2]  : E2M1 codes, element 2i in the low nibble of
+ *                               byte i and element 2i+1 in the high nibble;
+ *                               bit 3 of a code is the sign, codes 0..7 are
+ *                               0, .5, 1, 1.5, 2, 3, 4, 6 (OCP MX E2M1).
+ *      scales uint8 [N, K/16] : one UE4M3 scale per 16-element subblock
+ *                               (E4M3 with sign 0, bias 7; max 448 = 0x7E;
+ *                               bytes >= 0x7F are not valid scales).
+ *      g      float           : per-tensor scale.
+ *      w[n,k] = g * UE4M3(scales[n,k/16]) * E2M1(code[n,k]).
+ *  - Q8_0 activations A[M, K]:
+ *      q      int8   [M, K]     : codes in -127..127.
+ *      d      uint16 [M, K/32]  : IEEE binary16 bit patterns, one per 32.
+ *      a[m,k] = fp16(d[m,k/32]) * q[m,k].
+ *  - Output y float [M, N], row-major, overwritten (never accumulated into):
+ *      y[m,n] = sum_k w[n,k] * a[m,k]
+ *             = sum over 16-subblocks sb of g*s_w*d_a*0.5*isum[m,n,sb],
+ *      isum[m,n,sb] = sum over the subblock of (2*E2M1(code)) * q.
+ *    Accuracy: |y - exact| <= 1e-5 * sum_sb |term_sb| + 1e-6 per element.
+ *
+ * Conventions shared by every entry point:
+ *  - Shapes: K a positive multiple of 64 (the 64-element blocks of the row
+ *    dot).  The empty product (N == 0 or M == 0) is accepted and does
+ *    nothing.
+ *  - Device pointers must be 16-byte aligned (NVQ_ERR_MISALIGNED).
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  Device entry points only enqueue work and return at once;
+ *    results are ready when the stream reaches them.
+ *  - The library allocates no device memory and keeps no state beyond a
+ *    per-device cache of attributes.  It never prints and never aborts.
+ *  - Errors: arguments are validated on the host before anything is
+ *    enqueued, so a non-OK status other than NVQ_ERR_CUDA means nothing was
+ *    launched.  NVQ_ERR_CUDA reports a CUDA runtime error seen while
+ *    launching (cudaGetLastError); nvq_last_cuda_error() names it.
+ *  - Entry points may be called from several host threads at once.
+ */
+#ifndef NVQ_H_
+#define NVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int nvq_status;
+
+#define NVQ_OK                     0
+#define NVQ_ERR_INVALID_ARG        1  /* NULL pointer, negative size, bad value */
+#define NVQ_ERR_BAD_SHAPE          2  /* K % 64 != 0, M out of the entry's range */
+#define NVQ_ERR_MISALIGNED         3  /* a device pointer not 16-byte aligned */
+#define NVQ_ERR_CUDA               4  /* CUDA runtime error while launching */
+#define NVQ_ERR_UNSUPPORTED_DEVICE 5  /* current device is not sm_100 */
+#define NVQ_ERR_WORKSPACE          6  /* workspace missing or too small */
+
+/* Library version, major*10000 + minor*100 + patch. */
+int nvq_version(void);
+
+/* Short English description of a status code (a static string). */
+const char* nvq_status_string(nvq_status status);
+
+/* Name of the last CUDA error an entry point met on this host thread
+ * (a static string; "cudaSuccess" if none). */
+const char* nvq_last_cuda_error(void);
+
+/*
+ * nvq_pack_nvfp4 - host-side NVFP4 packer of fp32 weights (not timed; used
+ * by generators and loaders).
+ *
+ * w      host float [N, K] row-major, finite values.
+ * codes  host uint8 [N, K/2], scales host uint8 [N, K/16], g host float*:
+ *        outputs, caller-owned.
+ * Recipe, fp32 with one rounding per operation: g = amax(|w|) / (6*448);
+ * per 16-element subblock s = UE4M3(amax_blk / (6*g)) (nearest, ties to
+ * even, saturating at 448); code = E2M1(w / (g*s)) (nearest, ties to even,
+ * saturating at 6, zero stored as +0); a subblock whose s or g*s is 0 stores
+ * codes 0.  Requires K % 16 == 0 (K % 64 for the device entry points).
+ * Runs on the calling thread plus up to hardware_concurrency helper threads.
+ * Errors: NVQ_ERR_INVALID_ARG (NULL, negative sizes, non-finite w),
+ * NVQ_ERR_BAD_SHAPE (K % 16 != 0).
+ */
+nvq_status nvq_pack_nvfp4(const float* w, int64_t N, int64_t K,
+                          uint8_t* codes, uint8_t* scales, float* g);
+
+/*
+ * nvq_quantize_act_q8_0 - fused Q8_0 activation quantiser (one pass).
+ *
+ * x  device float [M, K] row-major, finite values.
+ * q  device int8 [M, K], d device uint16 (fp16 bits) [M, K/32]: outputs.
+ * Per 32-element block, fp32 IEEE arithmetic: amax = max|x|,
+ * d32 = amax / 127 (correctly rounded division), q = rint(x / d32) (true
+ * division, round half to even) clamped to +-127, d = fp16(d32) (round to
+ * nearest even).  A block with d32 == 0 gives q = 0, d = 0.  Bit-exact.
+ * Errors: NVQ_ERR_INVALID_ARG, NVQ_ERR_BAD_SHAPE (K % 32 != 0),
+ * NVQ_ERR_MISALIGNED, NVQ_ERR_UNSUPPORTED_DEVICE, NVQ_ERR_CUDA.
+ */
+nvq_status nvq_quantize_act_q8_0(const float* x, int64_t M, int64_t K,
+                                 int8_t* q, uint16_t* d, void* stream);
+
+/*
+ * nvq_gemv - decode GEMV, y[M, N] = A[M, K] . W[N, K]^T for M = 1..16.
+ *
+ * HBM-streaming kernel: each weight byte is read once with 128-bit loads;
+ * E2M1 codes are decoded in registers to the integer LUT 2*E2M1, the
+ * per-subblock integer sums are formed with dp4a, rescaled by s_w*d_a in
+ * fp32 and reduced across the warp; y = 0.5*g*acc.
+ * Errors: NVQ_ERR_INVALID_ARG, NVQ_ERR_BAD_SHAPE (K % 64 != 0, M outside
+ * 1..16), NVQ_ERR_MISALIGNED, NVQ_ERR_UNSUPPORTED_DEVICE, NVQ_ERR_CUDA.
+ */
+nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                    int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                    int64_t M, float* y, void* stream);
+
+/*
+ * nvq_gemm_workspace_size - bytes of device workspace nvq_gemm needs for
+ * M tokens of K features (0 when M == 0).  It holds the activations
+ * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q.
+ */
+size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * nvq_gemm - prefill GEMM, y[M, N] = A[M, K] . W[N, K]^T for any M >= 1
+ * (tuned for M >= 256) on the tcgen05 tensor cores.
+ *
+ * The activations are expanded once into `workspace` as fp16 pairs
+ * hi = fp16(d*q), lo = fp16(d*q - hi), exact (hi + lo == d*q).  Weight tiles
+ * are expanded in shared memory to fp16 w' = E2M1*s_w (exact) and every
+ * 64-wide K slice is multiplied by tcgen05.mma (kind::f16) against
+ * [hi; lo], accumulating in fp32 in tensor memory; y = g * (acc_hi + acc_lo).
+ * Every product is exact; only the fp32 accumulation rounds.
+ * workspace: device, caller-owned, >= nvq_gemm_workspace_size(M, N, K)
+ * bytes, 16-byte aligned; its contents are scratch.
+ * Errors: as nvq_gemv (M >= 1), plus NVQ_ERR_WORKSPACE.
+ */
+nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
+                    int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                    int64_t M, float* y, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * nvq_debug_subblock_sums - the integer per-16 subblock sums the GEMV forms,
+ * exported for bit-exact checking:
+ * isum[m, n, sb] = sum_{k in sb} (2*E2M1(code[n,k])) * q[m,k], int32
+ * [M, N, K/16] (|isum| <= 16*12*127).  Uses the GEMV's own decode and dp4a
+ * code.  Errors: as nvq_gemv (M = 1..16).
+ */
+nvq_status nvq_debug_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
+                                   const int8_t* q, int64_t M, int32_t* isum,
+                                   void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* NVQ_H_ */

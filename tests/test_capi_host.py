@@ -1,0 +1,139 @@
+"""Host-side tests of the C ABI: the library loads and exports every symbol
+the header declares, host validation returns the documented status codes
+before anything is launched, and the host NVFP4 packer is bit-exact against
+the oracle's packer.  No GPU is needed."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as o
+from bit_weight_quantized_nvq_b200 import capi, workloads as wl
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "nvq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 9
+    lib = capi.lib()
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in capi.SIGNATURES, name
+
+
+def test_version_and_status_strings():
+    assert capi.version() >= 10000
+    lib = capi.lib()
+    for s in range(7):
+        assert lib.nvq_status_string(s)
+    assert b"unknown" in lib.nvq_status_string(99)
+    assert lib.nvq_last_cuda_error() == b"cudaSuccess"
+
+
+def _dev_like(nbytes, offset=0):
+    # host buffers stand in for device pointers: validation never reads them
+    buf = np.zeros(nbytes + 64, np.uint8)
+    base = buf.ctypes.data
+    return buf, (base + (-base % 16) + offset)
+
+
+def test_host_validation_status_codes():
+    lib = capi.lib()
+    keep = []
+    def p(nbytes=4096, off=0):
+        b, a = _dev_like(nbytes, off)
+        keep.append(b)
+        return a
+    codes, scales, q, d, y = p(), p(), p(), p(), p()
+    gemv = lib.nvq_gemv
+    assert gemv(codes, scales, 1.0, 8, 100, q, d, 1, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert gemv(codes, scales, 1.0, 8, 0, q, d, 1, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert gemv(codes, scales, 1.0, 8, 64, q, d, 17, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert gemv(codes, scales, 1.0, -1, 64, q, d, 1, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert gemv(None, scales, 1.0, 8, 64, q, d, 1, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert gemv(codes, None, 1.0, 8, 64, q, d, 1, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert gemv(codes, scales, 1.0, 8, 64, q, d, 1, p(off=4), None) == capi.NVQ_ERR_MISALIGNED
+    assert gemv(p(off=8), scales, 1.0, 8, 64, q, d, 1, y, None) == capi.NVQ_ERR_MISALIGNED
+    assert gemv(codes, scales, float("nan"), 8, 64, q, d, 1, y, None) == capi.NVQ_ERR_INVALID_ARG
+    # the empty product is a no-op that launches nothing
+    assert gemv(codes, scales, 1.0, 0, 64, q, d, 1, y, None) == capi.NVQ_OK
+    assert gemv(None, None, 1.0, 8, 64, None, None, 0, None, None) == capi.NVQ_OK
+
+    quant = lib.nvq_quantize_act_q8_0
+    assert quant(p(), 1, 48, q, d, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert quant(None, 1, 64, q, d, None) == capi.NVQ_ERR_INVALID_ARG
+    assert quant(p(off=4), 1, 64, q, d, None) == capi.NVQ_ERR_MISALIGNED
+    assert quant(None, 0, 64, None, None, None) == capi.NVQ_OK
+
+    gemm = lib.nvq_gemm
+    ws = p(1 << 16)
+    need = lib.nvq_gemm_workspace_size(4, 8, 64)
+    assert need > 0
+    assert gemm(codes, scales, 1.0, 8, 64, q, d, 4, y, None, need, None) == capi.NVQ_ERR_WORKSPACE
+    assert gemm(codes, scales, 1.0, 8, 64, q, d, 4, y, ws, need - 1, None) == capi.NVQ_ERR_WORKSPACE
+    assert gemm(codes, scales, 1.0, 8, 96, q, d, 4, y, ws, need, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert gemm(codes, scales, 1.0, 8, 64, q, d, 4, y, p(1 << 16, 8), need, None) == capi.NVQ_ERR_MISALIGNED
+    assert lib.nvq_gemm_workspace_size(0, 8, 64) == 0
+
+    sums = lib.nvq_debug_subblock_sums
+    assert sums(codes, 8, 64, q, 17, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert sums(codes, 8, 32, q, 1, y, None) == capi.NVQ_ERR_BAD_SHAPE
+
+
+def test_pack_rejects_bad_arguments():
+    lib = capi.lib()
+    w = np.zeros((2, 24), np.float32)
+    out = np.zeros(64, np.uint8)
+    g = ctypes.c_float()
+    assert lib.nvq_pack_nvfp4(w.ctypes.data, 2, 24, out.ctypes.data, out.ctypes.data,
+                              ctypes.addressof(g)) == capi.NVQ_ERR_BAD_SHAPE
+    w = np.zeros((2, 32), np.float32)
+    w[1, 3] = np.inf
+    assert lib.nvq_pack_nvfp4(w.ctypes.data, 2, 32, out.ctypes.data, out.ctypes.data,
+                              ctypes.addressof(g)) == capi.NVQ_ERR_INVALID_ARG
+    assert lib.nvq_pack_nvfp4(None, 2, 32, out.ctypes.data, out.ctypes.data,
+                              ctypes.addressof(g)) == capi.NVQ_ERR_INVALID_ARG
+    with pytest.raises(capi.NVQError):
+        capi.pack_nvfp4(np.zeros((2, 40), np.float32))
+
+
+@pytest.mark.parametrize("case", ["gemv_4096", "decode_boost", "tiny_scales", "zeros",
+                                  "ties", "huge_range"])
+def test_host_packer_matches_oracle_bit_exactly(case):
+    rng = np.random.default_rng(77)
+    if case == "gemv_4096":
+        w = wl.weights("gemv_4096", "W", 512, 4096)
+    elif case == "decode_boost":
+        w = wl.weights("decode_sweep", "W", 300, 5120, boost_columns=True)
+    elif case == "tiny_scales":
+        w = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+        w[:, ::16] *= 1e5                    # one big element per subblock row
+        w[3, :] *= 1e-7                      # a row of subnormal-scale subblocks
+    elif case == "zeros":
+        w = np.zeros((8, 64), np.float32)
+    elif case == "ties":
+        # exact E2M1 ties: amax 6*448*2^-8 makes g = 2^-8 and s = 1 where the
+        # subblock max is 6*2^-8; ratios then land on 0.25, 0.75, ..., 5
+        w = np.zeros((4, 64), np.float32)
+        base = np.float32(2.0 ** -8)
+        w[:, 0] = 6 * 448 * base
+        for sb in range(1, 4):
+            w[:, sb * 16] = 6 * base
+            w[:, sb * 16 + 1:sb * 16 + 8] = np.float32([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]) * base
+            w[1::2, sb * 16 + 1:sb * 16 + 8] *= -1
+    else:  # huge_range
+        w = (rng.standard_normal((32, 128)) * 10.0 ** rng.uniform(-30, 30, (32, 1))).astype(np.float32)
+    c, s, g = capi.pack_nvfp4(w)
+    co, so, go = o.pack_nvfp4(w)
+    assert np.float32(g) == go
+    assert np.array_equal(s, so)
+    assert np.array_equal(c, co)
