@@ -26,6 +26,15 @@ _lib = ctypes.CDLL(LIB_PATH)
 _c_i64 = ctypes.c_int64
 _vp = ctypes.c_void_p
 
+
+class Linear(ctypes.Structure):
+    """``nvq_linear``: one NVFP4 weight matrix in device memory."""
+    _fields_ = [("codes", _vp), ("scales", _vp), ("g", ctypes.c_float),
+                ("N", _c_i64), ("K", _c_i64)]
+
+
+STACK_LINEARS = 7
+
 #: every symbol the C header declares, with (restype, argtypes)
 SIGNATURES = {
     "nvq_version": (ctypes.c_int, []),
@@ -40,6 +49,9 @@ SIGNATURES = {
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "nvq_debug_subblock_sums": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _vp,
                                                _vp]),
+    "nvq_decoder_stack": (ctypes.c_int, [ctypes.POINTER(Linear), _c_i64, _vp, _c_i64,
+                                         ctypes.POINTER(_vp), _vp, ctypes.c_size_t, _vp]),
+    "nvq_decoder_stack_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Linear), _c_i64]),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():
@@ -172,3 +184,39 @@ def debug_subblock_sums(codes: torch.Tensor, q: torch.Tensor,
     _check("nvq_debug_subblock_sums", _lib.nvq_debug_subblock_sums(
         _ptr(codes), N, K, _ptr(q), M, _ptr(isum), _stream(stream)))
     return isum
+
+
+class DecoderStack:
+    """Device-resident linear layers of a dense decoder stack (7 NVFP4
+    matrices per layer: q, k, v, o, up, gate, down) and the buffers of one
+    pass; ``forward`` enqueues every layer through ``nvq_decoder_stack``."""
+
+    def __init__(self, layers, M: int, device="cuda"):
+        """layers: list of n_layers lists of 7 (codes, scales, g) with codes
+        and scales device tensors."""
+        self.n_layers = len(layers)
+        self.M = M
+        arr = (Linear * (STACK_LINEARS * self.n_layers))()
+        self._keep = []
+        for l, layer in enumerate(layers):
+            if len(layer) != STACK_LINEARS:
+                raise ValueError("each layer needs 7 matrices")
+            for i, (codes, scales, g) in enumerate(layer):
+                arr[STACK_LINEARS * l + i] = Linear(codes.data_ptr(), scales.data_ptr(), float(g),
+                                                    codes.shape[0], codes.shape[1] * 2)
+                self._keep.append((codes, scales))
+        self.linears = arr
+        self.outs = [torch.empty((M, layers[0][i][0].shape[0]), dtype=torch.float32, device=device)
+                     for i in range(STACK_LINEARS)]
+        self._outs_ptrs = (_vp * STACK_LINEARS)(*[t.data_ptr() for t in self.outs])
+        nbytes = int(_lib.nvq_decoder_stack_workspace_size(arr, M))
+        if nbytes == 0:
+            raise NVQError("nvq_decoder_stack_workspace_size", NVQ_ERR_BAD_SHAPE)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def forward(self, x: torch.Tensor, stream=None, n_layers: int | None = None):
+        n = self.n_layers if n_layers is None else n_layers
+        _check("nvq_decoder_stack", _lib.nvq_decoder_stack(
+            self.linears, n, _ptr(x), self.M, self._outs_ptrs, _ptr(self.workspace),
+            self.workspace.numel(), _stream(stream)))
+        return self.outs

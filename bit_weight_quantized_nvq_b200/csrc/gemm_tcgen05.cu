@@ -1,16 +1,506 @@
-// Prefill GEMM (tcgen05) - under construction.
+// Prefill GEMM on the 5th-generation tensor cores (tcgen05, TMEM, TMA):
+//   y[M, N] = A[M, K] . W[N, K]^T,  NVFP4 weights, Q8_0 activations.
+//
+// The tiled prefill kernels of "HANDOFF: flint CPU optimization (Q4_1 +
+// NVFP4)", section 3, unpack NVFP4 weight tiles and Q8_0 activation tiles
+// and accumulate per-16 scaled integer sums; the K5 runtime of "TKintegers
+// K5: 3.21x prefill and 3.10x decode throughput vs TorchAO FP8 on NVIDIA L4"
+// expands compact weight tiles to FP16 tensor-core operands with FP32
+// accumulation.  This kernel keeps the exact arithmetic of the first with
+// the operand expansion of the second:
+//
+//  * weights: w' = E2M1(code) * s_w is exact in fp16 (at most 6 significant
+//    bits, range 2^-10 .. 2688), so the per-16 rescale is folded into the
+//    operand, expanded in shared memory from the packed codes;
+//  * activations: a = d*q has at most 18 significant bits, so it is split
+//    into the exact fp16 pair hi = fp16(a), lo = fp16(a - hi) (hi + lo == a;
+//    lo is a multiple of the ulp of d and below half an ulp of hi);
+//  * every product w'*hi and w'*lo is exact in fp32; the tensor core sums
+//    them in fp32, and y = g * 0.5 * sum(c*s*d*q) = g * (acc_hi + acc_lo).
+//  * the tensor core's fp32 accumulation does not round to nearest (its
+//    error grows with the number of chained MMAs and is biased toward
+//    zero: about 1e-5 of sum|terms| after 1600 of them at K = 25600), so
+//    partial sums are promoted: each 512-wide K chunk accumulates in one of
+//    two TMEM buffers and the epilogue threads add it to fp32 registers
+//    (round to nearest) while the tensor core fills the other buffer.
+//
+// Kernels:
+//  1. expand_act_kernel: Q8_0 (q, d) -> fp16 [hi rows | lo rows] in the
+//     caller's workspace, once per call (tokens padded to 128 with zeros).
+//     A token whose largest |d*q| would overflow fp16 (|x| > 65504) is
+//     scaled by 2^-e first and the epilogue multiplies by 2^e.
+//  2. gemm_kernel: one CTA per 128 weight rows x 128 tokens, 6 warps:
+//       warp 0    TMA producer: [hi; lo] activation tiles (2 x 128 rows x 64
+//                 fp16, 128-byte swizzle) into a 4-stage ring;
+//       warp 1    allocates 512 TMEM columns (two 256-column accumulators);
+//                 one thread issues tcgen05.mma (M=128, N=256, K=16) x 4
+//                 per stage, commits each stage back to the producers and
+//                 each finished 8-stage chunk to the draining threads;
+//       warps 2-5 one thread per weight row: cp.async the row's 32 code
+//                 bytes and 4 scale bytes for each stage, decode 64 codes
+//                 to fp16 w' with byte permutes and write them in the
+//                 128-byte swizzle layout; drain finished chunks (tcgen05.ld
+//                 of the hi and lo columns into 128 fp32 registers); the
+//                 epilogue scales and stores the registers.
+//     Every wait is bounded (4 s); a timeout raises an error flag and the
+//     CTA drains what it issued, frees TMEM and exits.
+#include <algorithm>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+
+#include "nvq_device.cuh"
 #include "nvq_internal.h"
+#include "tcgen05.cuh"
 
 namespace nvq {
+namespace {
 
-size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
-  return static_cast<size_t>(M) * static_cast<size_t>(K) * 4u + 256u;
+constexpr int kBN = 128;            // weight rows per tile = MMA M = TMEM lanes
+constexpr int kBT = 128;            // tokens per tile; MMA N = 2 * kBT ([hi; lo])
+constexpr int kBK = 64;             // K per stage: one 128-byte fp16 swizzle row
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kChunk = 8;           // K stages accumulated per TMEM buffer
+constexpr uint32_t kAccCols = 2 * kBT;        // one [hi | lo] accumulator
+constexpr uint32_t kTmemCols = 2 * kAccCols;  // two accumulators
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+constexpr uint32_t kAStageBytes = kBN * kBK * 2;        // 16 KB of w'
+constexpr uint32_t kBStageBytes = 2 * kBT * kBK * 2;    // 32 KB of [hi; lo]
+constexpr uint32_t kCodeStageBytes = kBN * kBK / 2;     // 4 KB of codes
+constexpr uint32_t kScaleStageBytes = kBN * kBK / 16;   // 512 B of scales
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kOffA + kStages * kAStageBytes;
+constexpr uint32_t kOffCodes = kOffB + kStages * kBStageBytes;
+constexpr uint32_t kOffScales = kOffCodes + kStages * kCodeStageBytes;
+constexpr uint32_t kOffBars = kOffScales + kStages * kScaleStageBytes;
+constexpr uint32_t kNumBars = 3 * kStages + 5;   // + acc_full[2], acc_empty[2], mma_done
+constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + slack to align to 1024
+static_assert(kOffB % 1024 == 0 && kOffCodes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+
+// fp16 high bytes of the E2M1 values: 0, .5, 1, 1.5, 2, 3, 4, 6 are 0x0000,
+// 0x3800, 0x3C00, 0x3E00, 0x4000, 0x4200, 0x4400, 0x4600 (low bytes zero);
+// codes 8..15 carry the sign bit 0x80.
+constexpr uint32_t kHbPosLo = 0x3E3C3800u;
+constexpr uint32_t kHbPosHi = 0x46444240u;
+constexpr uint32_t kHbNegLo = 0xBEBCB880u;
+constexpr uint32_t kHbNegHi = 0xC6C4C2C0u;
+
+// bit 0: a pipeline wait of the GEMM timed out
+__device__ unsigned int g_gemm_error_flags = 0;
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) {
+  return *reinterpret_cast<__half2*>(&u);
 }
 
-cudaError_t launch_gemm(const uint8_t*, const uint8_t*, float, int64_t, int64_t,
-                        const int8_t*, const uint16_t*, int64_t, float*, void*,
-                        cudaStream_t) {
-  return cudaErrorNotSupported;
+// Eight codes (one word) -> eight fp16 w' = E2M1 * s, as one 16-byte chunk.
+__device__ __forceinline__ uint4 expand8(uint32_t w, __half2 s2) {
+  uint32_t lo, hi;
+  dev::lut16_x8<kHbPosLo, kHbPosHi, kHbNegLo, kHbNegHi>(w, lo, hi);
+  uint4 r;
+  r.x = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x1404)), s2));
+  r.y = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x3424)), s2));
+  r.z = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x1404)), s2));
+  r.w = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x3424)), s2));
+  return r;
+}
+
+__device__ __forceinline__ __half2 ue4m3x2_to_half2(uint32_t two_bytes) {
+  uint32_t h2;
+  const uint16_t in = static_cast<uint16_t>(two_bytes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return bits_h2(h2);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// 1. activation expansion
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+expand_act_kernel(const int8_t* __restrict__ q, const __half* __restrict__ d, int M, int K,
+                  int M_pad, __half* __restrict__ act, float* __restrict__ tok_scale) {
+  const int row = blockIdx.x;
+  uint4* hi = reinterpret_cast<uint4*>(act + static_cast<size_t>(row) * K);
+  uint4* lo = reinterpret_cast<uint4*>(act + static_cast<size_t>(M_pad + row) * K);
+  const int K8 = K / 8;
+  if (row >= M) {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < K8; i += blockDim.x) {
+      hi[i] = z;
+      lo[i] = z;
+    }
+    if (threadIdx.x == 0) tok_scale[row] = 1.0f;
+    return;
+  }
+  const __half* drow = d + static_cast<size_t>(row) * (K / 32);
+  float dmax = 0.0f;
+  for (int b = threadIdx.x; b < K / 32; b += blockDim.x)
+    dmax = fmaxf(dmax, fabsf(__half2float(drow[b])));
+  __shared__ float red[8];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dmax;
+  __syncthreads();
+  dmax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) dmax = fmaxf(dmax, red[i]);
+  // smallest e >= 0 with |d*q| * 2^-e <= 65504 for every element of the row
+  int e = 0;
+  while (ldexpf(dmax * 127.0f, -e) > 65504.0f) ++e;
+  const float inv = ldexpf(1.0f, -e);
+  if (threadIdx.x == 0) tok_scale[row] = ldexpf(1.0f, e);
+
+  const uint2* qrow = reinterpret_cast<const uint2*>(q + static_cast<size_t>(row) * K);
+  for (int i = threadIdx.x; i < K8; i += blockDim.x) {
+    const uint2 qv = qrow[i];
+    const float dv = __half2float(drow[i >> 2]) * inv;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t word = j < 2 ? qv.x : qv.y;
+      const int sh = (j & 1) * 16;
+      const float a0 = static_cast<float>(static_cast<int8_t>((word >> sh) & 0xFF)) * dv;
+      const float a1 = static_cast<float>(static_cast<int8_t>((word >> (sh + 8)) & 0xFF)) * dv;
+      const __half h0 = __float2half_rn(a0), h1 = __float2half_rn(a1);
+      const __half l0 = __float2half_rn(a0 - __half2float(h0));
+      const __half l1 = __float2half_rn(a1 - __half2float(h1));
+      hw[j] = h2_bits(__halves2half2(h0, h1));
+      lw[j] = h2_bits(__halves2half2(l0, l1));
+    }
+    hi[i] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    lo[i] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. the tcgen05 GEMM
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restrict__ codes,
+            const uint8_t* __restrict__ scales, int N, int K, int M, int M_pad, float g,
+            const float* __restrict__ tok_scale, float* __restrict__ y) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_addr(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  auto full_a = [&](int s) { return sbase + kOffBars + 8u * s; };
+  auto full_b = [&](int s) { return sbase + kOffBars + 8u * (kStages + s); };
+  auto empty = [&](int s) { return sbase + kOffBars + 8u * (2 * kStages + s); };
+  auto acc_full = [&](int b) { return sbase + kOffBars + 8u * (3 * kStages + b); };
+  auto acc_empty = [&](int b) { return sbase + kOffBars + 8u * (3 * kStages + 2 + b); };
+  const uint32_t mma_done = sbase + kOffBars + 8u * (3 * kStages + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBN;
+  const int m0 = blockIdx.y * kBT;
+  const int num_kb = K / kBK;
+  const int num_chunks = (num_kb + kChunk - 1) / kChunk;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(full_a(s), kBN);
+      ptx::mbar_init(full_b(s), 1);
+      ptx::mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(acc_full(b), 1);
+      ptx::mbar_init(acc_empty(b), kBN);
+    }
+    ptx::mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tensormap(&act_map);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicOr(&g_gemm_error_flags, 1u);
+  };
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!ptx::mbar_wait_bounded(empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+          fail();
+          break;
+        }
+        const uint32_t dst = sbase + kOffB + s * kBStageBytes;
+        ptx::mbar_arrive_expect_tx(full_b(s), kBStageBytes);
+        ptx::tma_load_2d(dst, &act_map, kb * kBK, m0, full_b(s));
+        ptx::tma_load_2d(dst + kBStageBytes / 2, &act_map, kb * kBK, M_pad + m0, full_b(s));
+        ++issued;
+      }
+      if (*abort_flag) {
+        for (int kb = std::max(0, issued - kStages); kb < issued; ++kb)
+          ptx::mbar_wait_bounded(full_b(kb % kStages), (kb / kStages) & 1, nullptr, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer --------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_f16_f32(kBN, 2 * kBT);
+      bool ok = true;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        const int c = kb / kChunk;
+        const int b = c & 1;
+        const bool first = (kb % kChunk) == 0;
+        // a buffer is reused two chunks later, once the epilogue drained it
+        if (first && c >= 2 &&
+            !ptx::mbar_wait_bounded(acc_empty(b), ((c >> 1) - 1) & 1, abort_flag, kWaitLimitNs)) {
+          fail();
+          ok = false;
+          break;
+        }
+        if (!ptx::mbar_wait_bounded(full_a(s), ph, abort_flag, kWaitLimitNs) ||
+            !ptx::mbar_wait_bounded(full_b(s), ph, abort_flag, kWaitLimitNs)) {
+          fail();
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a0 = sbase + kOffA + s * kAStageBytes;
+        const uint32_t b0 = sbase + kOffB + s * kBStageBytes;
+        const uint32_t d_tmem = tmem_base + b * kAccCols;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          ptx::mma_f16(d_tmem, ptx::sw128_kmajor_desc(a0 + 32u * k),
+                       ptx::sw128_kmajor_desc(b0 + 32u * k), idesc, !(first && k == 0));
+        }
+        ptx::mma_commit(empty(s));
+        if ((kb % kChunk) == kChunk - 1 || kb == num_kb - 1) ptx::mma_commit(acc_full(b));
+      }
+      (void)ok;
+      // no MMA may still be writing TMEM when it is released
+      ptx::mma_commit(mma_done);
+      ptx::mbar_wait_bounded(mma_done, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    // ------------------- weight expansion, then the epilogue ------------------
+    const int t = threadIdx.x - 64;   // 0..127: row of the tile
+    const int row = n0 + t;
+    const bool valid = row < N;
+    const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2);
+    const uint8_t* srow = scales + static_cast<size_t>(valid ? row : 0) * (K / 16);
+    const uint32_t stg_c = sbase + kOffCodes + 32u * t;
+    const uint32_t stg_s = sbase + kOffScales + 4u * t;
+    auto issue = [&](int kb) {
+      if (kb < num_kb) {
+        const uint32_t slot = kb % kStages;
+        const uint32_t nb = valid ? 16u : 0u;
+        ptx::cp_async_16(stg_c + slot * kCodeStageBytes, crow + 32 * kb, nb);
+        ptx::cp_async_16(stg_c + slot * kCodeStageBytes + 16, crow + 32 * kb + 16, nb);
+        ptx::cp_async_4(stg_s + slot * kScaleStageBytes, srow + 4 * kb, valid ? 4u : 0u);
+      }
+      ptx::cp_async_commit();
+    };
+    for (int i = 0; i < kStages - 1; ++i) issue(i);
+    bool ok = true;
+    const uint32_t sw = t & 7;
+    const int quarter = warp & 3;            // TMEM lanes this warp may read
+    const uint32_t tlane = static_cast<uint32_t>(quarter * 32) << 16;
+    float run[kBT];
+#pragma unroll
+    for (int j = 0; j < kBT; ++j) run[j] = 0.0f;
+    int drained = 0;
+    // add finished chunk c (both halves) to the fp32 registers and hand its
+    // buffer back to the tensor core
+    auto drain = [&](int c) -> bool {
+      const int b = c & 1;
+      if (!ptx::mbar_wait_bounded(acc_full(b), (c >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
+      ptx::tc_fence_after();
+      const uint32_t base = tmem_base + tlane + b * kAccCols;
+#pragma unroll
+      for (int cc = 0; cc < 2 * kBT / 32; ++cc) {
+        uint32_t v[32];
+        ptx::tmem_ld_32cols(base + 32u * cc, v);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) run[(cc * 32 + j) % kBT] += __uint_as_float(v[j]);
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(acc_empty(b));
+      return true;
+    };
+    for (int kb = 0; kb < num_kb; ++kb) {
+      if ((kb % kChunk) == 0 && kb / kChunk >= 2) {
+        if (!drain(drained++)) {
+          fail();
+          ok = false;
+          break;
+        }
+      }
+      ptx::cp_async_wait<kStages - 2>();
+      const int s = kb % kStages;
+      const uint32_t ph = (kb / kStages) & 1;
+      if (!ptx::mbar_wait_bounded(empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+        fail();
+        ok = false;
+        break;
+      }
+      const uint8_t* cs = smem + kOffCodes + s * kCodeStageBytes + 32 * t;
+      const uint4 c0 = *reinterpret_cast<const uint4*>(cs);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(cs + 16);
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(smem + kOffScales + s * kScaleStageBytes + 4 * t);
+      const __half2 s01 = ue4m3x2_to_half2(sc & 0xFFFFu);
+      const __half2 s23 = ue4m3x2_to_half2(sc >> 16);
+      const __half2 sb0 = __low2half2(s01), sb1 = __high2half2(s01);
+      const __half2 sb2 = __low2half2(s23), sb3 = __high2half2(s23);
+      const uint32_t arow = sbase + kOffA + s * kAStageBytes + 128u * t;
+      st_shared_v4(arow + ((0u ^ sw) << 4), expand8(c0.x, sb0));
+      st_shared_v4(arow + ((1u ^ sw) << 4), expand8(c0.y, sb0));
+      st_shared_v4(arow + ((2u ^ sw) << 4), expand8(c0.z, sb1));
+      st_shared_v4(arow + ((3u ^ sw) << 4), expand8(c0.w, sb1));
+      st_shared_v4(arow + ((4u ^ sw) << 4), expand8(c1.x, sb2));
+      st_shared_v4(arow + ((5u ^ sw) << 4), expand8(c1.y, sb2));
+      st_shared_v4(arow + ((6u ^ sw) << 4), expand8(c1.z, sb3));
+      st_shared_v4(arow + ((7u ^ sw) << 4), expand8(c1.w, sb3));
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(full_a(s));
+      issue(kb + kStages - 1);
+    }
+    ptx::cp_async_wait<0>();
+    while (ok && drained < num_chunks) {
+      if (!drain(drained++)) {
+        fail();
+        ok = false;
+      }
+    }
+    if (ok) {
+      const int nrow = n0 + quarter * 32 + lane;
+      if (nrow < N) {
+#pragma unroll
+        for (int j = 0; j < kBT; ++j) {
+          const int m = m0 + j;
+          if (m < M) y[static_cast<size_t>(m) * N + nrow] = run[j] * (g * tok_scale[m]);
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int64_t padded_tokens(int64_t M) { return (M + kBT - 1) / kBT * kBT; }
+
+}  // namespace
+
+size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
+  const int64_t mp = padded_tokens(M);
+  return static_cast<size_t>(4 * mp * K + 4 * mp);
+}
+
+unsigned int gemm_error_flags(bool clear) {
+  unsigned int v = 0;
+  cudaMemcpyFromSymbol(&v, g_gemm_error_flags, sizeof(v));
+  if (clear) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_gemm_error_flags, &zero, sizeof(zero));
+  }
+  return v;
+}
+
+cudaError_t gemm_expand(const int8_t* q, const uint16_t* d, int64_t M, int64_t K,
+                        void* workspace, cudaStream_t stream) {
+  const int64_t M_pad = padded_tokens(M);
+  __half* act = static_cast<__half*>(workspace);
+  float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 4 * M_pad * K);
+  expand_act_kernel<<<static_cast<unsigned>(M_pad), 256, 0, stream>>>(
+      q, reinterpret_cast<const __half*>(d), static_cast<int>(M), static_cast<int>(K),
+      static_cast<int>(M_pad), act, tok_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                      int64_t K, int64_t M, float* y, const void* workspace,
+                      cudaStream_t stream) {
+  const int64_t M_pad = padded_tokens(M);
+  void* act = const_cast<void*>(workspace);
+  const float* tok_scale =
+      reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + 4 * M_pad * K);
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(2 * M_pad)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBT)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN), static_cast<unsigned>(M_pad / kBT));
+  gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, codes, scales, static_cast<int>(N),
+                                                      static_cast<int>(K), static_cast<int>(M),
+                                                      static_cast<int>(M_pad), g, tok_scale, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                        int64_t K, const int8_t* q, const uint16_t* d, int64_t M, float* y,
+                        void* workspace, cudaStream_t stream) {
+  cudaError_t e = gemm_expand(q, d, M, K, workspace, stream);
+  if (e != cudaSuccess) return e;
+  return gemm_main(codes, scales, g, N, K, M, y, workspace, stream);
 }
 
 }  // namespace nvq

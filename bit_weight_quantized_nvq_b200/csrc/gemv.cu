@@ -22,16 +22,191 @@
 //    multiplied by the chunk's d and accumulated in fp32; the activation
 //    block is read through L1 (it is shared by every row on the SM);
 //  * one shuffle reduction per row, then y = 0.5*g*acc.
+//
+// Two schedules share that arithmetic:
+//  * gemv_tma_kernel (K % 256 == 0, every workload shape): persistent CTAs,
+//    one per half SM, each owning a contiguous, balanced range of rows.  A
+//    producer warp streams groups of 8 rows (the whole K, or a K segment of
+//    at most 5120 elements) into a 4-stage shared-memory ring with 1-D TMA
+//    bulk copies; 8 consumer warps each own one row of the group and decode
+//    from shared memory.  Memory-level parallelism comes from the ring (up
+//    to ~90 KB in flight per CTA), not from registers.
+//  * gemv_kernel (any K % 64 == 0): one warp per row, loads straight to
+//    registers.
+#include <algorithm>
+
 #include <cuda_fp16.h>
 
 #include "nvq_device.cuh"
 #include "nvq_internal.h"
+#include "tcgen05.cuh"
 
 namespace nvq {
 namespace {
 
 constexpr int kWarps = 4;        // rows per CTA
 constexpr int kUnroll = 4;       // chunks per lane in flight
+
+// TMA-staged schedule
+constexpr int kTmaConsumers = 8;                  // consumer warps = rows per group
+constexpr int kTmaStages = 4;
+constexpr int kTmaThreads = (kTmaConsumers + 1) * 32;
+constexpr int kTmaMaxSeg = 5120;                  // K elements per stage and row
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per pipeline wait
+
+// bit 0: a pipeline wait of the GEMV timed out
+__device__ unsigned int g_gemv_error_flags = 0;
+
+__device__ __forceinline__ float gemv_chunk_dot(const uint4 w, uint32_t s2, const int8_t* q,
+                                                const __half* d, int c) {
+  uint32_t cw[8];
+  dev::decode_e2m1x8(w.x, cw[0], cw[1]);
+  dev::decode_e2m1x8(w.y, cw[2], cw[3]);
+  dev::decode_e2m1x8(w.z, cw[4], cw[5]);
+  dev::decode_e2m1x8(w.w, cw[6], cw[7]);
+  const float2 s = dev::ue4m3x2_to_float2(s2);
+  const uint4* qa = reinterpret_cast<const uint4*>(q) + 2 * c;
+  const uint4 q0 = __ldg(qa);
+  const uint4 q1 = __ldg(qa + 1);
+  const float dm = __half2float(__ldg(d + c));
+  const int i0 = dev::dp4a(cw[0], q0.x, dev::dp4a(cw[1], q0.y,
+                 dev::dp4a(cw[2], q0.z, dev::dp4a(cw[3], q0.w, 0))));
+  const int i1 = dev::dp4a(cw[4], q1.x, dev::dp4a(cw[5], q1.y,
+                 dev::dp4a(cw[6], q1.z, dev::dp4a(cw[7], q1.w, 0))));
+  return dm * fmaf(s.x, static_cast<float>(i0), s.y * static_cast<float>(i1));
+}
+
+// Shared memory of the TMA schedule: kTmaStages stages of
+// [8 rows x seg/2 code bytes][8 rows x seg/16 scale bytes], then the
+// full/empty barriers and the abort flag.
+__host__ __device__ constexpr uint32_t tma_stage_bytes(int seg) {
+  return static_cast<uint32_t>(kTmaConsumers) * (seg / 2 + seg / 16);
+}
+__host__ __device__ constexpr uint32_t tma_smem_bytes(int seg) {
+  return kTmaStages * tma_stage_bytes(seg) + 2 * kTmaStages * 8 + 16;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kTmaThreads, 2)
+gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                float half_g, int N, int K, int seg, const int8_t* __restrict__ q,
+                const __half* __restrict__ d, float* __restrict__ y) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t stage_bytes = tma_stage_bytes(seg);
+  const uint32_t codes_bytes = kTmaConsumers * (seg / 2);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTmaStages * stage_bytes);
+  uint64_t* empty = full + kTmaStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kTmaStages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
+  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
+  const int ngroups = (r_end - r_begin + kTmaConsumers - 1) / kTmaConsumers;
+  const int nseg = K / seg;
+  const int total = ngroups * nseg;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTmaStages; ++i) {
+      ptx::mbar_init(ptx::smem_addr(full + i), 1);
+      ptx::mbar_init(ptx::smem_addr(empty + i), kTmaConsumers);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kTmaConsumers) {
+    // ---------------- producer: one thread issues the bulk copies ----------
+    if (lane != 0) return;
+    int issued = 0;
+    for (int it = 0; it < total; ++it) {
+      const int s = it % kTmaStages;
+      const uint32_t ph = (it / kTmaStages) & 1;
+      if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        atomicOr(&g_gemv_error_flags, 1u);
+        break;
+      }
+      const int grp = it / nseg, sg = it % nseg;
+      const int row0 = r_begin + grp * kTmaConsumers;
+      const int nrows = min(kTmaConsumers, r_end - row0);
+      const uint32_t bar = ptx::smem_addr(full + s);
+      uint8_t* st = smem + s * stage_bytes;
+      ptx::mbar_arrive_expect_tx(bar, nrows * (seg / 2 + seg / 16));
+      if (nseg == 1) {
+        ptx::bulk_load(ptx::smem_addr(st), codes + static_cast<size_t>(row0) * (K / 2),
+                       nrows * (K / 2), bar);
+        ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
+                       scales + static_cast<size_t>(row0) * (K / 16), nrows * (K / 16), bar);
+      } else {
+        for (int r = 0; r < nrows; ++r) {
+          ptx::bulk_load(ptx::smem_addr(st + r * (seg / 2)),
+                         codes + static_cast<size_t>(row0 + r) * (K / 2) + sg * (seg / 2),
+                         seg / 2, bar);
+          ptx::bulk_load(ptx::smem_addr(st + codes_bytes + r * (seg / 16)),
+                         scales + static_cast<size_t>(row0 + r) * (K / 16) + sg * (seg / 16),
+                         seg / 16, bar);
+        }
+      }
+      ++issued;
+    }
+    if (*abort_flag) {
+      // let the copies already in flight land before the CTA exits
+      for (int it = max(0, issued - kTmaStages); it < issued; ++it)
+        ptx::mbar_wait_bounded(ptx::smem_addr(full + it % kTmaStages),
+                               (it / kTmaStages) & 1, nullptr, kWaitLimitNs);
+    }
+    return;
+  }
+
+  // ---------------- consumers: warp w owns row w of each group ------------
+  float acc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+  const int nch = seg / 32;
+  for (int it = 0; it < total; ++it) {
+    const int s = it % kTmaStages;
+    const uint32_t ph = (it / kTmaStages) & 1;
+    if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
+      *abort_flag = 1;
+      atomicOr(&g_gemv_error_flags, 1u);
+      break;
+    }
+    const int grp = it / nseg, sg = it % nseg;
+    const int row0 = r_begin + grp * kTmaConsumers;
+    const int nrows = min(kTmaConsumers, r_end - row0);
+    if (warp < nrows) {
+      const uint8_t* st = smem + s * stage_bytes;
+      const uint4* sc = reinterpret_cast<const uint4*>(st + warp * (seg / 2));
+      const uint16_t* ss = reinterpret_cast<const uint16_t*>(st + codes_bytes + warp * (seg / 16));
+      const int cbase = sg * nch;
+#pragma unroll 4
+      for (int j = lane; j < nch; j += 32) {
+        const uint4 w = sc[j];
+        const uint32_t s2 = ss[j];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          acc[m] += gemv_chunk_dot(w, s2, q + static_cast<size_t>(m) * K,
+                                   d + static_cast<size_t>(m) * (K >> 5), cbase + j);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(empty + s));
+    if (sg == nseg - 1) {
+      if (warp < nrows) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float v = dev::warp_sum(acc[m]);
+          if (lane == 0) y[static_cast<size_t>(m) * N + row0 + warp] = v * half_g;
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
+    }
+  }
+}
 
 template <int MT>
 __global__ void __launch_bounds__(kWarps * 32)
@@ -124,10 +299,39 @@ subblock_sums_kernel(const uint8_t* __restrict__ codes, int N, int K,
   }
 }
 
+// K elements per TMA stage and row: the largest multiple of 256 that divides
+// K and is at most kTmaMaxSeg; 0 when K is not a multiple of 256 (scale rows
+// would not be 16-byte aligned for the bulk copies).
+int tma_segment(int64_t K) {
+  if (K % 256 != 0) return 0;
+  for (int64_t seg = (kTmaMaxSeg / 256) * 256; seg >= 256; seg -= 256)
+    if (K % seg == 0) return static_cast<int>(seg);
+  return 0;
+}
+
 template <int MT>
 cudaError_t launch_gemv_m(const uint8_t* codes, const uint8_t* scales, float g,
                           int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
                           float* y, cudaStream_t stream) {
+  const int seg = tma_segment(K);
+  if (seg > 0) {
+    const uint32_t smem = tma_smem_bytes(seg);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(gemv_tma_kernel<MT>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(tma_smem_bytes(kTmaMaxSeg)));
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    const int64_t ctas = std::min<int64_t>(2 * static_cast<int64_t>(device_sm_count()), N);
+    gemv_tma_kernel<MT><<<static_cast<unsigned>(ctas), kTmaThreads, smem, stream>>>(
+        codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), seg, q,
+        reinterpret_cast<const __half*>(d), y);
+    return cudaGetLastError();
+  }
   const unsigned grid = static_cast<unsigned>((N + kWarps - 1) / kWarps);
   gemv_kernel<MT><<<grid, kWarps * 32, 0, stream>>>(
       codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), q,
@@ -150,6 +354,16 @@ cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
 #undef NVQ_GEMV_CASE
     default: return cudaErrorInvalidValue;
   }
+}
+
+unsigned int gemv_error_flags(bool clear) {
+  unsigned int v = 0;
+  cudaMemcpyFromSymbol(&v, g_gemv_error_flags, sizeof(v));
+  if (clear) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_gemv_error_flags, &zero, sizeof(zero));
+  }
+  return v;
 }
 
 cudaError_t launch_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,

@@ -81,6 +81,8 @@ nvq_status check_dot_args(const void* codes, const void* scales, int64_t N,
 }  // namespace
 
 namespace nvq {
+void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = e; }
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;

@@ -19,24 +19,30 @@ constexpr uint32_t kLutPosHi = 0x0C080604u;  // codes 4..7   ->  4,  6,  8, 12
 constexpr uint32_t kLutNegLo = 0xFDFEFF00u;  // codes 8..11  ->  0, -1, -2, -3
 constexpr uint32_t kLutNegHi = 0xF4F8FAFCu;  // codes 12..15 -> -4, -6, -8,-12
 
-// Decode the eight E2M1 codes of one 32-bit word (nibble i = element i) into
-// two words of four signed bytes c = 2*E2M1: `lo` holds elements 0..3 and
-// `hi` elements 4..7.  Each byte is looked up twice with a byte permute
-// (positive and negative halves of the table, indexed by the code's low
-// three bits) and the sign bit picks between the two.
-__device__ __forceinline__ void decode_e2m1x8(uint32_t w, uint32_t& lo,
-                                              uint32_t& hi) {
+// Look up the eight 4-bit codes of one 32-bit word (nibble i = element i)
+// in a 16-entry byte table given as four packed words (entries 0-3, 4-7,
+// 8-11, 12-15).  `lo` receives the bytes of elements 0..3, `hi` those of
+// elements 4..7.  Each byte is looked up twice with a byte permute (in the
+// table half of codes 0-7 and of codes 8-15, indexed by the code's low three
+// bits) and bit 3 of the code picks between the two.
+template <uint32_t T0, uint32_t T1, uint32_t T2, uint32_t T3>
+__device__ __forceinline__ void lut16_x8(uint32_t w, uint32_t& lo, uint32_t& hi) {
   const uint32_t idx = w & 0x77777777u;
   // selector of the final permute: byte i from p (i) or from n (4 + i)
   const uint32_t pick = ((w >> 1) & 0x44444444u) | 0x32103210u;
   const uint32_t idx_hi = idx >> 16;
   const uint32_t pick_hi = pick >> 16;
-  const uint32_t p0 = __byte_perm(kLutPosLo, kLutPosHi, idx);
-  const uint32_t n0 = __byte_perm(kLutNegLo, kLutNegHi, idx);
-  const uint32_t p1 = __byte_perm(kLutPosLo, kLutPosHi, idx_hi);
-  const uint32_t n1 = __byte_perm(kLutNegLo, kLutNegHi, idx_hi);
+  const uint32_t p0 = __byte_perm(T0, T1, idx);
+  const uint32_t n0 = __byte_perm(T2, T3, idx);
+  const uint32_t p1 = __byte_perm(T0, T1, idx_hi);
+  const uint32_t n1 = __byte_perm(T2, T3, idx_hi);
   lo = __byte_perm(p0, n0, pick);
   hi = __byte_perm(p1, n1, pick_hi);
+}
+
+// Decode eight E2M1 codes to signed bytes c = 2*E2M1.
+__device__ __forceinline__ void decode_e2m1x8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lut16_x8<kLutPosLo, kLutPosHi, kLutNegLo, kLutNegHi>(w, lo, hi);
 }
 
 // Two UE4M3 scale bytes (low byte = first subblock) to fp32, exactly.  UE4M3

@@ -19,6 +19,10 @@ cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                         const uint16_t* d, int64_t M, float* y,
                         cudaStream_t stream);
 
+// Error flags raised by GEMV kernels (bit 0: a pipeline wait timed out);
+// synchronous read, optionally clearing them.
+unsigned int gemv_error_flags(bool clear);
+
 // Integer per-16 subblock sums through the GEMV's decode/dot code.
 cudaError_t launch_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
                                  const int8_t* q, int64_t M, int32_t* isum,
@@ -30,6 +34,20 @@ cudaError_t launch_gemm(const uint8_t* codes, const uint8_t* scales, float g,
                         int64_t N, int64_t K, const int8_t* q,
                         const uint16_t* d, int64_t M, float* y,
                         void* workspace, cudaStream_t stream);
+// The two halves of launch_gemm: expand Q8_0 activations into the
+// workspace, then run the tensor-core GEMM on an expanded workspace (which
+// several weight matrices with the same K may share).
+cudaError_t gemm_expand(const int8_t* q, const uint16_t* d, int64_t M, int64_t K,
+                        void* workspace, cudaStream_t stream);
+cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                      int64_t K, int64_t M, float* y, const void* workspace,
+                      cudaStream_t stream);
+
+// Error flags raised by the GEMM kernel (bit 0: a pipeline wait timed out).
+unsigned int gemm_error_flags(bool clear);
+
+// Record the CUDA error reported by nvq_last_cuda_error() on this thread.
+void set_last_cuda_error(cudaError_t e);
 
 // Number of streaming multiprocessors of the current device (cached).
 int device_sm_count();

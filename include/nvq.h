@@ -171,6 +171,53 @@ nvq_status nvq_debug_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
                                    const int8_t* q, int64_t M, int32_t* isum,
                                    void* stream);
 
+/* One NVFP4 weight matrix W[N, K] in device memory (caller-owned). */
+typedef struct nvq_linear {
+  const uint8_t* codes;   /* device uint8 [N, K/2]  */
+  const uint8_t* scales;  /* device uint8 [N, K/16] */
+  float g;                /* per-tensor scale       */
+  int64_t N;
+  int64_t K;
+} nvq_linear;
+
+/* Linears per decoder layer, in execution order. */
+#define NVQ_STACK_LINEARS 7
+
+/*
+ * nvq_decoder_stack - every linear layer of a dense decoder stack, layer
+ * after layer, on one stream, for M tokens: the decode pass (M <= 16, the
+ * GEMV) or the prefill pass (M > 16, the tensor-core GEMM).
+ *
+ * Each layer holds NVQ_STACK_LINEARS matrices in the order q, k, v, o, up,
+ * gate, down (linears[7*l + i]), and runs
+ *     (q_a, d_a) = Q8_0(x);          y_q, y_k, y_v = W_q a, W_k a, W_v a
+ *     (q_a, d_a) = Q8_0(y_v);        y_o = W_o a
+ *     (q_a, d_a) = Q8_0(y_o);        y_up, y_gate = W_up a, W_gate a
+ *     (q_a, d_a) = Q8_0(y_up);       y_down = W_down a
+ * i.e. 7 products and 4 activation quantisations per layer.  Every layer
+ * starts again from the same input x: only the linear layers are modelled
+ * (no attention, norms or activation functions), so the chain stays in
+ * range over any depth.  Shapes: q, k, v have K = hidden (x is [M, hidden]);
+ * o.K = v.N; up.K = gate.K = o.N; down.K = up.N; every layer has the shapes
+ * of layer 0.
+ *
+ * linears   host array of 7 * n_layers descriptors (read during the call).
+ * x         device float [M, hidden].
+ * outs      host array of 7 device float pointers, outs[i] of [M, N_i];
+ *           overwritten by every layer, so they hold the last layer's outputs.
+ * workspace device scratch of nvq_decoder_stack_workspace_size(linears, M)
+ *           bytes (Q8_0 activations, and the fp16 expansion when M > 16).
+ * Errors: as nvq_gemv / nvq_gemm, NVQ_ERR_BAD_SHAPE when the shapes do not
+ * chain, NVQ_ERR_WORKSPACE.  Launch errors stop the pass at that point.
+ */
+nvq_status nvq_decoder_stack(const nvq_linear* linears, int64_t n_layers,
+                             const float* x, int64_t M, float* const* outs,
+                             void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Workspace bytes nvq_decoder_stack needs for M tokens (0 on bad input). */
+size_t nvq_decoder_stack_workspace_size(const nvq_linear* linears, int64_t M);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -25,8 +25,13 @@ def run_gemv(P, q, d, M):
     return y.cpu().numpy()
 
 
+# (1001, 1088), (37, 64), (1, 4160): K % 256 != 0, the register schedule.
+# (1001, 1280): the TMA schedule, one K segment, ragged row groups.
+# (37, 12800): the TMA schedule with five K segments of 2560 per row.
+# (300, 25600): the decode K with few rows (one or two rows per CTA).
 @pytest.mark.parametrize("M", list(range(1, 17)))
-@pytest.mark.parametrize("N,K", [(1001, 1088), (37, 64), (1, 4096 + 64)])
+@pytest.mark.parametrize("N,K", [(1001, 1088), (37, 64), (1, 4096 + 64),
+                                 (1001, 1280), (37, 12800), (300, 25600)])
 def test_small_shapes_all_rows(M, N, K):
     W = wl.weights("gemv_test", "W", N, K, boost_columns=True)
     x = wl.activations("gemv_test", "x", M, K, "student_t4")
