@@ -23,7 +23,20 @@
 //    block is read through L1 (it is shared by every row on the SM);
 //  * one shuffle reduction per row, then y = 0.5*g*acc.
 //
-// Two schedules share that arithmetic:
+// Three schedules share that arithmetic:
+//  * gemv_m1_kernel (M = 1, K % 256 == 0; the decode path): one CTA per SM
+//    owning a balanced row range; a producer warp streams groups of 16
+//    contiguous rows (whole K, or K segments of at most 5120) into a
+//    4-stage ring of ~46 KB stages with 1-D TMA bulk copies; 16 consumer
+//    warps own one row each.  The activation block of every chunk is staged
+//    once per CTA in shared memory as conflict-free 16-byte vectors (two
+//    halves of the 32 codes, and {d, corr0, corr1}); the weights are decoded
+//    to the +12-biased integer LUT of the "Bias trick" paragraph (9
+//    operations per 8 codes instead of 11) and the bias is removed by
+//    starting each subblock's dp4a chain at corr = -12 * bsum16, precomputed
+//    per activation subblock.  The chunk loop is fully unrolled for 4 or 5
+//    chunks per lane so all shared-memory loads of a stage are in flight
+//    together.  The consumers are instruction-bound, so these savings matter.
 //  * gemv_tma_kernel (K % 256 == 0, every workload shape): persistent CTAs,
 //    one per half SM, each owning a contiguous, balanced range of rows.  A
 //    producer warp streams groups of 8 rows (the whole K, or a K segment of
@@ -84,6 +97,192 @@ __host__ __device__ constexpr uint32_t tma_stage_bytes(int seg) {
 }
 __host__ __device__ constexpr uint32_t tma_smem_bytes(int seg) {
   return kTmaStages * tma_stage_bytes(seg) + 2 * kTmaStages * 8 + 16;
+}
+
+// ---------------------------------------------------------------------------
+// M = 1 schedule
+// ---------------------------------------------------------------------------
+constexpr int kM1Consumers = 16;                       // rows per group
+constexpr int kM1Threads = (kM1Consumers + 1) * 32;    // + producer warp
+constexpr int kM1Stages = 4;
+constexpr uint32_t kSmemPerCtaMax = 227 * 1024;
+
+// per 32-element activation chunk: its fp32 scale and the bias corrections
+// -12 * (sum of its 16 codes) of its two subblocks
+struct __align__(16) ActMeta {
+  float d;
+  int corr0;
+  int corr1;
+  int pad;
+};
+
+__host__ __device__ constexpr uint32_t m1_stage_bytes(int seg) {
+  return static_cast<uint32_t>(kM1Consumers) * (seg / 2 + seg / 16);
+}
+// stages | qa [K/32 x 16 B] | qb [K/32 x 16 B] | meta [K/32 x 16 B] | barriers
+__host__ __device__ constexpr uint32_t m1_smem_bytes(int K, int seg) {
+  return kM1Stages * m1_stage_bytes(seg) + static_cast<uint32_t>(K / 32) * 48 +
+         2 * kM1Stages * 8 + 16;
+}
+
+template <int NPL>   // chunks per lane per stage (seg / 1024); 0 = any seg
+__global__ void __launch_bounds__(kM1Threads, 1)
+gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+               float half_g, int N, int K, int seg, const int8_t* __restrict__ q,
+               const __half* __restrict__ d, float* __restrict__ y) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t stage_bytes = m1_stage_bytes(seg);
+  const uint32_t codes_bytes = kM1Consumers * (seg / 2);
+  const int nchunk = K / 32;
+  uint4* qa = reinterpret_cast<uint4*>(smem + kM1Stages * stage_bytes);
+  uint4* qb = qa + nchunk;
+  ActMeta* meta = reinterpret_cast<ActMeta*>(qb + nchunk);
+  uint64_t* full = reinterpret_cast<uint64_t*>(meta + nchunk);
+  uint64_t* empty = full + kM1Stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kM1Stages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
+  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
+  const int ngroups = (r_end - r_begin + kM1Consumers - 1) / kM1Consumers;
+  const int nseg = K / seg;
+  const int total = ngroups * nseg;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kM1Stages; ++i) {
+      ptx::mbar_init(ptx::smem_addr(full + i), 1);
+      ptx::mbar_init(ptx::smem_addr(empty + i), kM1Consumers);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  // stage the activation vector once per CTA
+  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
+    const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * c;
+    const uint4 a = src[0], b = src[1];
+    qa[c] = a;
+    qb[c] = b;
+    const int s0 = dev::dp4a(a.x, 0x01010101u, dev::dp4a(a.y, 0x01010101u,
+                   dev::dp4a(a.z, 0x01010101u, dev::dp4a(a.w, 0x01010101u, 0))));
+    const int s1 = dev::dp4a(b.x, 0x01010101u, dev::dp4a(b.y, 0x01010101u,
+                   dev::dp4a(b.z, 0x01010101u, dev::dp4a(b.w, 0x01010101u, 0))));
+    ActMeta mt;
+    mt.d = __half2float(d[c]);
+    mt.corr0 = -12 * s0;
+    mt.corr1 = -12 * s1;
+    mt.pad = 0;
+    meta[c] = mt;
+  }
+  __syncthreads();
+
+  if (warp == kM1Consumers) {
+    // ---------------- producer: one thread issues the bulk copies ----------
+    if (lane != 0) return;
+    int issued = 0;
+    for (int it = 0; it < total; ++it) {
+      const int s = it % kM1Stages;
+      const uint32_t ph = (it / kM1Stages) & 1;
+      if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        atomicOr(&g_gemv_error_flags, 1u);
+        break;
+      }
+      const int grp = it / nseg, sg = it % nseg;
+      const int row0 = r_begin + grp * kM1Consumers;
+      const int nrows = min(kM1Consumers, r_end - row0);
+      const uint32_t bar = ptx::smem_addr(full + s);
+      uint8_t* st = smem + s * stage_bytes;
+      ptx::mbar_arrive_expect_tx(bar, nrows * (seg / 2 + seg / 16));
+      if (nseg == 1) {
+        ptx::bulk_load(ptx::smem_addr(st), codes + static_cast<size_t>(row0) * (K / 2),
+                       nrows * (K / 2), bar);
+        ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
+                       scales + static_cast<size_t>(row0) * (K / 16), nrows * (K / 16), bar);
+      } else {
+        for (int r = 0; r < nrows; ++r) {
+          ptx::bulk_load(ptx::smem_addr(st + r * (seg / 2)),
+                         codes + static_cast<size_t>(row0 + r) * (K / 2) + sg * (seg / 2),
+                         seg / 2, bar);
+          ptx::bulk_load(ptx::smem_addr(st + codes_bytes + r * (seg / 16)),
+                         scales + static_cast<size_t>(row0 + r) * (K / 16) + sg * (seg / 16),
+                         seg / 16, bar);
+        }
+      }
+      ++issued;
+    }
+    if (*abort_flag) {
+      for (int it = max(0, issued - kM1Stages); it < issued; ++it)
+        ptx::mbar_wait_bounded(ptx::smem_addr(full + it % kM1Stages), (it / kM1Stages) & 1,
+                               nullptr, kWaitLimitNs);
+    }
+    return;
+  }
+
+  // ---------------- consumers: warp w owns row w of each group --------------
+  float acc = 0.0f;
+  const int nch = seg / 32;
+  for (int it = 0; it < total; ++it) {
+    const int s = it % kM1Stages;
+    const uint32_t ph = (it / kM1Stages) & 1;
+    if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
+      *abort_flag = 1;
+      atomicOr(&g_gemv_error_flags, 1u);
+      break;
+    }
+    const int grp = it / nseg, sg = it % nseg;
+    const int row0 = r_begin + grp * kM1Consumers;
+    const int nrows = min(kM1Consumers, r_end - row0);
+    if (warp < nrows) {
+      const uint8_t* st = smem + s * stage_bytes;
+      const uint4* cw = reinterpret_cast<const uint4*>(st + warp * (seg / 2));
+      const uint16_t* sw = reinterpret_cast<const uint16_t*>(st + codes_bytes + warp * (seg / 16));
+      const int cbase = sg * nch;
+      auto chunk = [&](const uint4 w, uint32_t s2, const uint4 a, const uint4 b, const ActMeta mt) {
+        uint32_t c[8];
+        dev::decode_e2m1x8_biased(w.x, c[0], c[1]);
+        dev::decode_e2m1x8_biased(w.y, c[2], c[3]);
+        dev::decode_e2m1x8_biased(w.z, c[4], c[5]);
+        dev::decode_e2m1x8_biased(w.w, c[6], c[7]);
+        const int i0 = dev::dp4a_us(c[0], a.x, dev::dp4a_us(c[1], a.y,
+                       dev::dp4a_us(c[2], a.z, dev::dp4a_us(c[3], a.w, mt.corr0))));
+        const int i1 = dev::dp4a_us(c[4], b.x, dev::dp4a_us(c[5], b.y,
+                       dev::dp4a_us(c[6], b.z, dev::dp4a_us(c[7], b.w, mt.corr1))));
+        const float2 sf = dev::ue4m3x2_to_float2(s2);
+        acc = fmaf(mt.d, fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
+      };
+      if constexpr (NPL > 0) {
+        uint4 w[NPL], a[NPL], b[NPL];
+        ActMeta mt[NPL];
+        uint32_t s2[NPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          const int j = lane + 32 * i;
+          w[i] = cw[j];
+          s2[i] = sw[j];
+          a[i] = qa[cbase + j];
+          b[i] = qb[cbase + j];
+          mt[i] = meta[cbase + j];
+        }
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) chunk(w[i], s2[i], a[i], b[i], mt[i]);
+      } else {
+#pragma unroll 2
+        for (int j = lane; j < nch; j += 32)
+          chunk(cw[j], sw[j], qa[cbase + j], qb[cbase + j], meta[cbase + j]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(empty + s));
+    if (sg == nseg - 1) {
+      if (warp < nrows) {
+        const float v = dev::warp_sum(acc);
+        if (lane == 0) y[row0 + warp] = v * half_g;
+      }
+      acc = 0.0f;
+    }
+  }
 }
 
 template <int MT>
@@ -309,11 +508,38 @@ int tma_segment(int64_t K) {
   return 0;
 }
 
+template <int NPL>
+cudaError_t launch_m1(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                      int64_t K, int seg, const int8_t* q, const uint16_t* d, float* y,
+                      cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_m1_kernel<NPL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemPerCtaMax));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int64_t ctas = std::min<int64_t>(device_sm_count(), N);
+  gemv_m1_kernel<NPL><<<static_cast<unsigned>(ctas), kM1Threads,
+                        m1_smem_bytes(static_cast<int>(K), seg), stream>>>(
+      codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), seg, q,
+      reinterpret_cast<const __half*>(d), y);
+  return cudaGetLastError();
+}
+
 template <int MT>
 cudaError_t launch_gemv_m(const uint8_t* codes, const uint8_t* scales, float g,
                           int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
                           float* y, cudaStream_t stream) {
   const int seg = tma_segment(K);
+  if (MT == 1 && seg > 0 && m1_smem_bytes(static_cast<int>(K), seg) <= kSmemPerCtaMax) {
+    if (seg == 5120) return launch_m1<5>(codes, scales, g, N, K, seg, q, d, y, stream);
+    if (seg == 4096) return launch_m1<4>(codes, scales, g, N, K, seg, q, d, y, stream);
+    return launch_m1<0>(codes, scales, g, N, K, seg, q, d, y, stream);
+  }
   if (seg > 0) {
     const uint32_t smem = tma_smem_bytes(seg);
     static bool attr_set[64] = {};

@@ -45,6 +45,40 @@ __device__ __forceinline__ void decode_e2m1x8(uint32_t w, uint32_t& lo, uint32_t
   lut16_x8<kLutPosLo, kLutPosHi, kLutNegLo, kLutNegHi>(w, lo, hi);
 }
 
+// The same integer LUT biased by +12 (0..24, unsigned bytes), the storage
+// form of the "Bias trick" paragraph of "HANDOFF: flint CPU optimization
+// (Q4_1 + NVFP4)", section 3: c + 12 for codes 0..7 and for codes 8..15.
+constexpr uint32_t kBiasPosLo = 0x0F0E0D0Cu;  // codes 0..3   -> 12, 13, 14, 15
+constexpr uint32_t kBiasPosHi = 0x18141210u;  // codes 4..7   -> 16, 18, 20, 24
+constexpr uint32_t kBiasNegLo = 0x090A0B0Cu;  // codes 8..11  -> 12, 11, 10,  9
+constexpr uint32_t kBiasNegHi = 0x00040608u;  // codes 12..15 ->  8,  6,  4,  0
+
+// Byte permute with the sign-replicating selector mode: a selector nibble
+// with bit 3 set yields the sign (bit 7) of the selected byte, replicated.
+__device__ __forceinline__ uint32_t prmt_sr(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Decode eight E2M1 codes to the biased bytes c + 12.  Every table byte is
+// below 0x80, so a lookup whose selector has bit 3 set gives 0: the lookup
+// in the positive half with the raw codes fills the bytes of codes 0..7 and
+// zeroes the others, the lookup in the negative half with bit 3 flipped
+// does the converse, and an OR merges them (9 operations per 8 codes).
+__device__ __forceinline__ void decode_e2m1x8_biased(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t wn = w ^ 0x88888888u;
+  lo = prmt_sr(kBiasPosLo, kBiasPosHi, w) | prmt_sr(kBiasNegLo, kBiasNegHi, wn);
+  hi = prmt_sr(kBiasPosLo, kBiasPosHi, w >> 16) | prmt_sr(kBiasNegLo, kBiasNegHi, wn >> 16);
+}
+
+// dp4a with unsigned bytes in a and signed bytes in b.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int r;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
 // Two UE4M3 scale bytes (low byte = first subblock) to fp32, exactly.  UE4M3
 // is E4M3 with the sign bit 0, so the hardware E4M3 -> f16 conversion
 // applies; every UE4M3 value (2^-9 .. 448) is exact in fp16.
