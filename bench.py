@@ -4,31 +4,43 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl nvq|reference]
 
-Prints ONE JSON line on rank 0.  Default workload ``decode_sweep``: one step
-quantises one token's activations (Q8_0) and runs the decode GEMV for each of
-the four linear shapes of a 27B-class dense decoder, (K, N) = (5120, 5120),
-(5120, 25600), (25600, 5120), (5120, 152064); the metric is weight GB/s
-(NVFP4 weight bytes N*K*0.5625 streamed per second).  Other workloads:
-``gemv_4096`` (M=1, K=N=4096), ``small_batch`` (M=2..16), ``prefill`` (GEMM,
-M in {256, 2048}; metric TFLOP/s = 2*M*N*K/s), ``stack_decode`` and
-``stack_prefill`` (all linears of a 64-layer dense decoder; tokens/s).
+Prints ONE JSON line on rank 0.
 
-Timing: W untimed warm-up steps, then exactly K steps bracketed by a
-barrier and a device synchronize, timed with CUDA events on the launching
-stream; the time is the max over ranks.  The weights of one step exceed the
-126 MB L2 (about 600 MB for the decode sweep), so no L2 flush is inserted.
-The dominant kernel is additionally bracketed by its own events inside the
-timed region for the roofline entry.  ``e2e`` repeats the K steps through the
-same public entry points with each step's activations copied from pinned
-host memory and its outputs copied back inside the timed region.
+Workloads (``--workload``):
+  decode_sweep (default)  one step quantises one token's activations (Q8_0)
+                          and runs the decode GEMV for each of the four
+                          linear shapes of a 27B-class dense decoder,
+                          (K, N) = (5120, 5120), (5120, 25600), (25600, 5120),
+                          (5120, 152064).  Metric: weight GB/s (NVFP4 weight
+                          bytes N*K*0.5625 streamed per second).
+  gemv_4096               M=1, K=N=4096.
+  small_batch_m{2,4,8,16} decode GEMV at M tokens, (5120, 25600), (25600, 5120).
+  prefill_m{256,2048}     Q8_0 + tcgen05 GEMM over (5120, 5120), (5120, 25600),
+                          (25600, 5120).  Metric: algorithmic TFLOP/s 2*M*N*K.
+  stack_decode            all 448 linears of a 64-layer dense decoder (17.9 GB
+                          of NVFP4 weights resident), one token.  Metric:
+                          tokens/s of the linear layers.
+  stack_prefill           the same stack for 2048 tokens.
+
+Timing: W untimed eager warm-up steps; the K timed steps are captured once
+into a CUDA graph (the public entry points are graph-capturable: they only
+enqueue work) and replayed inside the timed region, bracketed by a barrier
+and a device synchronize and timed with CUDA events on the launching stream;
+the time is the max over ranks.  The dominant kernel of every step is
+bracketed by its own (graph-recorded) events for the roofline entry.  One
+step's weights exceed the 126 MB L2 in every workload (600 MB for the decode
+sweep), so no L2 flush is inserted.  ``e2e`` runs the same K steps through
+the public Python API eagerly, with each step's activations copied from
+pinned host memory and its outputs copied back inside the timed region (the
+weights are resident model parameters).
 
 Multi-GPU (``torchrun --nproc-per-node N``): every rank runs the same
 workload on its own GPU with no data exchange (independent replicas; the
 only collectives are the timing barrier and max).  ``value`` is the units of
-all ranks divided by the max time, ``scaling`` is "weak".
+all ranks divided by the max time; ``scaling`` is "weak".
 
-``--impl reference`` times the plain CPU oracle on the host cores (rank 0
-only), each step a bounded sample of the same workload, on the same metric.
+``--impl reference`` times the plain CPU oracle on the host (rank 0 only),
+each step a bounded sample of the same workload, on the same metric.
 """
 from __future__ import annotations
 
@@ -55,7 +67,7 @@ WEIGHT_BYTES_PER_ELEMENT = 0.5625       # 4-bit code + one UE4M3 byte per 16
 
 
 # ---------------------------------------------------------------------------
-# process group, peaks, clocks
+# process group, peaks, clocks, profiles
 # ---------------------------------------------------------------------------
 
 class Dist:
@@ -107,7 +119,7 @@ _REASON_FIELDS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms."""
+    """nvidia-smi SM clocks, power and throttle reasons every 100 ms."""
 
     def __init__(self, device_index: int):
         self.samples = []
@@ -157,14 +169,17 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self, t0: float, t1: float) -> dict:
-        inside = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if not inside:
+            inside, window = self.samples, "whole run (timed region shorter than one sample)"
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         reasons = sorted({r for s in inside for r in s[4]})
         return {"sm_mhz": statistics.median(s[1] for s in inside),
                 "sm_max_mhz": max(s[2] for s in inside),
                 "power_w_max": max(s[3] for s in inside),
-                "reasons": reasons, "samples": len(inside)}
+                "reasons": reasons, "samples": len(inside), "window": window}
 
 
 def source_hash(*names: str) -> str:
@@ -178,7 +193,7 @@ def source_hash(*names: str) -> str:
 def profiled_traffic(kernel: str, workload: str, src_hash: str):
     """DRAM bytes per launch from the committed ncu summary of this kernel on
     this workload, or None when absent or taken on other kernel sources."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
@@ -190,6 +205,33 @@ def profiled_traffic(kernel: str, workload: str, src_hash: str):
     return float(m_bytes.group(1))
 
 
+class EventLog:
+    """Start/stop events around the dominant kernel of each step; created
+    external so that they become timestamp nodes when captured in a graph."""
+
+    def __init__(self):
+        self.pairs = []
+        self._open = None
+
+    def begin(self, stream):
+        import torch
+        ev = torch.cuda.Event(enable_timing=True, external=True)
+        ev.record(stream)
+        self._open = ev
+
+    def end(self, stream, amount):
+        import torch
+        ev = torch.cuda.Event(enable_timing=True, external=True)
+        ev.record(stream)
+        self.pairs.append((self._open, ev, amount))
+        self._open = None
+
+    def totals(self):
+        ms = sum(a.elapsed_time(b) for a, b, _ in self.pairs)
+        amount = sum(x for _, _, x in self.pairs)
+        return ms, amount, len(self.pairs)
+
+
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
@@ -199,24 +241,24 @@ class GemvWorkload:
     each shape's activations and runs its GEMV."""
 
     kernel = "gemv"
-    sources = ("gemv.cu", "nvq_device.cuh")
+    sources = ("gemv.cu", "nvq_device.cuh", "tcgen05.cuh")
+    bound = "hbm"
+    metric = "nvfp4_q8_0_gemv_weight_GBps"
+    unit = "GB/s"
 
     def __init__(self, name, shapes, M, make_case):
         self.name, self.shapes, self.M, self.make_case = name, shapes, M, make_case
-        self.metric = "nvfp4_q8_0_gemv_weight_GBps"
-        self.unit = "GB/s"
 
-    # --- setup -------------------------------------------------------------
     def setup(self, device):
         import torch
         from bit_weight_quantized_nvq_b200 import capi
         self.capi = capi
-        self.layers = []
+        self.cases = []
         for K, N in self.shapes:
             W, x = self.make_case(K, N)
             codes, scales, g = capi.pack_nvfp4(W)
             del W
-            L = {"K": K, "N": N, "g": g,
+            c = {"K": K, "N": N, "g": g,
                  "codes": torch.from_numpy(codes).to(device),
                  "scales": torch.from_numpy(scales).to(device),
                  "x": torch.from_numpy(x).to(device),
@@ -224,14 +266,14 @@ class GemvWorkload:
                  "q": torch.empty((self.M, K), dtype=torch.int8, device=device),
                  "d": torch.empty((self.M, K // 32), dtype=torch.float16, device=device),
                  "y": torch.empty((self.M, N), dtype=torch.float32, device=device)}
-            L["y_host"] = torch.empty_like(L["y"], device="cpu").pin_memory()
-            self.layers.append(L)
+            c["y_host"] = torch.empty((self.M, N), dtype=torch.float32).pin_memory()
+            self.cases.append(c)
 
     def config(self):
         return {"workload": self.name, "M": self.M,
                 "shapes_KN": [list(s) for s in self.shapes],
                 "weights": "NVFP4 (E2M1 + UE4M3 per 16 + fp32 g), N(0,0.02^2)",
-                "activations": "Q8_0 quantised per step on the GPU",
+                "activations": "fp32 -> Q8_0 on the GPU every step",
                 "l2": "inputs larger than L2 (weights of one step %.0f MB > 126 MB)"
                       % (self.weight_bytes() / 1e6),
                 "parallelism": "replicas"}
@@ -242,52 +284,47 @@ class GemvWorkload:
     def units_per_step(self):
         return self.weight_bytes() / 1e9          # GB
 
-    def kernel_bytes(self, L):
-        """Algorithmic bytes of one GEMV launch: weights + scales, the Q8_0
+    def kernel_amount(self, c):
+        """Algorithmic bytes of one GEMV launch: NVFP4 weights, Q8_0
         activations and the fp32 output."""
-        M, K, N = self.M, L["K"], L["N"]
+        M, K, N = self.M, c["K"], c["N"]
         return N * K * WEIGHT_BYTES_PER_ELEMENT + M * K * (1 + 2 / 32) + 4 * M * N
 
     def launches_per_step(self):
-        return 2 * len(self.layers)
+        return 2 * len(self.cases)
 
-    # --- one step ------------------------------------------------------------
-    def step(self, stream, events=None, e2e=False):
+    def step(self, stream, log=None, e2e=False):
         capi = self.capi
-        for L in self.layers:
+        for c in self.cases:
             if e2e:
-                L["x"].copy_(L["x_host"], non_blocking=True)
-            capi.quantize_act_q8_0(L["x"], L["q"], L["d"], stream=stream)
-            if events is not None:
-                ev0, ev1 = events.pop()
-                ev0.record(stream)
-            capi.gemv(L["codes"], L["scales"], L["g"], L["q"], L["d"], L["y"], stream=stream)
-            if events is not None:
-                ev1.record(stream)
-                events.done.append((ev0, ev1, self.kernel_bytes(L)))
+                c["x"].copy_(c["x_host"], non_blocking=True)
+            capi.quantize_act_q8_0(c["x"], c["q"], c["d"], stream=stream)
+            if log is not None:
+                log.begin(stream)
+            capi.gemv(c["codes"], c["scales"], c["g"], c["q"], c["d"], c["y"], stream=stream)
+            if log is not None:
+                log.end(stream, self.kernel_amount(c))
             if e2e:
-                L["y_host"].copy_(L["y"], non_blocking=True)
+                c["y_host"].copy_(c["y"], non_blocking=True)
 
     def e2e_bytes(self):
-        h2d = sum(L["x"].numel() * 4 for L in self.layers)
-        d2h = sum(L["y"].numel() * 4 for L in self.layers)
-        return h2d, d2h
+        return (sum(c["x"].numel() * 4 for c in self.cases),
+                sum(c["y"].numel() * 4 for c in self.cases))
 
     # --- CPU oracle sample ---------------------------------------------------
-    def oracle_prepare(self, rows_per_shape):
+    def oracle_prepare(self, size):
         import oracle as o
         self.o = o
         self.samples = []
         for K, N in self.shapes:
             W, x = self.make_case(K, N)
             g = o.nvfp4_tensor_scale(W)
-            r = min(rows_per_shape, N)
+            r = min(size, N)
             codes, scales, _ = o.pack_nvfp4(W[:r], g=g)
             del W
             self.samples.append((K, r, codes, scales, g, x))
 
     def oracle_step(self):
-        """Quantise and dot the sampled rows; returns the sample's GB."""
         o = self.o
         gb = 0.0
         for K, r, codes, scales, g, x in self.samples:
@@ -296,20 +333,218 @@ class GemvWorkload:
             gb += r * K * WEIGHT_BYTES_PER_ELEMENT / 1e9
         return gb
 
-    def oracle_sample_desc(self, rows):
-        return (f"first {rows} rows of each of the {len(self.shapes)} shapes, "
-                f"M={self.M}: oracle Q8_0 quantisation + fp64 dequantise-then-dot")
+    def oracle_sample_desc(self, size):
+        return (f"first {size} rows of each of the {len(self.shapes)} shapes, M={self.M}: "
+                "oracle Q8_0 quantisation + fp64 dequantise-then-dot")
 
 
-class EventPool:
-    def __init__(self, n):
+class GemmWorkload:
+    """Prefill: Q8_0 of M tokens and the tcgen05 GEMM for each shape."""
+
+    kernel = "gemm"
+    sources = ("gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+    bound = "tensor"
+    metric = "nvfp4_q8_0_prefill_gemm_TFLOPs"
+    unit = "TFLOP/s"
+
+    def __init__(self, name, shapes, M):
+        self.name, self.shapes, self.M = name, shapes, M
+
+    def setup(self, device):
         import torch
-        self.free = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                     for _ in range(n)]
-        self.done = []
+        from bit_weight_quantized_nvq_b200 import capi, workloads as wl
+        self.capi = capi
+        self.cases = []
+        M = self.M
+        for K, N in self.shapes:
+            W, x = wl.prefill_case(M, K, N)
+            codes, scales, g = capi.pack_nvfp4(W)
+            del W
+            c = {"K": K, "N": N, "g": g,
+                 "codes": torch.from_numpy(codes).to(device),
+                 "scales": torch.from_numpy(scales).to(device),
+                 "x": torch.from_numpy(x).to(device),
+                 "x_host": torch.from_numpy(x).pin_memory(),
+                 "q": torch.empty((M, K), dtype=torch.int8, device=device),
+                 "d": torch.empty((M, K // 32), dtype=torch.float16, device=device),
+                 "y": torch.empty((M, N), dtype=torch.float32, device=device),
+                 "ws": torch.empty(capi.gemm_workspace_size(M, N, K), dtype=torch.uint8,
+                                   device=device)}
+            c["y_host"] = torch.empty((M, N), dtype=torch.float32).pin_memory()
+            self.cases.append(c)
 
-    def pop(self):
-        return self.free.pop()
+    def config(self):
+        return {"workload": self.name, "M": self.M,
+                "shapes_KN": [list(s) for s in self.shapes],
+                "weights": "NVFP4, N(0,0.02^2)",
+                "activations": "fp32 N(0,1), 0.1% channels x50 -> Q8_0 on the GPU every step",
+                "l2": "inputs larger than L2 (activations and weights of one step > 126 MB)",
+                "parallelism": "replicas"}
+
+    def flops(self, c):
+        return 2.0 * self.M * c["N"] * c["K"]
+
+    def units_per_step(self):
+        return sum(2.0 * self.M * N * K for K, N in self.shapes) / 1e12   # TFLOP
+
+    def kernel_amount(self, c):
+        return self.flops(c)
+
+    def launches_per_step(self):
+        return 3 * len(self.cases)       # quantise, expand, tcgen05 GEMM
+
+    def step(self, stream, log=None, e2e=False):
+        capi = self.capi
+        for c in self.cases:
+            if e2e:
+                c["x"].copy_(c["x_host"], non_blocking=True)
+            capi.quantize_act_q8_0(c["x"], c["q"], c["d"], stream=stream)
+            if log is not None:
+                log.begin(stream)
+            capi.gemm(c["codes"], c["scales"], c["g"], c["q"], c["d"], c["y"], c["ws"],
+                      stream=stream)
+            if log is not None:
+                log.end(stream, self.kernel_amount(c))
+            if e2e:
+                c["y_host"].copy_(c["y"], non_blocking=True)
+
+    def e2e_bytes(self):
+        return (sum(c["x"].numel() * 4 for c in self.cases),
+                sum(c["y"].numel() * 4 for c in self.cases))
+
+    def oracle_prepare(self, size):
+        import oracle as o
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        self.o = o
+        self.samples = []
+        toks = max(1, min(self.M, size // 64))
+        for K, N in self.shapes:
+            W, x = wl.prefill_case(self.M, K, N)
+            g = o.nvfp4_tensor_scale(W)
+            r = min(size, N)
+            codes, scales, _ = o.pack_nvfp4(W[:r], g=g)
+            del W
+            self.samples.append((K, r, codes, scales, g, x[:toks]))
+
+    def oracle_step(self):
+        o = self.o
+        tf = 0.0
+        for K, r, codes, scales, g, x in self.samples:
+            q, d = o.quantize_q8_0(x)
+            o.dot_fp64(codes, scales, g, q, d)
+            tf += 2.0 * x.shape[0] * r * K / 1e12
+        return tf
+
+    def oracle_sample_desc(self, size):
+        toks = max(1, min(self.M, size // 64))
+        return (f"{toks} tokens x first {size} rows of each of the {len(self.shapes)} shapes: "
+                "oracle Q8_0 + fp64 dequantise-then-dot")
+
+
+class StackWorkload:
+    """Every linear of a 64-layer dense decoder through nvq_decoder_stack."""
+
+    kernel = "stack_pass"
+    sources = ("nvq_stack.cpp", "gemv.cu", "gemm_tcgen05.cu", "quantize_q8_0.cu")
+    unit = "tokens/s"
+
+    def __init__(self, name, M):
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        self.name, self.M = name, M
+        self.bound = "hbm" if M <= 16 else "tensor"
+        self.metric = "nvfp4_q8_0_linear_stack_tokens_per_s"
+        self.n_layers = wl.STACK_LAYERS
+        self.linears = wl.STACK_LINEARS
+
+    def setup(self, device):
+        import torch
+        from bit_weight_quantized_nvq_b200 import capi, workloads as wl
+        self.capi = capi
+        self.layer_host = []
+        for name, W in wl.stack_layer_weights():
+            codes, scales, g = capi.pack_nvfp4(W)
+            self.layer_host.append((codes, scales, g))
+            del W
+        layers = []
+        for _ in range(wl.STACK_LAYERS):
+            layers.append([(torch.from_numpy(c).to(device), torch.from_numpy(s).to(device), g)
+                           for c, s, g in self.layer_host])
+        self.stack = capi.DecoderStack(layers, self.M, device=device)
+        x = wl.stack_input(self.M)
+        self.x = torch.from_numpy(x).to(device)
+        self.x_host = torch.from_numpy(x).pin_memory()
+        self.y_host = torch.empty(tuple(self.stack.outs[6].shape), dtype=torch.float32).pin_memory()
+
+    def weight_bytes(self):
+        return self.n_layers * sum(N * K * WEIGHT_BYTES_PER_ELEMENT for _, K, N in self.linears)
+
+    def flops(self):
+        return 2.0 * self.M * self.n_layers * sum(N * K for _, K, N in self.linears)
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "layers": self.n_layers,
+                "linears_KN": {n: [K, N] for n, K, N in self.linears},
+                "weights_GB": round(self.weight_bytes() / 1e9, 2),
+                "dataflow": "per layer: Q8_0(x)->q,k,v; Q8_0(y_v)->o; Q8_0(y_o)->up,gate; "
+                            "Q8_0(y_up)->down; every layer restarts from the same x",
+                "l2": "inputs larger than L2 (17.9 GB of weights per pass)",
+                "parallelism": "replicas"}
+
+    def units_per_step(self):
+        return float(self.M)                        # tokens
+
+    def kernel_amount(self, _=None):
+        return self.weight_bytes() if self.bound == "hbm" else self.flops()
+
+    def launches_per_step(self):
+        per_layer = 4 + 7 + (4 if self.M > 16 else 0)
+        return per_layer * self.n_layers
+
+    def step(self, stream, log=None, e2e=False):
+        if e2e:
+            self.x.copy_(self.x_host, non_blocking=True)
+        if log is not None:
+            log.begin(stream)
+        self.stack.forward(self.x, stream=stream)
+        if log is not None:
+            log.end(stream, self.kernel_amount())
+        if e2e:
+            self.y_host.copy_(self.stack.outs[6], non_blocking=True)
+
+    def e2e_bytes(self):
+        return self.x.numel() * 4, self.stack.outs[6].numel() * 4
+
+    def oracle_prepare(self, size):
+        import oracle as o
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        self.o = o
+        self.samples = []
+        toks = max(1, min(self.M, size // 256))
+        for name, W in wl.stack_layer_weights():
+            g = o.nvfp4_tensor_scale(W)
+            r = min(size, W.shape[0])
+            codes, scales, _ = o.pack_nvfp4(W[:r], g=g)
+            self.samples.append((W.shape[1], W.shape[0], r, codes, scales, g))
+        self.x_s = wl.stack_input(self.M)[:toks]
+
+    def oracle_step(self):
+        """One layer's 7 products on a row sample; returns tokens of the
+        64-layer pass that this much work is worth (row fraction x layers)."""
+        o = self.o
+        frac = 0.0
+        rng = np.random.default_rng(0)
+        for K, N, r, codes, scales, g in self.samples:
+            x = rng.standard_normal((self.x_s.shape[0], K)).astype(np.float32)
+            q, d = o.quantize_q8_0(x)
+            o.dot_fp64(codes, scales, g, q, d)
+            frac += r * K / sum(KK * NN for _, KK, NN in self.linears)
+        return self.x_s.shape[0] * frac / self.n_layers
+
+    def oracle_sample_desc(self, size):
+        toks = max(1, min(self.M, size // 256))
+        return (f"{toks} token(s) x first {size} rows of each of the 7 linears of one layer "
+                "(random activations), scaled to the 64-layer pass by the fraction of weights "
+                "processed")
 
 
 def make_workload(name: str):
@@ -322,12 +557,51 @@ def make_workload(name: str):
         M = int(name[len("small_batch_m"):])
         return GemvWorkload(name, wl.SMALL_BATCH_SHAPES, M,
                             lambda K, N: wl.small_batch_case(M, K, N))
+    if name.startswith("prefill_m"):
+        return GemmWorkload(name, wl.PREFILL_SHAPES, int(name[len("prefill_m"):]))
+    if name == "stack_decode":
+        return StackWorkload(name, 1)
+    if name == "stack_prefill":
+        return StackWorkload(name, 2048)
     raise SystemExit(f"unknown workload {name!r}")
 
 
 # ---------------------------------------------------------------------------
-# arms
+# timing
 # ---------------------------------------------------------------------------
+
+def capture_steps(wk, steps: int, stream):
+    """A CUDA graph of `steps` steps with the dominant-kernel events."""
+    import torch
+    log = EventLog()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        s = torch.cuda.current_stream()
+        for _ in range(steps):
+            wk.step(s, log)
+    return graph, log
+
+
+def roofline_entry(wk, log, peaks):
+    kernel_ms, amount, n = log.totals()
+    src_hash = source_hash(*wk.sources)
+    traffic = profiled_traffic(wk.kernel, wk.name, src_hash)
+    if wk.bound == "hbm":
+        achieved = amount / (kernel_ms / 1e3) / 1e9
+        peak, unit, src = peaks["hbm_gbs"], "GB/s", "hbm_gbs (copy)"
+    else:
+        achieved = amount / (kernel_ms / 1e3) / 1e12
+        peak, unit, src = peaks["bf16_tflops"], "TFLOP/s", "bf16_tflops (burst; fp16 runs at the bf16 rate)"
+    entry = {"bound": wk.bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+             "frac": round(achieved / peak, 4), "traffic": traffic,
+             "kernel": wk.kernel, "launches": n,
+             "avg_launch_us": round(kernel_ms * 1e3 / max(1, n), 3),
+             "algorithmic_per_launch": amount / max(1, n),
+             "peak_source": f"{peaks['source']} MEASURED_PEAKS.json {src}"}
+    if wk.bound == "tensor" and wk.kernel == "gemm":
+        entry["issued_frac"] = round(2 * achieved / peak, 4)   # hi and lo halves
+    return entry
+
 
 def run_nvq(args, dist: Dist):
     import torch
@@ -337,37 +611,38 @@ def run_nvq(args, dist: Dist):
     peaks = load_peaks()
     wk = make_workload(args.workload)
     wk.setup(device)
-    stream = torch.cuda.current_stream(device)
+    # graphs are captured on a side stream; everything runs on it
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
 
     for _ in range(args.warmup):
         wk.step(stream)
     torch.cuda.synchronize()
+    graph, log = capture_steps(wk, args.steps, stream)
+    graph.replay()                        # one untimed replay (graph upload)
+    torch.cuda.synchronize()
 
     sampler = ClockSampler(dist.local_rank)
     sampler.start()
-    time.sleep(0.3)
-    nlaunch = len(wk.shapes) * args.steps
-    events = EventPool(nlaunch)
+    time.sleep(0.35)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record(stream)
-    for _ in range(args.steps):
-        wk.step(stream, events)
+    graph.replay()
     end.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
     dist.barrier()
     ms = start.elapsed_time(end)
-    kernel_ms = sum(a.elapsed_time(b) for a, b, _ in events.done)
-    kernel_bytes = sum(nb for _, _, nb in events.done)
-    n_kernel = len(events.done)
-    time.sleep(0.2)
+    roofline = roofline_entry(wk, log, peaks)
+    time.sleep(0.25)
     sampler.stop()
-    clocks = sampler.summary(t_wall0 - 0.15, t_wall1 + 0.15)
+    clocks = sampler.summary(t_wall0 - 0.1, t_wall1 + 0.1)
+    del graph
 
-    # e2e: the same K steps with host<->device copies inside the timed region
+    # e2e: the same K steps through the public API, eagerly, with copies
     for _ in range(max(1, args.warmup // 2)):
         wk.step(stream, e2e=True)
     torch.cuda.synchronize()
@@ -387,17 +662,9 @@ def run_nvq(args, dist: Dist):
     value = units / (ms_max / 1e3)
     e2e_value = units / (e2e_ms_max / 1e3)
 
-    achieved = kernel_bytes / (kernel_ms / 1e3) / 1e9       # GB/s
-    src_hash = source_hash(*wk.sources)
-    traffic = profiled_traffic(wk.kernel, wk.name, src_hash)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic,
-                "algorithmic_bytes_per_launch": kernel_bytes / max(1, n_kernel),
-                "kernel": wk.kernel, "launches": n_kernel,
-                "avg_launch_us": round(kernel_ms * 1e3 / max(1, n_kernel), 3),
-                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)"}
+    extra = {}
+    if args.workload == "decode_sweep" and dist.world == 1 and not args.no_prefill_summary:
+        extra["prefill_gemm"] = prefill_summary(device, peaks)
 
     cpu = None
     if dist.rank == 0 and not args.no_cpu_baseline:
@@ -405,42 +672,74 @@ def run_nvq(args, dist: Dist):
 
     h2d, d2h = wk.e2e_bytes()
     line = {
-        "metric": wk.metric, "value": round(value, 2), "unit": wk.unit,
+        "metric": wk.metric, "value": round(value, 3), "unit": wk.unit,
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_max / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4 x q8_0 (int32 subblock sums, fp32 accumulate)",
+        "dtype": "nvfp4 x q8_0 (int32 subblock sums / exact fp16 operands, fp32 accumulate)",
         "data": "synthetic (seeded; shapes and distributions of the workload)",
         "config": wk.config(),
         "impl": "nvq",
-        "e2e": {"value": round(e2e_value, 2), "unit": wk.unit,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "timing": "CUDA graph of the K steps replayed once; events on the launching stream",
+        "e2e": {"value": round(e2e_value, 3), "unit": wk.unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "eager public API calls with pinned-host copies"},
         "gpu_launches": wk.launches_per_step() * args.steps,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "clocks": clocks,
     }
+    line.update(extra)
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()
 
 
+def prefill_summary(device, peaks):
+    """The prefill GEMM at 2048 tokens, timed the same way (graph replay),
+    reported next to the decode line."""
+    import torch
+    wk = make_workload("prefill_m2048")
+    wk.setup(device)
+    stream = torch.cuda.current_stream(device)   # the side stream set by run_nvq
+    for _ in range(3):
+        wk.step(stream)
+    torch.cuda.synchronize()
+    steps = 10
+    graph, log = capture_steps(wk, steps, stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    roof = roofline_entry(wk, log, peaks)
+    out = {"workload": "prefill_m2048", "shapes_KN": [list(s) for s in wk.shapes],
+           "step_TFLOPs": round(wk.units_per_step() * steps / (ms / 1e3), 2),
+           "roofline": roof}
+    del graph, wk
+    torch.cuda.empty_cache()
+    return out
+
+
 def cpu_baseline(wk, seconds: float):
-    """The oracle, timed on the host on a bounded sample of the workload."""
+    """The oracle, timed on one host core on a bounded sample of the workload."""
     import threadpoolctl
-    rows = 64
-    wk.oracle_prepare(rows)
+    size = 64
     with threadpoolctl.threadpool_limits(1):
+        wk.oracle_prepare(size)
         t0 = time.perf_counter()
         wk.oracle_step()
         t_small = time.perf_counter() - t0
-        rows = int(max(64, min(8192, rows * seconds / max(t_small, 1e-3))))
-        wk.oracle_prepare(rows)
+        size = int(max(64, min(65536, size * seconds / max(t_small, 1e-3))))
+        wk.oracle_prepare(size)
         t0 = time.perf_counter()
-        gb = wk.oracle_step()
+        units = wk.oracle_step()
         t = time.perf_counter() - t0
-    return {"value": round(gb / t, 4), "unit": wk.unit, "cores": 1, "kind": "oracle",
-            "sample": wk.oracle_sample_desc(rows), "seconds": round(t, 2)}
+    return {"value": round(units / t, 6), "unit": wk.unit, "cores": 1, "kind": "oracle",
+            "sample": wk.oracle_sample_desc(size), "seconds": round(t, 2)}
 
 
 def run_reference(args, dist: Dist):
@@ -450,38 +749,37 @@ def run_reference(args, dist: Dist):
     import threadpoolctl
     wk = make_workload(args.workload)
     # size the per-step sample so that warm-up + timed steps take about
-    # --cpu-seconds * 6 in total (a few minutes at most)
+    # 6 * --cpu-seconds in total (a few minutes at most)
     budget = 6 * args.cpu_seconds / (args.steps + args.warmup)
-    rows = 64
-    wk.oracle_prepare(rows)
+    size = 64
     with threadpoolctl.threadpool_limits(1):
+        wk.oracle_prepare(size)
         t0 = time.perf_counter()
         wk.oracle_step()
         t_small = time.perf_counter() - t0
-    rows = int(max(8, min(8192, rows * budget / max(t_small, 1e-4))))
-    wk.oracle_prepare(rows)
-    with threadpoolctl.threadpool_limits(1):
+        size = int(max(8, min(65536, size * budget / max(t_small, 1e-4))))
+        wk.oracle_prepare(size)
         for _ in range(args.warmup):
             wk.oracle_step()
         t0 = time.perf_counter()
-        gb = 0.0
+        units = 0.0
         for _ in range(args.steps):
-            gb += wk.oracle_step()
+            units += wk.oracle_step()
         t = time.perf_counter() - t0
-    value = gb / t
-    desc = wk.oracle_sample_desc(rows)
+    value = units / t
+    desc = wk.oracle_sample_desc(size)
     line = {
-        "metric": wk.metric, "value": round(value, 4), "unit": wk.unit,
+        "metric": wk.metric, "value": round(value, 6), "unit": wk.unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (int64 subblock sums)",
-        "data": "synthetic (seeded; a bounded row sample of the workload)",
-        "config": wk.config() if hasattr(wk, "config") else {"workload": args.workload},
+        "data": "synthetic (seeded; a bounded sample of the workload per step)",
+        "config": dict(wk.config(), sample_per_step=desc),
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 4), "unit": wk.unit, "cores": 1,
+        "cpu_baseline": {"value": round(value, 6), "unit": wk.unit, "cores": 1,
                          "kind": "oracle", "sample": desc},
-        "e2e": {"value": round(value, 4), "unit": wk.unit,
+        "e2e": {"value": round(value, 6), "unit": wk.unit,
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -499,6 +797,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target duration of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill-summary", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

@@ -82,3 +82,64 @@ def assert_within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, sa: np.ndarray
             f"{bad.sum()} of {bad.size} outside tolerance; first at {tuple(i)}: "
             f"gpu={y_gpu[tuple(i)]!r} ref={y_ref[tuple(i)]!r} tol={tol[tuple(i)]!r}")
     return float((err / np.maximum(tol, 1e-300)).max())
+
+
+# ---------------------------------------------------------------------------
+# chained products (the decoder stack): tolerance propagation
+# ---------------------------------------------------------------------------
+
+def requant_bound(x_ref: np.ndarray, x_tol: np.ndarray) -> np.ndarray:
+    """Bound on |a_gpu - a_ref| for a = fp16(d)*q when the quantiser's input
+    is known only to within x_tol of the oracle's x_ref (fp32 values).
+
+    Per 32-block, the largest |x| lies within the tolerance of the oracle's,
+    so d32 and the fp16 d lie in an interval; every element's x/d32 lies in
+    an interval, and rint is monotone, so q lies in [q_lo, q_hi].  The bound
+    is the largest distance of d*q over those intervals from the oracle's
+    d_ref*q_ref.  It is zero wherever neither d nor q can change (the usual
+    case); only elements near a rounding tie get a nonzero bound.  Computed
+    from oracle quantities only."""
+    x = np.asarray(x_ref, np.float64)
+    M, K = x.shape
+    xb = x.reshape(M, K // 32, 32)
+    tb = np.asarray(x_tol, np.float64).reshape(M, K // 32, 32)
+    T = tb.max(axis=2)
+    amax = np.abs(xb).max(axis=2)
+    ulp32 = 2.0 ** -23
+    d32_lo = np.maximum(amax - T, 0) / 127 * (1 - 2 * ulp32)
+    d32_hi = (amax + T) / 127 * (1 + 2 * ulp32)
+    fp16 = o.fp16_values()
+    d_lo = fp16[o.fp32_to_fp16_bits(d32_lo.astype(np.float32))]
+    d_hi = fp16[o.fp32_to_fp16_bits(d32_hi.astype(np.float32))]
+    # the oracle's own quantisation of x_ref: the activations it multiplies
+    q_o, d_o = o.quantize_q8_0(np.asarray(x_ref, np.float32))
+    a_ref = (fp16[d_o][..., None] * q_o.reshape(M, K // 32, 32).astype(np.float64))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r_a = (xb - tb) / d32_lo[..., None]
+        r_b = (xb + tb) / d32_lo[..., None]
+        r_c = (xb - tb) / d32_hi[..., None]
+        r_d = (xb + tb) / d32_hi[..., None]
+    rs = np.stack([r_a, r_b, r_c, r_d])
+    rs = np.where(np.isfinite(rs), rs, 0.0)
+    q_lo = np.clip(np.rint(rs.min(axis=0) - 1e-6), -127, 127)
+    q_hi = np.clip(np.rint(rs.max(axis=0) + 1e-6), -127, 127)
+    cand = [d_lo[..., None] * q_lo, d_lo[..., None] * q_hi,
+            d_hi[..., None] * q_lo, d_hi[..., None] * q_hi]
+    bound = np.max([np.abs(c - a_ref) for c in cand], axis=0)
+    return bound.reshape(M, K)
+
+
+def chained_reference(P: Packed, x_ref: np.ndarray, da: np.ndarray):
+    """Oracle output of one product whose input activations come from a
+    requantisation with per-element uncertainty da (zeros for exact inputs):
+    returns (y_ref fp64, tol) with tol = the usual bound on the larger
+    sum|terms| plus sum_k |w[n, k]| * da[m, k]."""
+    q_ref, d_ref = o.quantize_q8_0(x_ref.astype(np.float32))
+    y, sa, _ = reference(P, q_ref, d_ref)
+    if np.any(da > 0):
+        w_abs = np.abs(o.dequantize_weights(P.ref_codes, P.ref_scales, P.ref_g))
+        spread = da @ w_abs.T
+    else:
+        spread = np.zeros_like(y)
+    tol = o.tolerance(sa + spread) + spread
+    return y, tol
