@@ -285,6 +285,191 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
   }
 }
 
+// ---------------------------------------------------------------------------
+// M = 1 schedule with the activations in registers (K = 1024 * NPL * WPR)
+// ---------------------------------------------------------------------------
+// Every lane of a consumer warp handles the same NPL chunk positions of
+// every row it ever processes, so the activation data of those chunks (32
+// codes, d and the two bias corrections) is loaded once into registers for
+// the whole kernel.  A row is split across WPR warps (warp part p owns the
+// p-th contiguous K segment of 1024 * NPL elements); a stage is R = 16/WPR
+// (or fewer, to fit 46 KB) whole, contiguous rows, fetched with two bulk
+// copies.  With WPR > 1 each warp leaves its row partial in shared memory
+// (one slot per stage) and the producer thread adds the WPR partials in a
+// fixed order when it recycles the stage, so results are deterministic.
+constexpr uint32_t kRegStageMax = 46080;
+
+__host__ __device__ constexpr int reg_rows(int K, int wpr) {
+  int r = kM1Consumers / wpr;
+  while (r > 1 && static_cast<uint32_t>(r) * (K / 2 + K / 16) > kRegStageMax) --r;
+  return r;
+}
+__host__ __device__ constexpr uint32_t reg_smem_bytes(int K, int wpr) {
+  return kM1Stages * static_cast<uint32_t>(reg_rows(K, wpr)) * (K / 2 + K / 16) +
+         kM1Stages * kM1Consumers * 4 + 2 * kM1Stages * 8 + 16;
+}
+
+template <int NPL, int WPR>
+__global__ void __launch_bounds__(kM1Threads, 1)
+gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                   float half_g, int N, int K, const int8_t* __restrict__ q,
+                   const __half* __restrict__ d, float* __restrict__ y) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int R = reg_rows(K, WPR);
+  const int active = R * WPR;                      // consumer warps in use
+  const uint32_t row_code = K / 2, row_scale = K / 16;
+  const uint32_t stage_bytes = static_cast<uint32_t>(R) * (row_code + row_scale);
+  const uint32_t codes_bytes = static_cast<uint32_t>(R) * row_code;
+  float* part = reinterpret_cast<float*>(smem + kM1Stages * stage_bytes);  // [stage][warp]
+  uint64_t* full = reinterpret_cast<uint64_t*>(part + kM1Stages * kM1Consumers);
+  uint64_t* empty = full + kM1Stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kM1Stages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
+  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
+  const int total = (r_end - r_begin + R - 1) / R;   // stages = row groups
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kM1Stages; ++i) {
+      ptx::mbar_init(ptx::smem_addr(full + i), 1);
+      ptx::mbar_init(ptx::smem_addr(empty + i), active);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kM1Consumers) {
+    // ------------- producer: bulk copies, and the sum of row partials --------
+    if (lane != 0) return;
+    auto finalize = [&](int it) {   // rows of stage `it`, once its slot is empty
+      if (WPR == 1) return;
+      const int s = it % kM1Stages;
+      const int row0 = r_begin + it * R;
+      const int nrows = min(R, r_end - row0);
+      for (int r = 0; r < nrows; ++r) {
+        float v = 0.0f;
+#pragma unroll
+        for (int p = 0; p < WPR; ++p) v += part[s * kM1Consumers + r * WPR + p];
+        y[row0 + r] = v * half_g;
+      }
+    };
+    int issued = 0;
+    bool ok = true;
+    for (int it = 0; it < total; ++it) {
+      const int s = it % kM1Stages;
+      const uint32_t ph = (it / kM1Stages) & 1;
+      if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        atomicOr(&g_gemv_error_flags, 1u);
+        ok = false;
+        break;
+      }
+      if (it >= kM1Stages) finalize(it - kM1Stages);
+      const int row0 = r_begin + it * R;
+      const int nrows = min(R, r_end - row0);
+      const uint32_t bar = ptx::smem_addr(full + s);
+      uint8_t* st = smem + s * stage_bytes;
+      ptx::mbar_arrive_expect_tx(bar, nrows * (row_code + row_scale));
+      ptx::bulk_load(ptx::smem_addr(st), codes + static_cast<size_t>(row0) * row_code,
+                     nrows * row_code, bar);
+      ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
+                     scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
+      ++issued;
+    }
+    if (ok) {
+      // the last stages: wait until consumed, then add their partials
+      for (int it = max(0, total - kM1Stages); it < total; ++it) {
+        if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + it % kM1Stages),
+                                    (it / kM1Stages) & 1, abort_flag, kWaitLimitNs)) {
+          *abort_flag = 1;
+          atomicOr(&g_gemv_error_flags, 1u);
+          break;
+        }
+        finalize(it);
+      }
+    } else {
+      for (int it = max(0, issued - kM1Stages); it < issued; ++it)
+        ptx::mbar_wait_bounded(ptx::smem_addr(full + it % kM1Stages), (it / kM1Stages) & 1,
+                               nullptr, kWaitLimitNs);
+    }
+    return;
+  }
+  if (warp >= active) return;
+
+  // ------------- consumers: warp w = (row w / WPR, part w % WPR) -------------
+  const int rl = warp / WPR;
+  const int p = warp % WPR;
+  uint4 qa[NPL], qb[NPL];
+  float dd[NPL];
+  int c0[NPL], c1[NPL];
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int c = p * (NPL * 32) + lane + 32 * i;   // chunk index in the row
+    const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * c;
+    qa[i] = __ldg(src);
+    qb[i] = __ldg(src + 1);
+    dd[i] = __half2float(__ldg(d + c));
+    const int s0 = dev::dp4a(qa[i].x, 0x01010101u, dev::dp4a(qa[i].y, 0x01010101u,
+                   dev::dp4a(qa[i].z, 0x01010101u, dev::dp4a(qa[i].w, 0x01010101u, 0))));
+    const int s1 = dev::dp4a(qb[i].x, 0x01010101u, dev::dp4a(qb[i].y, 0x01010101u,
+                   dev::dp4a(qb[i].z, 0x01010101u, dev::dp4a(qb[i].w, 0x01010101u, 0))));
+    c0[i] = -12 * s0;
+    c1[i] = -12 * s1;
+  }
+  for (int it = 0; it < total; ++it) {
+    const int s = it % kM1Stages;
+    const uint32_t ph = (it / kM1Stages) & 1;
+    if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
+      *abort_flag = 1;
+      atomicOr(&g_gemv_error_flags, 1u);
+      break;
+    }
+    const int row0 = r_begin + it * R;
+    const int nrows = min(R, r_end - row0);
+    float acc = 0.0f;
+    if (rl < nrows) {
+      const uint8_t* st = smem + s * stage_bytes;
+      const uint4* cw = reinterpret_cast<const uint4*>(st + rl * row_code) + p * (NPL * 32);
+      const uint16_t* sw =
+          reinterpret_cast<const uint16_t*>(st + codes_bytes + rl * row_scale) + p * (NPL * 32);
+      uint4 w[NPL];
+      uint32_t s2[NPL];
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        w[i] = cw[lane + 32 * i];
+        s2[i] = sw[lane + 32 * i];
+      }
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        uint32_t cb[8];
+        dev::decode_e2m1x8_biased(w[i].x, cb[0], cb[1]);
+        dev::decode_e2m1x8_biased(w[i].y, cb[2], cb[3]);
+        dev::decode_e2m1x8_biased(w[i].z, cb[4], cb[5]);
+        dev::decode_e2m1x8_biased(w[i].w, cb[6], cb[7]);
+        const int i0 = dev::dp4a_us(cb[0], qa[i].x, dev::dp4a_us(cb[1], qa[i].y,
+                       dev::dp4a_us(cb[2], qa[i].z, dev::dp4a_us(cb[3], qa[i].w, c0[i]))));
+        const int i1 = dev::dp4a_us(cb[4], qb[i].x, dev::dp4a_us(cb[5], qb[i].y,
+                       dev::dp4a_us(cb[6], qb[i].z, dev::dp4a_us(cb[7], qb[i].w, c1[i]))));
+        const float2 sf = dev::ue4m3x2_to_float2(s2[i]);
+        acc = fmaf(dd[i], fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
+      }
+      acc = dev::warp_sum(acc);
+      if (lane == 0) {
+        if (WPR == 1)
+          y[row0 + rl] = acc * half_g;
+        else
+          part[s * kM1Consumers + warp] = acc;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(empty + s));
+  }
+}
+
 template <int MT>
 __global__ void __launch_bounds__(kTmaThreads, 2)
 gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
@@ -530,11 +715,58 @@ cudaError_t launch_m1(const uint8_t* codes, const uint8_t* scales, float g, int6
   return cudaGetLastError();
 }
 
+template <int NPL, int WPR>
+cudaError_t launch_m1_reg(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                          int64_t K, const int8_t* q, const uint16_t* d, float* y,
+                          cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_m1_reg_kernel<NPL, WPR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemPerCtaMax));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int64_t ctas = std::min<int64_t>(device_sm_count(), N);
+  gemv_m1_reg_kernel<NPL, WPR><<<static_cast<unsigned>(ctas), kM1Threads,
+                                 reg_smem_bytes(static_cast<int>(K), WPR), stream>>>(
+      codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), q,
+      reinterpret_cast<const __half*>(d), y);
+  return cudaGetLastError();
+}
+
+// The register schedule covers K = 1024 * NPL * WPR for the (NPL, WPR) pairs
+// instantiated here; returns cudaErrorNotSupported for other K.
+cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, float g,
+                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                                   float* y, cudaStream_t stream) {
+  if (K % 1024 != 0) return cudaErrorNotSupported;
+  switch (K / 1024) {
+    case 4: return launch_m1_reg<4, 1>(codes, scales, g, N, K, q, d, y, stream);
+    case 5: return launch_m1_reg<5, 1>(codes, scales, g, N, K, q, d, y, stream);
+    case 6: return launch_m1_reg<6, 1>(codes, scales, g, N, K, q, d, y, stream);
+    case 8: return launch_m1_reg<4, 2>(codes, scales, g, N, K, q, d, y, stream);
+    case 10: return launch_m1_reg<5, 2>(codes, scales, g, N, K, q, d, y, stream);
+    case 12: return launch_m1_reg<6, 2>(codes, scales, g, N, K, q, d, y, stream);
+    case 15: return launch_m1_reg<5, 3>(codes, scales, g, N, K, q, d, y, stream);
+    case 16: return launch_m1_reg<4, 4>(codes, scales, g, N, K, q, d, y, stream);
+    case 20: return launch_m1_reg<5, 4>(codes, scales, g, N, K, q, d, y, stream);
+    case 25: return launch_m1_reg<5, 5>(codes, scales, g, N, K, q, d, y, stream);
+    default: return cudaErrorNotSupported;
+  }
+}
+
 template <int MT>
 cudaError_t launch_gemv_m(const uint8_t* codes, const uint8_t* scales, float g,
                           int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
                           float* y, cudaStream_t stream) {
   const int seg = tma_segment(K);
+  if (MT == 1) {
+    const cudaError_t e = launch_m1_reg_dispatch(codes, scales, g, N, K, q, d, y, stream);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if (MT == 1 && seg > 0 && m1_smem_bytes(static_cast<int>(K), seg) <= kSmemPerCtaMax) {
     if (seg == 5120) return launch_m1<5>(codes, scales, g, N, K, seg, q, d, y, stream);
     if (seg == 4096) return launch_m1<4>(codes, scales, g, N, K, seg, q, d, y, stream);
