@@ -44,6 +44,7 @@ SIGNATURES = {
     "nvq_quantize_act_q8_0": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp]),
     "nvq_gemv": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp]),
+    "nvq_quant_gemv": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp, _vp]),
     "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
@@ -149,6 +150,24 @@ def gemv(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
     _check("nvq_gemv", _lib.nvq_gemv(
         _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y),
         _stream(stream)))
+    return y
+
+
+def quant_gemv_supported(K: int) -> bool:
+    """Whether nvq_quant_gemv handles this K (asked of the library with an
+    empty product, which launches nothing)."""
+    return _lib.nvq_quant_gemv(None, None, 1.0, 0, K, None, None, None) == NVQ_OK
+
+
+def quant_gemv(codes: torch.Tensor, scales: torch.Tensor, g: float, x: torch.Tensor,
+               y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Q8_0 of one fp32 token fused into the decode GEMV: y[1, N] fp32."""
+    N = codes.shape[0]
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check("nvq_quant_gemv", _lib.nvq_quant_gemv(
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(x), _ptr(y), _stream(stream)))
     return y
 
 

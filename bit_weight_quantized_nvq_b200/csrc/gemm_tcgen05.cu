@@ -267,7 +267,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     // ------------------------------ MMA issuer --------------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_f16_f32(kBN, 2 * kBT);
-      bool ok = true;
       for (int kb = 0; kb < num_kb; ++kb) {
         const int s = kb % kStages;
         const uint32_t ph = (kb / kStages) & 1;
@@ -278,13 +277,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
         if (first && c >= 2 &&
             !ptx::mbar_wait_bounded(acc_empty(b), ((c >> 1) - 1) & 1, abort_flag, kWaitLimitNs)) {
           fail();
-          ok = false;
           break;
         }
         if (!ptx::mbar_wait_bounded(full_a(s), ph, abort_flag, kWaitLimitNs) ||
             !ptx::mbar_wait_bounded(full_b(s), ph, abort_flag, kWaitLimitNs)) {
           fail();
-          ok = false;
           break;
         }
         ptx::tc_fence_after();
@@ -299,7 +296,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
         ptx::mma_commit(empty(s));
         if ((kb % kChunk) == kChunk - 1 || kb == num_kb - 1) ptx::mma_commit(acc_full(b));
       }
-      (void)ok;
       // no MMA may still be writing TMEM when it is released
       ptx::mma_commit(mma_done);
       ptx::mbar_wait_bounded(mma_done, 0, nullptr, kWaitLimitNs);

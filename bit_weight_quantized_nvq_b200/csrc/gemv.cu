@@ -34,7 +34,8 @@
 //    to the +12-biased integer LUT of the "Bias trick" paragraph (9
 //    operations per 8 codes instead of 11) and the bias is removed by
 //    starting each subblock's dp4a chain at corr = -12 * bsum16, precomputed
-//    per activation subblock.  The chunk loop is fully unrolled for 4 or 5
+//    per activation subblock.  (The register schedule below goes further and
+//    feeds both table halves to dp4a instead of OR-merging them.)  The chunk loop is fully unrolled for 4 or 5
 //    chunks per lane so all shared-memory loads of a stage are in flight
 //    together.  The consumers are instruction-bound, so these savings matter.
 //  * gemv_tma_kernel (K % 256 == 0, every workload shape): persistent CTAs,
@@ -290,13 +291,22 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
 // ---------------------------------------------------------------------------
 // Every lane of a consumer warp handles the same NPL chunk positions of
 // every row it ever processes, so the activation data of those chunks (32
-// codes, d and the two bias corrections) is loaded once into registers for
-// the whole kernel.  A row is split across WPR warps (warp part p owns the
-// p-th contiguous K segment of 1024 * NPL elements); a stage is R = 16/WPR
-// (or fewer, to fit 46 KB) whole, contiguous rows, fetched with two bulk
-// copies.  With WPR > 1 each warp leaves its row partial in shared memory
-// (one slot per stage) and the producer thread adds the WPR partials in a
-// fixed order when it recycles the stage, so results are deterministic.
+// codes, d and the two bias corrections) is loaded once into registers and
+// held there for the whole kernel.  With XF32 the kernel takes the fp32
+// activations instead and performs the Q8_0 quantisation itself, once per
+// CTA into shared memory (the same IEEE operations as
+// nvq_quantize_act_q8_0, so the codes are identical); every CTA repeats
+// that work, so it pays off only where a launch costs more than it.
+// A row is split across WPR warps (warp part p owns the p-th contiguous K
+// segment of 1024 * NPL elements); a stage is R = 16/WPR (or fewer, to fit
+// 46 KB) whole, contiguous rows, fetched with two bulk copies.  With
+// WPR > 1 each warp leaves its row partial in shared memory (one slot per
+// stage) and the producer thread adds the WPR partials in a fixed order when
+// it recycles the stage, so results are deterministic.
+// The kernel is launched with programmatic stream serialisation: it lets
+// the next kernel of the stream launch early and waits for the previous
+// one (griddepcontrol) before it reads any global input, so launch latency
+// and prologue overlap the previous kernel's tail without changing results.
 constexpr uint32_t kRegStageMax = 46080;
 
 __host__ __device__ constexpr int reg_rows(int K, int wpr) {
@@ -304,24 +314,84 @@ __host__ __device__ constexpr int reg_rows(int K, int wpr) {
   while (r > 1 && static_cast<uint32_t>(r) * (K / 2 + K / 16) > kRegStageMax) --r;
   return r;
 }
+// stages | row partials [stage][warp] | activation words [K/32][8] |
+// ActMeta [K/32] | barriers
 __host__ __device__ constexpr uint32_t reg_smem_bytes(int K, int wpr) {
   return kM1Stages * static_cast<uint32_t>(reg_rows(K, wpr)) * (K / 2 + K / 16) +
-         kM1Stages * kM1Consumers * 4 + 2 * kM1Stages * 8 + 16;
+         kM1Stages * kM1Consumers * 4 + static_cast<uint32_t>(K / 32) * 48 +
+         2 * kM1Stages * 8 + 16;
 }
 
-template <int NPL, int WPR>
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Stage chunk c of the activation vector: lane j (0..7) of a group of eight
+// handles elements 4j..4j+3, i.e. word j of the chunk's 32 codes.  With
+// XF32 the codes are quantised here exactly as the Q8_0 quantiser does
+// (amax over the block by shuffles, IEEE divisions, rint, clamp, fp16 d).
+template <bool XF32>
+__device__ __forceinline__ void stage_act_chunk(int c, int j, unsigned gmask,
+                                                const float* __restrict__ x,
+                                                const int8_t* __restrict__ q,
+                                                const __half* __restrict__ d,
+                                                uint32_t* words, ActMeta* meta) {
+  uint32_t word;
+  float dval;
+  if constexpr (XF32) {
+    const float4 v = reinterpret_cast<const float4*>(x)[8 * c + j];
+    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    a = fmaxf(a, __shfl_xor_sync(gmask, a, 1, 8));
+    a = fmaxf(a, __shfl_xor_sync(gmask, a, 2, 8));
+    a = fmaxf(a, __shfl_xor_sync(gmask, a, 4, 8));
+    const float d32 = __fdiv_rn(a, 127.0f);
+    word = 0;
+    if (d32 > 0.0f) {
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        int qi = __float2int_rn(__fdiv_rn(e[i], d32));
+        qi = max(-127, min(127, qi));
+        word |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * i);
+      }
+    }
+    dval = __half2float(__float2half_rn(d32));
+  } else {
+    word = reinterpret_cast<const uint32_t*>(q)[8 * c + j];
+    dval = __half2float(d[c]);
+  }
+  int s = dev::dp4a(word, 0x01010101u, 0);
+  s += __shfl_xor_sync(gmask, s, 1, 8);
+  s += __shfl_xor_sync(gmask, s, 2, 8);   // lanes 0-3: subblock 0, lanes 4-7: subblock 1
+  words[8 * c + j] = word;
+  if (j == 0) {
+    meta[c].d = dval;
+    meta[c].corr0 = -12 * s;
+    meta[c].pad = 0;
+  }
+  if (j == 4) meta[c].corr1 = -12 * s;
+}
+
+template <int NPL, int WPR, bool XF32>
 __global__ void __launch_bounds__(kM1Threads, 1)
 gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                   float half_g, int N, int K, const int8_t* __restrict__ q,
-                   const __half* __restrict__ d, float* __restrict__ y) {
+                   float half_g, int N, int K, const float* __restrict__ x,
+                   const int8_t* __restrict__ q, const __half* __restrict__ d,
+                   float* __restrict__ y) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int R = reg_rows(K, WPR);
   const int active = R * WPR;                      // consumer warps in use
+  const int nchunk = K / 32;
   const uint32_t row_code = K / 2, row_scale = K / 16;
   const uint32_t stage_bytes = static_cast<uint32_t>(R) * (row_code + row_scale);
   const uint32_t codes_bytes = static_cast<uint32_t>(R) * row_code;
   float* part = reinterpret_cast<float*>(smem + kM1Stages * stage_bytes);  // [stage][warp]
-  uint64_t* full = reinterpret_cast<uint64_t*>(part + kM1Stages * kM1Consumers);
+  uint32_t* act_words = reinterpret_cast<uint32_t*>(part + kM1Stages * kM1Consumers);
+  ActMeta* meta = reinterpret_cast<ActMeta*>(act_words + 8 * nchunk);
+  uint64_t* full = reinterpret_cast<uint64_t*>(meta + nchunk);
   uint64_t* empty = full + kM1Stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kM1Stages);
 
@@ -332,6 +402,7 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
   const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
   const int total = (r_end - r_begin + R - 1) / R;   // stages = row groups
 
+  grid_dependents_launch();
   if (threadIdx.x == 0) {
     for (int i = 0; i < kM1Stages; ++i) {
       ptx::mbar_init(ptx::smem_addr(full + i), 1);
@@ -341,6 +412,7 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  grid_dependency_wait();   // inputs written by the previous kernel are visible
 
   if (warp == kM1Consumers) {
     // ------------- producer: bulk copies, and the sum of row partials --------
@@ -398,7 +470,6 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
     }
     return;
   }
-  if (warp >= active) return;
 
   // ------------- consumers: warp w = (row w / WPR, part w % WPR) -------------
   const int rl = warp / WPR;
@@ -406,19 +477,42 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
   uint4 qa[NPL], qb[NPL];
   float dd[NPL];
   int c0[NPL], c1[NPL];
+  if constexpr (XF32) {
+    // quantise the fp32 token once per CTA into shared memory (all 16 warps)
+    const unsigned gmask = 0xFFu << (lane & 24);
+    for (int cb = warp * 4; cb < nchunk; cb += kM1Consumers * 4) {
+      const int c = cb + (lane >> 3);
+      if (c < nchunk) stage_act_chunk<true>(c, lane & 7, gmask, x, q, d, act_words, meta);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kM1Consumers * 32) : "memory");
+    if (warp >= active) return;
 #pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    const int c = p * (NPL * 32) + lane + 32 * i;   // chunk index in the row
-    const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * c;
-    qa[i] = __ldg(src);
-    qb[i] = __ldg(src + 1);
-    dd[i] = __half2float(__ldg(d + c));
-    const int s0 = dev::dp4a(qa[i].x, 0x01010101u, dev::dp4a(qa[i].y, 0x01010101u,
-                   dev::dp4a(qa[i].z, 0x01010101u, dev::dp4a(qa[i].w, 0x01010101u, 0))));
-    const int s1 = dev::dp4a(qb[i].x, 0x01010101u, dev::dp4a(qb[i].y, 0x01010101u,
-                   dev::dp4a(qb[i].z, 0x01010101u, dev::dp4a(qb[i].w, 0x01010101u, 0))));
-    c0[i] = -12 * s0;
-    c1[i] = -12 * s1;
+    for (int i = 0; i < NPL; ++i) {
+      const int c = p * (NPL * 32) + lane + 32 * i;   // chunk index in the row
+      qa[i] = reinterpret_cast<const uint4*>(act_words)[2 * c];
+      qb[i] = reinterpret_cast<const uint4*>(act_words)[2 * c + 1];
+      const ActMeta mt = meta[c];
+      dd[i] = mt.d;
+      c0[i] = mt.corr0;
+      c1[i] = mt.corr1;
+    }
+  } else {
+    // Q8_0 input: each lane loads its own chunks straight into registers
+    if (warp >= active) return;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int c = p * (NPL * 32) + lane + 32 * i;
+      const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * c;
+      qa[i] = __ldg(src);
+      qb[i] = __ldg(src + 1);
+      dd[i] = __half2float(__ldg(d + c));
+      const int s0 = dev::dp4a(qa[i].x, 0x01010101u, dev::dp4a(qa[i].y, 0x01010101u,
+                     dev::dp4a(qa[i].z, 0x01010101u, dev::dp4a(qa[i].w, 0x01010101u, 0))));
+      const int s1 = dev::dp4a(qb[i].x, 0x01010101u, dev::dp4a(qb[i].y, 0x01010101u,
+                     dev::dp4a(qb[i].z, 0x01010101u, dev::dp4a(qb[i].w, 0x01010101u, 0))));
+      c0[i] = -12 * s0;
+      c1[i] = -12 * s1;
+    }
   }
   for (int it = 0; it < total; ++it) {
     const int s = it % kM1Stages;
@@ -445,15 +539,8 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
       }
 #pragma unroll
       for (int i = 0; i < NPL; ++i) {
-        uint32_t cb[8];
-        dev::decode_e2m1x8_biased(w[i].x, cb[0], cb[1]);
-        dev::decode_e2m1x8_biased(w[i].y, cb[2], cb[3]);
-        dev::decode_e2m1x8_biased(w[i].z, cb[4], cb[5]);
-        dev::decode_e2m1x8_biased(w[i].w, cb[6], cb[7]);
-        const int i0 = dev::dp4a_us(cb[0], qa[i].x, dev::dp4a_us(cb[1], qa[i].y,
-                       dev::dp4a_us(cb[2], qa[i].z, dev::dp4a_us(cb[3], qa[i].w, c0[i]))));
-        const int i1 = dev::dp4a_us(cb[4], qb[i].x, dev::dp4a_us(cb[5], qb[i].y,
-                       dev::dp4a_us(cb[6], qb[i].z, dev::dp4a_us(cb[7], qb[i].w, c1[i]))));
+        const int i0 = dev::dot16_biased(w[i].x, w[i].y, qa[i], c0[i]);
+        const int i1 = dev::dot16_biased(w[i].z, w[i].w, qb[i], c1[i]);
         const float2 sf = dev::ue4m3x2_to_float2(s2[i]);
         acc = fmaf(dd[i], fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
       }
@@ -715,47 +802,58 @@ cudaError_t launch_m1(const uint8_t* codes, const uint8_t* scales, float g, int6
   return cudaGetLastError();
 }
 
-template <int NPL, int WPR>
+template <int NPL, int WPR, bool XF32>
 cudaError_t launch_m1_reg(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
-                          int64_t K, const int8_t* q, const uint16_t* d, float* y,
-                          cudaStream_t stream) {
+                          int64_t K, const float* x, const int8_t* q, const uint16_t* d,
+                          float* y, cudaStream_t stream) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
+  auto kernel = gemv_m1_reg_kernel<NPL, WPR, XF32>;
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_m1_reg_kernel<NPL, WPR>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSmemPerCtaMax));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const int64_t ctas = std::min<int64_t>(device_sm_count(), N);
-  gemv_m1_reg_kernel<NPL, WPR><<<static_cast<unsigned>(ctas), kM1Threads,
-                                 reg_smem_bytes(static_cast<int>(K), WPR), stream>>>(
-      codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), q,
-      reinterpret_cast<const __half*>(d), y);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+  cfg.blockDim = dim3(kM1Threads);
+  cfg.dynamicSmemBytes = reg_smem_bytes(static_cast<int>(K), WPR);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, codes, scales, 0.5f * g, static_cast<int>(N),
+                            static_cast<int>(K), x, q, reinterpret_cast<const __half*>(d), y);
 }
 
 // The register schedule covers K = 1024 * NPL * WPR for the (NPL, WPR) pairs
 // instantiated here; returns cudaErrorNotSupported for other K.
+template <bool XF32>
 cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, float g,
-                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
-                                   float* y, cudaStream_t stream) {
+                                   int64_t N, int64_t K, const float* x, const int8_t* q,
+                                   const uint16_t* d, float* y, cudaStream_t stream) {
   if (K % 1024 != 0) return cudaErrorNotSupported;
+#define NVQ_REG(npl, wpr) \
+  return launch_m1_reg<npl, wpr, XF32>(codes, scales, g, N, K, x, q, d, y, stream)
   switch (K / 1024) {
-    case 4: return launch_m1_reg<4, 1>(codes, scales, g, N, K, q, d, y, stream);
-    case 5: return launch_m1_reg<5, 1>(codes, scales, g, N, K, q, d, y, stream);
-    case 6: return launch_m1_reg<6, 1>(codes, scales, g, N, K, q, d, y, stream);
-    case 8: return launch_m1_reg<4, 2>(codes, scales, g, N, K, q, d, y, stream);
-    case 10: return launch_m1_reg<5, 2>(codes, scales, g, N, K, q, d, y, stream);
-    case 12: return launch_m1_reg<6, 2>(codes, scales, g, N, K, q, d, y, stream);
-    case 15: return launch_m1_reg<5, 3>(codes, scales, g, N, K, q, d, y, stream);
-    case 16: return launch_m1_reg<4, 4>(codes, scales, g, N, K, q, d, y, stream);
-    case 20: return launch_m1_reg<5, 4>(codes, scales, g, N, K, q, d, y, stream);
-    case 25: return launch_m1_reg<5, 5>(codes, scales, g, N, K, q, d, y, stream);
+    case 4: NVQ_REG(4, 1);
+    case 5: NVQ_REG(5, 1);
+    case 6: NVQ_REG(6, 1);
+    case 8: NVQ_REG(4, 2);
+    case 10: NVQ_REG(5, 2);
+    case 12: NVQ_REG(6, 2);
+    case 15: NVQ_REG(5, 3);
+    case 16: NVQ_REG(4, 4);
+    case 20: NVQ_REG(5, 4);
+    case 25: NVQ_REG(5, 5);
     default: return cudaErrorNotSupported;
   }
+#undef NVQ_REG
 }
 
 template <int MT>
@@ -764,7 +862,8 @@ cudaError_t launch_gemv_m(const uint8_t* codes, const uint8_t* scales, float g,
                           float* y, cudaStream_t stream) {
   const int seg = tma_segment(K);
   if (MT == 1) {
-    const cudaError_t e = launch_m1_reg_dispatch(codes, scales, g, N, K, q, d, y, stream);
+    const cudaError_t e =
+        launch_m1_reg_dispatch<false>(codes, scales, g, N, K, nullptr, q, d, y, stream);
     if (e != cudaErrorNotSupported) return e;
   }
   if (MT == 1 && seg > 0 && m1_smem_bytes(static_cast<int>(K), seg) <= kSmemPerCtaMax) {
@@ -812,6 +911,22 @@ cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
 #undef NVQ_GEMV_CASE
     default: return cudaErrorInvalidValue;
   }
+}
+
+bool quant_gemv_supported(int64_t K) {
+  if (K % 1024 != 0) return false;
+  switch (K / 1024) {
+    case 4: case 5: case 6: case 8: case 10: case 12: case 15: case 16: case 20: case 25:
+      return true;
+    default:
+      return false;
+  }
+}
+
+cudaError_t launch_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                              int64_t N, int64_t K, const float* x, float* y,
+                              cudaStream_t stream) {
+  return launch_m1_reg_dispatch<true>(codes, scales, g, N, K, x, nullptr, nullptr, y, stream);
 }
 
 unsigned int gemv_error_flags(bool clear) {

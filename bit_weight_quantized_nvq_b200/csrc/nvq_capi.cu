@@ -5,7 +5,7 @@
 
 #include <cuda_runtime.h>
 
-#include "../../include/nvq.h"
+#include "nvq.h"
 #include "nvq_internal.h"
 
 namespace {
@@ -135,6 +135,20 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
   if (st != NVQ_OK) return st;
   return cuda_status(nvq::launch_gemv(codes, scales, g, N, K, q, d, M, y,
                                       static_cast<cudaStream_t>(stream)));
+}
+
+nvq_status nvq_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                          int64_t N, int64_t K, const float* x, float* y, void* stream) {
+  // x plays the part of q (checked for NULL and alignment); d is not used
+  nvq_status st = check_dot_args(codes, scales, N, K, x, x, 1, y, 1, 1, true);
+  if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
+  if (!nvq::quant_gemv_supported(K)) return NVQ_ERR_BAD_SHAPE;
+  if (N == 0) return NVQ_OK;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_quant_gemv(codes, scales, g, N, K, x, y,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {

@@ -79,6 +79,26 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   return r;
 }
 
+// Integer sum of one 16-element subblock, sum((c + 12) * q) + corr, from its
+// two code words and four activation words.  The two lookups of each group
+// of four codes (positive and negative table half, each zero where the
+// other applies) go to dp4a separately instead of being OR-merged: this
+// moves work from the integer ALU pipe, which limits the decode GEMV, to the
+// dp4a pipe (measured +6 % on the decode sweep, +8 % on the largest shape).
+__device__ __forceinline__ int dot16_biased(uint32_t w0, uint32_t w1, const uint4 q, int corr) {
+  const uint32_t n0 = w0 ^ 0x88888888u, n1 = w1 ^ 0x88888888u;
+  int a = corr;
+  a = dp4a_us(prmt_sr(kBiasPosLo, kBiasPosHi, w0), q.x, a);
+  a = dp4a_us(prmt_sr(kBiasNegLo, kBiasNegHi, n0), q.x, a);
+  a = dp4a_us(prmt_sr(kBiasPosLo, kBiasPosHi, w0 >> 16), q.y, a);
+  a = dp4a_us(prmt_sr(kBiasNegLo, kBiasNegHi, n0 >> 16), q.y, a);
+  a = dp4a_us(prmt_sr(kBiasPosLo, kBiasPosHi, w1), q.z, a);
+  a = dp4a_us(prmt_sr(kBiasNegLo, kBiasNegHi, n1), q.z, a);
+  a = dp4a_us(prmt_sr(kBiasPosLo, kBiasPosHi, w1 >> 16), q.w, a);
+  a = dp4a_us(prmt_sr(kBiasNegLo, kBiasNegHi, n1 >> 16), q.w, a);
+  return a;
+}
+
 // Two UE4M3 scale bytes (low byte = first subblock) to fp32, exactly.  UE4M3
 // is E4M3 with the sign bit 0, so the hardware E4M3 -> f16 conversion
 // applies; every UE4M3 value (2^-9 .. 448) is exact in fp16.

@@ -19,6 +19,13 @@ cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                         const uint16_t* d, int64_t M, float* y,
                         cudaStream_t stream);
 
+// Q8_0 quantisation of one fp32 token fused into the decode GEMV (M = 1);
+// supported for K = 1024 * T, T in {4, 5, 6, 8, 10, 12, 15, 16, 20, 25}.
+bool quant_gemv_supported(int64_t K);
+cudaError_t launch_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                              int64_t N, int64_t K, const float* x, float* y,
+                              cudaStream_t stream);
+
 // Error flags raised by GEMV kernels (bit 0: a pipeline wait timed out);
 // synchronous read, optionally clearing them.
 unsigned int gemv_error_flags(bool clear);

@@ -22,7 +22,7 @@
 #include <thread>
 #include <vector>
 
-#include "../../include/nvq.h"
+#include "nvq.h"
 
 namespace {
 

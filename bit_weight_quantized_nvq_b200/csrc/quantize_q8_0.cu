@@ -12,7 +12,8 @@
 // four consecutive blocks with fully coalesced 512-byte loads and 128-byte
 // code stores; the block amax is reduced with three shuffles inside each
 // group of eight lanes.  The kernel is HBM-bound: 4 + 1 + 2/32 bytes per
-// element.
+// element.  It is launched with programmatic stream serialisation (see the
+// decode GEMV), so at one token its launch overlaps the previous kernel.
 #include <cuda_fp16.h>
 
 #include "nvq_device.cuh"
@@ -26,6 +27,10 @@ constexpr int kThreads = 256;
 __global__ void __launch_bounds__(kThreads)
 quantize_q8_0_kernel(const float4* __restrict__ x, int64_t nblocks,
                      uint32_t* __restrict__ q, __half* __restrict__ d) {
+  // programmatic dependent launch: let the next kernel launch early, and
+  // read x only once the kernel that wrote it has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
   const int64_t b = t >> 3;
   if (b >= nblocks) return;  // whole groups of eight leave together
@@ -61,10 +66,17 @@ cudaError_t launch_quantize_q8_0(const float* x, int64_t M, int64_t K,
   if (nblocks == 0) return cudaSuccess;
   const int64_t threads = nblocks * 8;
   const int64_t grid = (threads + kThreads - 1) / kThreads;
-  quantize_q8_0_kernel<<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(
-      reinterpret_cast<const float4*>(x), nblocks, reinterpret_cast<uint32_t*>(q),
-      reinterpret_cast<__half*>(d));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_q8_0_kernel, reinterpret_cast<const float4*>(x),
+                            nblocks, reinterpret_cast<uint32_t*>(q), reinterpret_cast<__half*>(d));
 }
 
 }  // namespace nvq

@@ -135,6 +135,22 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                     int64_t M, float* y, void* stream);
 
 /*
+ * nvq_quant_gemv - decode GEMV of one fp32 token with its Q8_0 quantisation
+ * fused in: y[1, N] = Q8_0(x)[1, K] . W[N, K]^T.
+ *
+ * x  device float [1, K] (finite).  The kernel quantises x exactly as
+ * nvq_quantize_act_q8_0 does (same IEEE operations, so the codes and scales
+ * are identical) and then runs the nvq_gemv product, so y is bit-identical
+ * to nvq_quantize_act_q8_0 followed by nvq_gemv; it saves one launch and
+ * one round trip of the activations.  Supported for K = 1024 * T with T in
+ * {4, 5, 6, 8, 10, 12, 15, 16, 20, 25} (NVQ_ERR_BAD_SHAPE otherwise).
+ * Errors: as nvq_gemv.
+ */
+nvq_status nvq_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                          int64_t N, int64_t K, const float* x, float* y,
+                          void* stream);
+
+/*
  * nvq_gemm_workspace_size - bytes of device workspace nvq_gemm needs for
  * M tokens of K features (0 when M == 0).  It holds the activations
  * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q.

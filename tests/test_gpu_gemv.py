@@ -135,3 +135,32 @@ def test_error_status_on_device():
     with pytest.raises(capi.NVQError) as e:
         capi.gemv(codes, scales, 1.0, q, d)
     assert e.value.status == capi.NVQ_ERR_BAD_SHAPE
+
+
+@pytest.mark.parametrize("K,N", [(4096, 1000), (5120, 1537), (25600, 700), (10240, 301),
+                                 (6144, 257), (5120, 152064)])
+def test_fused_quant_gemv_is_bit_identical_and_within_tolerance(K, N):
+    W = wl.weights("gemv_test", "Wf", N, K, boost_columns=True)
+    x = wl.activations("gemv_test", "xf", 1, K, "student_t4")
+    x[0, :32] = 0.0                               # a zero block (d = 0)
+    rows = sample_rows(N, 300, seed=K + N) if N > 2000 else None
+    P = Packed(W, rows)
+    xd = torch.from_numpy(x).cuda()
+    y_f = capi.quant_gemv(P.codes, P.scales, P.g, xd)
+    q, d = capi.quantize_act_q8_0(xd)
+    y_u = capi.gemv(P.codes, P.scales, P.g, q, d)
+    torch.cuda.synchronize()
+    assert torch.equal(y_f, y_u)
+    q_ref, d_ref = o.quantize_q8_0(x)
+    y_ref, sa, _ = reference(P, q_ref, d_ref)
+    y = y_f.cpu().numpy()
+    assert_within_tolerance(y if rows is None else y[:, rows], y_ref, sa)
+
+
+def test_fused_quant_gemv_rejects_unsupported_k():
+    codes = torch.zeros((4, 1088 // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((4, 1088 // 16), dtype=torch.uint8, device="cuda")
+    x = torch.zeros((1, 1088), device="cuda")
+    with pytest.raises(capi.NVQError) as e:
+        capi.quant_gemv(codes, scales, 1.0, x)
+    assert e.value.status == capi.NVQ_ERR_BAD_SHAPE
