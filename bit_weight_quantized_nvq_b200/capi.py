@@ -48,6 +48,8 @@ SIGNATURES = {
     "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
+    "nvq_gemm_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
+                                        _c_i64, _vp, _vp]),
     "nvq_debug_subblock_sums": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _vp,
                                                _vp]),
     "nvq_decoder_stack": (ctypes.c_int, [ctypes.POINTER(Linear), _c_i64, _vp, _c_i64,
@@ -189,6 +191,20 @@ def gemm(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
     _check("nvq_gemm", _lib.nvq_gemm(
         _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y),
         _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return y
+
+
+def gemm_noalloc(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
+                 d: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Prefill GEMM with the library's own 64 MiB device scratch instead of a
+    caller workspace (nvq_gemm_noalloc): y[M, N] fp32."""
+    N = codes.shape[0]
+    M, K = q.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=q.device)
+    _check("nvq_gemm_noalloc", _lib.nvq_gemm_noalloc(
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y),
         _stream(stream)))
     return y
 

@@ -45,6 +45,7 @@
 //     Every wait is bounded (4 s); a timeout raises an error flag and the
 //     CTA drains what it issued, frees TMEM and exits.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -411,6 +412,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   }
 }
 
+// Scratch of nvq_gemm_noalloc: the expanded activations [2 * M_pad, K] fp16
+// and the M_pad token scales of one call, in device memory that the library
+// itself owns (a file-scope array exists on every GPU that loads the library,
+// from module load until the process exits), so that the call needs no
+// allocation and no workspace from its caller.
+constexpr size_t kNoAllocScratchBytes = size_t{64} << 20;   // 64 MiB
+static __device__ __align__(256) unsigned char g_gemm_noalloc_scratch[kNoAllocScratchBytes];
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -432,6 +441,34 @@ int64_t padded_tokens(int64_t M) { return (M + kBT - 1) / kBT * kBT; }
 size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
   const int64_t mp = padded_tokens(M);
   return static_cast<size_t>(4 * mp * K + 4 * mp);
+}
+
+size_t gemm_noalloc_limit() { return kNoAllocScratchBytes; }
+
+// The scratch array's device address on the current device.  Host code may
+// not use the array's name as an address (it names a host-side shadow), so
+// the address is looked up with cudaGetSymbolAddress, once per device with
+// that device current, and cached.
+cudaError_t gemm_noalloc_scratch(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<void*> cache[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(mu);
+    p = cache[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      e = cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch);
+      if (e != cudaSuccess) return e;
+      cache[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return cudaSuccess;
 }
 
 unsigned int gemm_error_flags(bool clear) {

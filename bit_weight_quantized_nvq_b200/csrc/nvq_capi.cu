@@ -174,6 +174,27 @@ nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
                                       static_cast<cudaStream_t>(stream)));
 }
 
+nvq_status nvq_gemm_noalloc(const uint8_t* codes, const uint8_t* scales, float g,
+                            int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                            int64_t M, float* y, void* stream) {
+  nvq_status st = check_dot_args(codes, scales, N, K, q, d, M, y, 1,
+                                 int64_t{1} << 24, true);
+  if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
+  if (N == 0 || M == 0) return NVQ_OK;
+  if (nvq::gemm_workspace_size(M, N, K) > nvq::gemm_noalloc_limit()) return NVQ_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  void* scratch = nullptr;
+  cudaError_t e = nvq::gemm_noalloc_scratch(&scratch);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  return cuda_status(nvq::launch_gemm(codes, scales, g, N, K, q, d, M, y, scratch,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 nvq_status nvq_debug_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
                                    const int8_t* q, int64_t M, int32_t* isum,
                                    void* stream) {

@@ -50,6 +50,12 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
                       int64_t K, int64_t M, float* y, const void* workspace,
                       cudaStream_t stream);
 
+// The allocation-free GEMM: bytes of its library-owned scratch, and the
+// scratch's device address on the current device (looked up once per
+// device, on first use).
+size_t gemm_noalloc_limit();
+cudaError_t gemm_noalloc_scratch(void** out);
+
 // Error flags raised by the GEMM kernel (bit 0: a pipeline wait timed out).
 unsigned int gemm_error_flags(bool clear);
 

@@ -177,6 +177,40 @@ nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
                     size_t workspace_bytes, void* stream);
 
 /*
+ * nvq_gemm_noalloc - nvq_gemm for callers that cannot allocate device memory
+ * and cannot hand the library a workspace.  (An addition of this library;
+ * the web pages describing the method have no counterpart.)
+ *
+ * Some callers may not allocate: code that runs inside a host framework
+ * which owns every device allocation (through its own pool or arena) and
+ * gives its plugins no scratch, and latency-critical serving loops that must
+ * not call cudaMalloc, which can synchronise the device and fragment memory.
+ * This entry point needs neither: it keeps the GEMM's scratch (the expanded
+ * activations) in a 64 MiB array of device memory that the library itself
+ * holds on every GPU that loads it, from load until the process exits.  It
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Arguments, layouts, result and accuracy are those of nvq_gemm (y is the
+ * same); there is no workspace argument.  Limit: the problem must fit the
+ * scratch, nvq_gemm_workspace_size(M, N, K) <= 64 MiB, i.e. roughly
+ * 4 * ceil(M/128)*128 * K bytes (for example M = 2048 up to K = 8160, or
+ * M = 256 up to K = 65280); larger problems return NVQ_ERR_WORKSPACE and
+ * should use nvq_gemm with a caller workspace.
+ * Set-up: the first call on a device looks up the scratch's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ * Sharing: every call, on every stream and host thread, uses the same
+ * array, so calls whose work overlaps on the GPU race and corrupt each
+ * other's results; serialise them (one stream, or events).  The array keeps
+ * the last call's contents; nothing in it needs to start at zero, since
+ * each call writes every byte it reads before reading it.
+ * Errors: as nvq_gemm, with NVQ_ERR_WORKSPACE for problems over the limit.
+ */
+nvq_status nvq_gemm_noalloc(const uint8_t* codes, const uint8_t* scales, float g,
+                            int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                            int64_t M, float* y, void* stream);
+
+/*
  * nvq_debug_subblock_sums - the integer per-16 subblock sums the GEMV forms,
  * exported for bit-exact checking:
  * isum[m, n, sb] = sum_{k in sb} (2*E2M1(code[n,k])) * q[m,k], int32
