@@ -29,19 +29,20 @@
 //     caller's workspace, once per call (tokens padded to 128 with zeros).
 //     A token whose largest |d*q| would overflow fp16 (|x| > 65504) is
 //     scaled by 2^-e first and the epilogue multiplies by 2^e.
-//  2. gemm_kernel: one CTA per 128 weight rows x 128 tokens, 6 warps:
+//  2. gemm_kernel: one CTA per 128 weight rows x 128 tokens, 10 warps:
 //       warp 0    TMA producer: [hi; lo] activation tiles (2 x 128 rows x 64
 //                 fp16, 128-byte swizzle) into a 4-stage ring;
 //       warp 1    allocates 512 TMEM columns (two 256-column accumulators);
 //                 one thread issues tcgen05.mma (M=128, N=256, K=16) x 4
 //                 per stage, commits each stage back to the producers and
 //                 each finished 8-stage chunk to the draining threads;
-//       warps 2-5 one thread per weight row: cp.async the row's 32 code
-//                 bytes and 4 scale bytes for each stage, decode 64 codes
-//                 to fp16 w' with byte permutes and write them in the
-//                 128-byte swizzle layout; drain finished chunks (tcgen05.ld
-//                 of the hi and lo columns into 128 fp32 registers); the
-//                 epilogue scales and stores the registers.
+//       warps 2-9 two threads per weight row (two warps per scheduler, so
+//                 each hides the other's latency): cp.async the half row's
+//                 16 code bytes and the row's 4 scale bytes for each stage,
+//                 decode 32 codes to fp16 w' with byte permutes and write them
+//                 in the 128-byte swizzle layout; drain finished chunks
+//                 (tcgen05.ld of half the hi and lo columns into 64 fp32
+//                 registers); the epilogue scales and stores the registers.
 //     Every wait is bounded (4 s); a timeout raises an error flag and the
 //     CTA drains what it issued, frees TMEM and exits.
 #include <algorithm>
@@ -63,7 +64,8 @@ constexpr int kBN = 128;            // weight rows per tile = MMA M = TMEM lanes
 constexpr int kBT = 128;            // tokens per tile; MMA N = 2 * kBT ([hi; lo])
 constexpr int kBK = 64;             // K per stage: one 128-byte fp16 swizzle row
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kExpThreads = 256;     // weight expansion + epilogue: 2 per row
+constexpr int kThreads = 64 + kExpThreads;
 constexpr int kChunk = 8;           // K stages accumulated per TMEM buffer
 constexpr uint32_t kAccCols = 2 * kBT;        // one [hi | lo] accumulator
 constexpr uint32_t kTmemCols = 2 * kAccCols;  // two accumulators
@@ -72,7 +74,7 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint32_t kAStageBytes = kBN * kBK * 2;        // 16 KB of w'
 constexpr uint32_t kBStageBytes = 2 * kBT * kBK * 2;    // 32 KB of [hi; lo]
 constexpr uint32_t kCodeStageBytes = kBN * kBK / 2;     // 4 KB of codes
-constexpr uint32_t kScaleStageBytes = kBN * kBK / 16;   // 512 B of scales
+constexpr uint32_t kScaleStageBytes = kBN * 8;         // 4 scale bytes per half row
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kAStageBytes;
 constexpr uint32_t kOffCodes = kOffB + kStages * kBStageBytes;
@@ -215,13 +217,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(full_a(s), kBN);
+      ptx::mbar_init(full_a(s), kExpThreads);
       ptx::mbar_init(full_b(s), 1);
       ptx::mbar_init(empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(acc_full(b), 1);
-      ptx::mbar_init(acc_empty(b), kBN);
+      ptx::mbar_init(acc_empty(b), kExpThreads);
     }
     ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -303,46 +305,54 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     }
   } else {
     // ------------------- weight expansion, then the epilogue ------------------
-    const int t = threadIdx.x - 64;   // 0..127: row of the tile
-    const int row = n0 + t;
+    // Two threads per weight row (warps 2-5: first half of the 64-wide K
+    // slice, warps 6-9: second half).  In the epilogue the warp pair that
+    // shares a TMEM lane quarter splits the 128 token columns.
+    const int t = threadIdx.x - 64;         // 0..255
+    const int rt = t & (kBN - 1);           // row of the tile
+    const int h = t >> 7;                   // half of the K slice
+    const int row = n0 + rt;
     const bool valid = row < N;
-    const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2);
+    const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2) + 16 * h;
     const uint8_t* srow = scales + static_cast<size_t>(valid ? row : 0) * (K / 16);
-    const uint32_t stg_c = sbase + kOffCodes + 32u * t;
-    const uint32_t stg_s = sbase + kOffScales + 4u * t;
+    const uint32_t stg_c = sbase + kOffCodes + 32u * rt + 16u * h;
+    const uint32_t stg_s = sbase + kOffScales + 8u * rt + 4u * h;
     auto issue = [&](int kb) {
       if (kb < num_kb) {
         const uint32_t slot = kb % kStages;
-        const uint32_t nb = valid ? 16u : 0u;
-        ptx::cp_async_16(stg_c + slot * kCodeStageBytes, crow + 32 * kb, nb);
-        ptx::cp_async_16(stg_c + slot * kCodeStageBytes + 16, crow + 32 * kb + 16, nb);
+        ptx::cp_async_16(stg_c + slot * kCodeStageBytes, crow + 32 * kb, valid ? 16u : 0u);
         ptx::cp_async_4(stg_s + slot * kScaleStageBytes, srow + 4 * kb, valid ? 4u : 0u);
       }
       ptx::cp_async_commit();
     };
     for (int i = 0; i < kStages - 1; ++i) issue(i);
     bool ok = true;
-    const uint32_t sw = t & 7;
+    const uint32_t sw = rt & 7;
     const int quarter = warp & 3;            // TMEM lanes this warp may read
+    const int col_half = (warp - 2) >> 2;    // token columns [64 * col_half, +64)
     const uint32_t tlane = static_cast<uint32_t>(quarter * 32) << 16;
-    float run[kBT];
+    constexpr int kCols = kBT / 2;
+    float run[kCols];
 #pragma unroll
-    for (int j = 0; j < kBT; ++j) run[j] = 0.0f;
+    for (int j = 0; j < kCols; ++j) run[j] = 0.0f;
     int drained = 0;
-    // add finished chunk c (both halves) to the fp32 registers and hand its
-    // buffer back to the tensor core
+    // add finished chunk c (its hi and lo columns) to the fp32 registers and
+    // hand its buffer back to the tensor core
     auto drain = [&](int c) -> bool {
       const int b = c & 1;
       if (!ptx::mbar_wait_bounded(acc_full(b), (c >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
       ptx::tc_fence_after();
-      const uint32_t base = tmem_base + tlane + b * kAccCols;
+      const uint32_t base = tmem_base + tlane + b * kAccCols + kCols * col_half;
 #pragma unroll
-      for (int cc = 0; cc < 2 * kBT / 32; ++cc) {
-        uint32_t v[32];
-        ptx::tmem_ld_32cols(base + 32u * cc, v);
-        ptx::tmem_wait_ld();
+      for (int part = 0; part < 2; ++part) {         // hi columns, then lo columns
 #pragma unroll
-        for (int j = 0; j < 32; ++j) run[(cc * 32 + j) % kBT] += __uint_as_float(v[j]);
+        for (int cc = 0; cc < kCols / 32; ++cc) {
+          uint32_t v[32];
+          ptx::tmem_ld_32cols(base + part * kBT + 32u * cc, v);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) run[cc * 32 + j] += __uint_as_float(v[j]);
+        }
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(acc_empty(b));
@@ -364,23 +374,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
         ok = false;
         break;
       }
-      const uint8_t* cs = smem + kOffCodes + s * kCodeStageBytes + 32 * t;
-      const uint4 c0 = *reinterpret_cast<const uint4*>(cs);
-      const uint4 c1 = *reinterpret_cast<const uint4*>(cs + 16);
-      const uint32_t sc = *reinterpret_cast<const uint32_t*>(smem + kOffScales + s * kScaleStageBytes + 4 * t);
-      const __half2 s01 = ue4m3x2_to_half2(sc & 0xFFFFu);
-      const __half2 s23 = ue4m3x2_to_half2(sc >> 16);
-      const __half2 sb0 = __low2half2(s01), sb1 = __high2half2(s01);
-      const __half2 sb2 = __low2half2(s23), sb3 = __high2half2(s23);
-      const uint32_t arow = sbase + kOffA + s * kAStageBytes + 128u * t;
-      st_shared_v4(arow + ((0u ^ sw) << 4), expand8(c0.x, sb0));
-      st_shared_v4(arow + ((1u ^ sw) << 4), expand8(c0.y, sb0));
-      st_shared_v4(arow + ((2u ^ sw) << 4), expand8(c0.z, sb1));
-      st_shared_v4(arow + ((3u ^ sw) << 4), expand8(c0.w, sb1));
-      st_shared_v4(arow + ((4u ^ sw) << 4), expand8(c1.x, sb2));
-      st_shared_v4(arow + ((5u ^ sw) << 4), expand8(c1.y, sb2));
-      st_shared_v4(arow + ((6u ^ sw) << 4), expand8(c1.z, sb3));
-      st_shared_v4(arow + ((7u ^ sw) << 4), expand8(c1.w, sb3));
+      const uint4 c = *reinterpret_cast<const uint4*>(smem + kOffCodes + s * kCodeStageBytes +
+                                                      32 * rt + 16 * h);
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(smem + kOffScales +
+                                                             s * kScaleStageBytes + 8 * rt + 4 * h);
+      // this half holds subblocks 2h and 2h + 1 of the slice
+      const __half2 sp = ue4m3x2_to_half2(sc >> (16 * h));
+      const __half2 sa = __low2half2(sp), sb = __high2half2(sp);
+      const uint32_t arow = sbase + kOffA + s * kAStageBytes + 128u * rt;
+      const uint32_t c0 = 4u * h;
+      st_shared_v4(arow + (((c0 + 0u) ^ sw) << 4), expand8(c.x, sa));
+      st_shared_v4(arow + (((c0 + 1u) ^ sw) << 4), expand8(c.y, sa));
+      st_shared_v4(arow + (((c0 + 2u) ^ sw) << 4), expand8(c.z, sb));
+      st_shared_v4(arow + (((c0 + 3u) ^ sw) << 4), expand8(c.w, sb));
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(full_a(s));
       issue(kb + kStages - 1);
@@ -396,8 +402,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       const int nrow = n0 + quarter * 32 + lane;
       if (nrow < N) {
 #pragma unroll
-        for (int j = 0; j < kBT; ++j) {
-          const int m = m0 + j;
+        for (int j = 0; j < kCols; ++j) {
+          const int m = m0 + kCols * col_half + j;
           if (m < M) y[static_cast<size_t>(m) * N + nrow] = run[j] * (g * tok_scale[m]);
         }
       }
