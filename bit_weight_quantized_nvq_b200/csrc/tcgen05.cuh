@@ -47,16 +47,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that suspends the thread until the phase completes or about
+// `hint_ns` pass, so waiting threads neither spin nor issue instructions.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity` of an mbarrier, for at most `limit_ns`.  Returns
 // false on timeout, or early when another thread of the CTA has raised
 // *abort (pass nullptr to wait regardless of aborts).  Every pipeline wait in
-// the library goes through this, so no kernel can spin forever.
+// the library goes through this, so no kernel can spin forever.  The thread
+// sleeps inside try_wait (hint 0.5 ms) and looks at the abort flag and the
+// clock only when a sleep slice ends without the phase completing, so
+// waiting costs no issue slots or shared-memory bandwidth.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
     if (abort != nullptr && *abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
