@@ -29,22 +29,26 @@
 //     caller's workspace, once per call (tokens padded to 128 with zeros).
 //     A token whose largest |d*q| would overflow fp16 (|x| > 65504) is
 //     scaled by 2^-e first and the epilogue multiplies by 2^e.
-//  2. gemm_kernel: one CTA per 128 weight rows x 128 tokens, 10 warps:
-//       warp 0    TMA producer: [hi; lo] activation tiles (2 x 128 rows x 64
-//                 fp16, 128-byte swizzle) into a 4-stage ring;
-//       warp 1    allocates 512 TMEM columns (two 256-column accumulators);
-//                 one thread issues tcgen05.mma (M=128, N=256, K=16) x 4
-//                 per stage, commits each stage back to the producers and
-//                 each finished 8-stage chunk to the draining threads;
-//       warps 2-9 two threads per weight row (two warps per scheduler, so
-//                 each hides the other's latency): cp.async the half row's
-//                 16 code bytes and the row's 4 scale bytes for each stage,
-//                 decode 32 codes to fp16 w' with byte permutes and write them
-//                 in the 128-byte swizzle layout; drain finished chunks
-//                 (tcgen05.ld of half the hi and lo columns into 64 fp32
-//                 registers); the epilogue scales and stores the registers.
-//     Every wait is bounded (4 s); a timeout raises an error flag and the
-//     CTA drains what it issued, frees TMEM and exits.
+//  2. gemm_kernel: CTA pairs (clusters of 2).  Each CTA owns 128 weight
+//     rows; the pair shares a tile of 128 tokens and the even CTA issues
+//     tcgen05.mma.cta_group::2 (M = 256, N = 128, K = 16) for both:
+//       warp 0    TMA: this CTA's hi and lo rows of 64 of the tokens (two
+//                 64 x 64 fp16 boxes, 128-byte swizzle) into an 8-stage ring;
+//       warp 1    allocates the pair's 512 TMEM columns; in the even CTA it
+//                 waits for each stage and issues 8 pair MMAs (hi and lo of
+//                 4 K-steps into the same accumulator), with A read from
+//                 tensor memory and B from both CTAs' shared memory;
+//       warps 2-9 two threads per weight row: cp.async the packed codes and
+//                 scales, decode them to fp16 w' and tcgen05.st them into the
+//                 8-stage A ring in tensor memory (row m in lane m); drain
+//                 finished 512-wide K chunks into fp32 registers; store y;
+//       warp 10   forwards "this CTA's rows of the stage landed" to the even
+//                 CTA's stage barrier.
+//     Every role runs with its whole warp converged on the waits (a wait in
+//     a diverged lane stalls the issuing loop by ~150-200 cycles a stage)
+//     and one lane issuing.  Every wait is bounded (4 s); a timeout raises
+//     an error flag and the CTA drains what it issued, and the pair frees
+//     TMEM together after a cluster barrier.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -60,30 +64,43 @@
 namespace nvq {
 namespace {
 
-constexpr int kBN = 128;            // weight rows per tile = MMA M = TMEM lanes
-constexpr int kBT = 128;            // tokens per tile; MMA N = 2 * kBT ([hi; lo])
+constexpr int kBN = 128;            // weight rows per CTA = TMEM lanes
+constexpr int kBT = 128;            // tokens per tile = pair MMA N (hi and lo issued separately)
+constexpr int kBTc = kBT / 2;       // tokens whose hi and lo rows one CTA of the pair loads
 constexpr int kBK = 64;             // K per stage: one 128-byte fp16 swizzle row
-constexpr int kStages = 4;
-constexpr int kExpThreads = 256;     // weight expansion + epilogue: 2 per row
-constexpr int kThreads = 64 + kExpThreads;
+constexpr int kStages = 8;          // pipeline depth: activation ring (shared memory) and
+                                    // expanded-weight ring (tensor memory) advance together
+constexpr int kCStages = 8;         // packed-weight staging (shared memory)
+constexpr int kTPR = 2;             // expansion threads per weight row
+constexpr int kExpThreads = kTPR * kBN;   // weight expansion + epilogue
+constexpr int kExpWarps = kExpThreads / 32;
+constexpr int kFwdWarp = 2 + kExpWarps;   // forwarder: after the expansion warps
+constexpr int kThreads = 32 * (kFwdWarp + 1);
+constexpr int kEPT = kBK / kTPR;    // K elements one thread expands per stage
+constexpr int kCPT = kEPT / 2;      // their code bytes = TMEM columns
+static_assert(kTPR == 2 || kTPR == 4, "a thread expands one or two 16-element subblocks");
 constexpr int kChunk = 8;           // K stages accumulated per TMEM buffer
-constexpr uint32_t kAccCols = 2 * kBT;        // one [hi | lo] accumulator
-constexpr uint32_t kTmemCols = 2 * kAccCols;  // two accumulators
+constexpr uint32_t kAccCols = kBT;                  // one accumulator: 128 fp32 columns
+constexpr uint32_t kACols = kBK / 2;                // one A stage: 64 fp16 = 32 columns
+constexpr uint32_t kAColBase = 2 * kAccCols;        // A ring after the two accumulators
+constexpr uint32_t kTmemCols = kAColBase + kStages * kACols;   // 512
+static_assert(kTmemCols == 512, "the tile uses all of tensor memory");
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
-constexpr uint32_t kAStageBytes = kBN * kBK * 2;        // 16 KB of w'
-constexpr uint32_t kBStageBytes = 2 * kBT * kBK * 2;    // 32 KB of [hi; lo]
+constexpr uint32_t kBHalfBytes = kBTc * kBK * 2;        // 8 KB: this CTA's hi (or lo) rows
+constexpr uint32_t kBStageBytes = 2 * kBHalfBytes;      // 16 KB of [hi; lo]
 constexpr uint32_t kCodeStageBytes = kBN * kBK / 2;     // 4 KB of codes
-constexpr uint32_t kScaleStageBytes = kBN * 8;         // 4 scale bytes per half row
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kAStageBytes;
+constexpr uint32_t kScaleStageBytes = kExpThreads * 4;  // the row's 4 scale bytes, per thread
+constexpr uint32_t kOffB = 0;
 constexpr uint32_t kOffCodes = kOffB + kStages * kBStageBytes;
-constexpr uint32_t kOffScales = kOffCodes + kStages * kCodeStageBytes;
-constexpr uint32_t kOffBars = kOffScales + kStages * kScaleStageBytes;
-constexpr uint32_t kNumBars = 3 * kStages + 5;   // + acc_full[2], acc_empty[2], mma_done
+constexpr uint32_t kOffScales = kOffCodes + kCStages * kCodeStageBytes;
+constexpr uint32_t kOffBars = kOffScales + kCStages * kScaleStageBytes;
+// full_b, stage_full, stage_empty, acc_full[2], acc_empty[2], mma_done
+constexpr uint32_t kNumBars = 3 * kStages + 5;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + slack to align to 1024
-static_assert(kOffB % 1024 == 0 && kOffCodes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+static_assert(kOffCodes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+static_assert(kSmemBytes <= 232448, "over the opt-in shared memory of one CTA");
 
 // fp16 high bytes of the E2M1 values: 0, .5, 1, 1.5, 2, 3, 4, 6 are 0x0000,
 // 0x3800, 0x3C00, 0x3E00, 0x4000, 0x4200, 0x4400, 0x4600 (low bytes zero);
@@ -120,12 +137,6 @@ __device__ __forceinline__ __half2 ue4m3x2_to_half2(uint32_t two_bytes) {
   const uint16_t in = static_cast<uint16_t>(two_bytes);
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return bits_h2(h2);
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -199,17 +210,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw + pad;
-  auto full_a = [&](int s) { return sbase + kOffBars + 8u * s; };
-  auto full_b = [&](int s) { return sbase + kOffBars + 8u * (kStages + s); };
-  auto empty = [&](int s) { return sbase + kOffBars + 8u * (2 * kStages + s); };
-  auto acc_full = [&](int b) { return sbase + kOffBars + 8u * (3 * kStages + b); };
-  auto acc_empty = [&](int b) { return sbase + kOffBars + 8u * (3 * kStages + 2 + b); };
-  const uint32_t mma_done = sbase + kOffBars + 8u * (3 * kStages + 4);
+  // full_b(s):      this CTA's activation rows of stage s landed (TMA tx)
+  // stage_full(s):  (leader) stage s complete in both CTAs: A written by all
+  //                 expansion warps of the pair, both CTAs' B rows forwarded
+  // stage_empty(s): the pair MMAs of stage s finished (committed to both CTAs)
+  auto full_b = [&](int s) { return sbase + kOffBars + 8u * s; };
+  auto stage_full = [&](int s) { return sbase + kOffBars + 8u * (kStages + s); };
+  auto stage_empty = [&](int s) { return sbase + kOffBars + 8u * (2 * kStages + s); };
+  constexpr uint32_t kOffAcc = 8u * (3 * kStages);
+  auto acc_full = [&](int b) { return sbase + kOffBars + kOffAcc + 8u * b; };
+  auto acc_empty = [&](int b) { return sbase + kOffBars + kOffAcc + 8u * (2 + b); };
+  const uint32_t mma_done = sbase + kOffBars + kOffAcc + 32u;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // The two CTAs of a cluster are a pair: CTA 0 (the leader) issues the
+  // pair MMAs for both.  Each CTA owns 128 weight rows and loads the hi and
+  // lo rows of half of the 128 tokens.
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
   const int n0 = blockIdx.x * kBN;
   const int m0 = blockIdx.y * kBT;
   const int num_kb = K / kBK;
@@ -217,13 +238,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(full_a(s), kExpThreads);
       ptx::mbar_init(full_b(s), 1);
-      ptx::mbar_init(empty(s), 1);
+      ptx::mbar_init(stage_full(s), 2 * kExpWarps + 2);
+      ptx::mbar_init(stage_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(acc_full(b), 1);
-      ptx::mbar_init(acc_empty(b), kExpThreads);
+      ptx::mbar_init(acc_empty(b), 2 * kExpWarps);
     }
     ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -231,11 +252,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     ptx::prefetch_tensormap(&act_map);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), kTmemCols);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(ptx::smem_addr(tmem_holder), kTmemCols);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();   // both CTAs' barriers exist before any remote arrival
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -243,119 +264,158 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     *abort_flag = 1;
     atomicOr(&g_gemm_error_flags, 1u);
   };
+  // Every role runs its loop with the whole warp converged: all lanes wait
+  // (a wait in a diverged lane costs the tensor pipe ~150-200 cycles per
+  // stage), one lane issues, and the outcome is made warp-uniform.
+  auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    const bool got = ptx::mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
+    return __all_sync(0xffffffffu, got);
+  };
 
   if (warp == 0) {
-    // ------------------------------ TMA producer ------------------------------
-    if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1;
-        if (!ptx::mbar_wait_bounded(empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) {
-          fail();
-          break;
-        }
+    // ------------------------------- TMA producer ------------------------------
+    int issued = 0;
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (kb / kStages) & 1;
+      if (!warp_wait(stage_empty(s), ph ^ 1)) {
+        fail();
+        break;
+      }
+      if (lane == 0) {
         const uint32_t dst = sbase + kOffB + s * kBStageBytes;
         ptx::mbar_arrive_expect_tx(full_b(s), kBStageBytes);
-        ptx::tma_load_2d(dst, &act_map, kb * kBK, m0, full_b(s));
-        ptx::tma_load_2d(dst + kBStageBytes / 2, &act_map, kb * kBK, M_pad + m0, full_b(s));
-        ++issued;
+        ptx::tma_load_2d(dst, &act_map, kb * kBK, m0 + kBTc * rank, full_b(s));
+        ptx::tma_load_2d(dst + kBHalfBytes, &act_map, kb * kBK, M_pad + m0 + kBTc * rank,
+                         full_b(s));
       }
-      if (*abort_flag) {
-        for (int kb = std::max(0, issued - kStages); kb < issued; ++kb)
-          ptx::mbar_wait_bounded(full_b(kb % kStages), (kb / kStages) & 1, nullptr, kWaitLimitNs);
+      __syncwarp();
+      ++issued;
+    }
+    if (*abort_flag) {
+      // the MMAs may have stopped: wait for this CTA's copies in flight
+      // before the CTA can leave
+      for (int kb = std::max(0, issued - kStages); kb < issued; ++kb)
+        ptx::mbar_wait_bounded(full_b(kb % kStages), (kb / kStages) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == kFwdWarp) {
+    // ------------ forwarder: this CTA's activation rows have landed ---------
+    const uint32_t leader_stage_full0 = ptx::mapa_shared(stage_full(0), 0);
+    for (int kb = 0; kb < num_kb; ++kb) {
+      const int s = kb % kStages;
+      if (!warp_wait(full_b(s), (kb / kStages) & 1)) {
+        fail();
+        break;
       }
+      if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * s);
+      __syncwarp();
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer --------------------------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_f16_f32(kBN, 2 * kBT);
+    // -------------------------- pair MMA issuer (leader) ------------------------
+    if (leader) {
+      constexpr uint32_t idesc = ptx::idesc_f16_f32(2 * kBN, kBT);
+      // completion of the pair MMAs is signalled to the same barrier in both CTAs
+      auto commit_both = [&](uint32_t bar) {
+        ptx::mma_commit_pair(ptx::mapa_shared(bar, 0));
+        ptx::mma_commit_pair(ptx::mapa_shared(bar, 1));
+      };
       for (int kb = 0; kb < num_kb; ++kb) {
         const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1;
         const int c = kb / kChunk;
         const int b = c & 1;
         const bool first = (kb % kChunk) == 0;
-        // a buffer is reused two chunks later, once the epilogue drained it
-        if (first && c >= 2 &&
-            !ptx::mbar_wait_bounded(acc_empty(b), ((c >> 1) - 1) & 1, abort_flag, kWaitLimitNs)) {
+        // a buffer is reused two chunks later, once both epilogues drained it
+        if (first && c >= 2 && !warp_wait(acc_empty(b), ((c >> 1) - 1) & 1)) {
           fail();
           break;
         }
-        if (!ptx::mbar_wait_bounded(full_a(s), ph, abort_flag, kWaitLimitNs) ||
-            !ptx::mbar_wait_bounded(full_b(s), ph, abort_flag, kWaitLimitNs)) {
+        if (!warp_wait(stage_full(s), (kb / kStages) & 1)) {
           fail();
           break;
         }
-        ptx::tc_fence_after();
-        const uint32_t a0 = sbase + kOffA + s * kAStageBytes;
-        const uint32_t b0 = sbase + kOffB + s * kBStageBytes;
-        const uint32_t d_tmem = tmem_base + b * kAccCols;
+        if (lane == 0) {
+          ptx::tc_fence_after();
+          const uint32_t a_cols = tmem_base + kAColBase + s * kACols;
+          const uint64_t bdesc = ptx::sw128_kmajor_desc(sbase + kOffB + s * kBStageBytes);
+          const uint32_t d_tmem = tmem_base + b * kAccCols;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          ptx::mma_f16(d_tmem, ptx::sw128_kmajor_desc(a0 + 32u * k),
-                       ptx::sw128_kmajor_desc(b0 + 32u * k), idesc, !(first && k == 0));
+          for (int k = 0; k < kBK / 16; ++k) {
+            // hi and lo products go to the same accumulator; descriptor start
+            // addresses are in 16-byte units (32 bytes = the next 16 K)
+            ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + 2u * k, idesc,
+                                 !(first && k == 0));
+            ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + (kBHalfBytes >> 4) + 2u * k,
+                                 idesc, 1u);
+          }
+          commit_both(stage_empty(s));
+          if ((kb % kChunk) == kChunk - 1 || kb == num_kb - 1) commit_both(acc_full(b));
         }
-        ptx::mma_commit(empty(s));
-        if ((kb % kChunk) == kChunk - 1 || kb == num_kb - 1) ptx::mma_commit(acc_full(b));
+        __syncwarp();
       }
-      // no MMA may still be writing TMEM when it is released
-      ptx::mma_commit(mma_done);
+      // no MMA may still be reading or writing tensor memory when it is released
+      if (lane == 0) commit_both(mma_done);
+      __syncwarp();
       ptx::mbar_wait_bounded(mma_done, 0, nullptr, kWaitLimitNs);
     }
   } else {
     // ------------------- weight expansion, then the epilogue ------------------
-    // Two threads per weight row (warps 2-5: first half of the 64-wide K
-    // slice, warps 6-9: second half).  In the epilogue the warp pair that
-    // shares a TMEM lane quarter splits the 128 token columns.
-    const int t = threadIdx.x - 64;         // 0..255
-    const int rt = t & (kBN - 1);           // row of the tile
-    const int h = t >> 7;                   // half of the K slice
+    // A warp may only touch the TMEM lanes of its quarter (warp % 4), so the
+    // threads of TMEM lane rt = 32 * (warp % 4) + lane expand weight row
+    // n0 + rt: warp group p = (warp - 2) / 4 takes part p of each 64-wide K
+    // slice (kEPT elements, TMEM columns kCPT * p ..).  In the epilogue the
+    // same threads split the 128 token columns.
+    const int quarter = warp & 3;
+    const int p = (warp - 2) >> 2;
+    const int rt = quarter * 32 + lane;
     const int row = n0 + rt;
     const bool valid = row < N;
-    const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2) + 16 * h;
+    const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2) + kCPT * p;
     const uint8_t* srow = scales + static_cast<size_t>(valid ? row : 0) * (K / 16);
-    const uint32_t stg_c = sbase + kOffCodes + 32u * rt + 16u * h;
-    const uint32_t stg_s = sbase + kOffScales + 8u * rt + 4u * h;
+    const uint32_t stg_c = sbase + kOffCodes + 32u * rt + kCPT * p;
+    const int t = threadIdx.x - 64;    // 0 .. kExpThreads - 1
+    const uint32_t stg_s = sbase + kOffScales + 4u * t;
     auto issue = [&](int kb) {
       if (kb < num_kb) {
-        const uint32_t slot = kb % kStages;
-        ptx::cp_async_16(stg_c + slot * kCodeStageBytes, crow + 32 * kb, valid ? 16u : 0u);
+        const uint32_t slot = kb % kCStages;
+        if constexpr (kCPT == 16)
+          ptx::cp_async_16(stg_c + slot * kCodeStageBytes, crow + 32 * kb, valid ? 16u : 0u);
+        else
+          ptx::cp_async_8(stg_c + slot * kCodeStageBytes, crow + 32 * kb, valid ? 8u : 0u);
         ptx::cp_async_4(stg_s + slot * kScaleStageBytes, srow + 4 * kb, valid ? 4u : 0u);
       }
       ptx::cp_async_commit();
     };
-    for (int i = 0; i < kStages - 1; ++i) issue(i);
+    for (int i = 0; i < kCStages - 1; ++i) issue(i);
+    // One arrival per warp (lane 0, after __syncwarp); arrivals go to the
+    // leader's barriers.
+    const uint32_t leader_stage_full0 = ptx::mapa_shared(stage_full(0), 0);
+    const uint32_t leader_acc_empty0 = ptx::mapa_shared(acc_empty(0), 0);
     bool ok = true;
-    const uint32_t sw = rt & 7;
-    const int quarter = warp & 3;            // TMEM lanes this warp may read
-    const int col_half = (warp - 2) >> 2;    // token columns [64 * col_half, +64)
     const uint32_t tlane = static_cast<uint32_t>(quarter * 32) << 16;
-    constexpr int kCols = kBT / 2;
+    const uint32_t a_dst = tmem_base + tlane + kAColBase + kCPT * p;
+    constexpr int kCols = kBT / kTPR;
     float run[kCols];
 #pragma unroll
     for (int j = 0; j < kCols; ++j) run[j] = 0.0f;
     int drained = 0;
-    // add finished chunk c (its hi and lo columns) to the fp32 registers and
-    // hand its buffer back to the tensor core
+    int stored = 0;   // stages whose A tile this warp stored
+    // add finished chunk c to the fp32 registers and hand its buffer back
     auto drain = [&](int c) -> bool {
       const int b = c & 1;
-      if (!ptx::mbar_wait_bounded(acc_full(b), (c >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
+      if (!warp_wait(acc_full(b), (c >> 1) & 1)) return false;
       ptx::tc_fence_after();
-      const uint32_t base = tmem_base + tlane + b * kAccCols + kCols * col_half;
+      const uint32_t base = tmem_base + tlane + b * kAccCols + kCols * p;
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {         // hi columns, then lo columns
+      for (int cc = 0; cc < kCols / 32; ++cc) {
+        uint32_t v[32];
+        ptx::tmem_ld_32cols(base + 32u * cc, v);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < kCols / 32; ++cc) {
-          uint32_t v[32];
-          ptx::tmem_ld_32cols(base + part * kBT + 32u * cc, v);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) run[cc * 32 + j] += __uint_as_float(v[j]);
-        }
+        for (int j = 0; j < 32; ++j) run[cc * 32 + j] += __uint_as_float(v[j]);
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(acc_empty(b));
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(leader_acc_empty0 + 8u * b);
       return true;
     };
     for (int kb = 0; kb < num_kb; ++kb) {
@@ -366,30 +426,58 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
           break;
         }
       }
-      ptx::cp_async_wait<kStages - 2>();
+      ptx::cp_async_wait<kCStages - 2>();
       const int s = kb % kStages;
-      const uint32_t ph = (kb / kStages) & 1;
-      if (!ptx::mbar_wait_bounded(empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+      if (!warp_wait(stage_empty(s), ((kb / kStages) & 1) ^ 1)) {
         fail();
         ok = false;
         break;
       }
-      const uint4 c = *reinterpret_cast<const uint4*>(smem + kOffCodes + s * kCodeStageBytes +
-                                                      32 * rt + 16 * h);
-      const uint32_t sc = *reinterpret_cast<const uint32_t*>(smem + kOffScales +
-                                                             s * kScaleStageBytes + 8 * rt + 4 * h);
-      // this half holds subblocks 2h and 2h + 1 of the slice
-      const __half2 sp = ue4m3x2_to_half2(sc >> (16 * h));
-      const __half2 sa = __low2half2(sp), sb = __high2half2(sp);
-      const uint32_t arow = sbase + kOffA + s * kAStageBytes + 128u * rt;
-      const uint32_t c0 = 4u * h;
-      st_shared_v4(arow + (((c0 + 0u) ^ sw) << 4), expand8(c.x, sa));
-      st_shared_v4(arow + (((c0 + 1u) ^ sw) << 4), expand8(c.y, sa));
-      st_shared_v4(arow + (((c0 + 2u) ^ sw) << 4), expand8(c.z, sb));
-      st_shared_v4(arow + (((c0 + 3u) ^ sw) << 4), expand8(c.w, sb));
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(full_a(s));
-      issue(kb + kStages - 1);
+      ptx::tc_fence_after();
+      const int cs = kb % kCStages;
+      const uint8_t* stg = smem + kOffCodes + cs * kCodeStageBytes + 32 * rt + kCPT * p;
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(
+          smem + kOffScales + cs * kScaleStageBytes + 4 * t);
+      // The previous stage's tensor-memory store is waited for (and the
+      // stage announced) only after this stage's decode, so the store's
+      // latency overlaps the decode instead of stalling the warp.
+      auto announce_prev = [&]() {
+        if (kb > 0) {
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * ((kb - 1) % kStages));
+        }
+      };
+      if constexpr (kCPT == 16) {
+        // subblocks 2p and 2p + 1 of the slice
+        const uint4 c = *reinterpret_cast<const uint4*>(stg);
+        const __half2 sp = ue4m3x2_to_half2(sc >> (16 * p));
+        const __half2 s_lo = __low2half2(sp), s_hi = __high2half2(sp);
+        const uint4 e0 = expand8(c.x, s_lo), e1 = expand8(c.y, s_lo);
+        const uint4 e2 = expand8(c.z, s_hi), e3 = expand8(c.w, s_hi);
+        const uint32_t v[16] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w,
+                                e2.x, e2.y, e2.z, e2.w, e3.x, e3.y, e3.z, e3.w};
+        announce_prev();
+        ptx::tmem_st_16cols(a_dst + s * kACols, v);
+      } else {
+        // subblock p of the slice
+        const uint2 c = *reinterpret_cast<const uint2*>(stg);
+        const __half2 s2 = __low2half2(ue4m3x2_to_half2((sc >> (8 * p)) & 0xFFu));
+        const uint4 e0 = expand8(c.x, s2), e1 = expand8(c.y, s2);
+        const uint32_t v[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+        announce_prev();
+        ptx::tmem_st_8cols(a_dst + s * kACols, v);
+      }
+      issue(kb + kCStages - 1);
+      ++stored;
+    }
+    if (stored > 0) {
+      // announce the last stage this warp stored
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * ((stored - 1) % kStages));
     }
     ptx::cp_async_wait<0>();
     while (ok && drained < num_chunks) {
@@ -399,22 +487,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       }
     }
     if (ok) {
-      const int nrow = n0 + quarter * 32 + lane;
+      const int nrow = n0 + rt;
       if (nrow < N) {
 #pragma unroll
         for (int j = 0; j < kCols; ++j) {
-          const int m = m0 + kCols * col_half + j;
+          const int m = m0 + kCols * p + j;
           if (m < M) y[static_cast<size_t>(m) * N + nrow] = run[j] * (g * tok_scale[m]);
         }
       }
     }
   }
 
+  // Neither CTA leaves (or frees tensor memory) while the pair's MMAs or the
+  // peer's remote arrivals may still touch it.
+  __syncwarp();
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, kTmemCols);
+    ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -510,7 +601,7 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(2 * M_pad)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBT)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBTc)};
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act, dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -527,10 +618,26 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN), static_cast<unsigned>(M_pad / kBT));
-  gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, codes, scales, static_cast<int>(N),
-                                                      static_cast<int>(K), static_cast<int>(M),
-                                                      static_cast<int>(M_pad), g, tok_scale, y);
+  // pairs of CTAs along N: an even number of 128-row tiles (an odd last
+  // tile gets an all-padding partner)
+  const int64_t tiles_n = (N + kBN - 1) / kBN;
+  const dim3 grid(static_cast<unsigned>((tiles_n + 1) / 2 * 2), static_cast<unsigned>(M_pad / kBT));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, map, codes, scales, static_cast<int>(N),
+                                     static_cast<int>(K), static_cast<int>(M),
+                                     static_cast<int>(M_pad), g, tok_scale, y);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -163,10 +163,12 @@ size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *
  * The activations are expanded once into `workspace` as fp16 pairs
  * hi = fp16(d*q), lo = fp16(d*q - hi), exact (hi + lo == d*q).  Weight tiles
- * are expanded in shared memory to fp16 w' = E2M1*s_w (exact) and every
- * 64-wide K slice is multiplied by tcgen05.mma (kind::f16) against
- * [hi; lo], accumulating in fp32 in tensor memory; y = g * (acc_hi + acc_lo).
- * Every product is exact; only the fp32 accumulation rounds.
+ * are expanded in tensor memory to fp16 w' = E2M1*s_w (exact) and every
+ * 64-wide K slice is multiplied by tcgen05.mma (kind::f16, CTA pairs)
+ * against hi and against lo, both accumulating in fp32 into one tensor-
+ * memory accumulator per 512-wide K chunk whose partial sums are added in
+ * fp32 registers; y = g * sum.  Every product is exact; only the fp32
+ * accumulation rounds.
  * workspace: device, caller-owned, >= nvq_gemm_workspace_size(M, N, K)
  * bytes, 16-byte aligned; its contents are scratch.
  * Errors: as nvq_gemv (M >= 1), plus NVQ_ERR_WORKSPACE.
