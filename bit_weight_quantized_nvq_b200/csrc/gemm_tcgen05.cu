@@ -268,6 +268,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   // (a wait in a diverged lane costs the tensor pipe ~150-200 cycles per
   // stage), one lane issues, and the outcome is made warp-uniform.
   auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
     const bool got = ptx::mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
     return __all_sync(0xffffffffu, got);
   };
@@ -319,38 +320,50 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 0));
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 1));
       };
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % kStages;
-        const int c = kb / kChunk;
+      // The warp shares its scheduler with two decoding warps, so every
+      // instruction between MMA bursts is a bubble: a chunk is one pass over
+      // the 8 ring stages, unrolled, so stage indices, first-of-chunk and
+      // end-of-chunk are constants and the descriptors are plain adds.
+      static_assert(kChunk == kStages, "one chunk = one pass over the ring");
+      const uint32_t a_cols0 = tmem_base + kAColBase;
+      const uint64_t bdesc0 = ptx::sw128_kmajor_desc(sbase + kOffB);
+      bool ok_mma = true;
+      for (int c = 0; c < num_chunks && ok_mma; ++c) {
         const int b = c & 1;
-        const bool first = (kb % kChunk) == 0;
+        const uint32_t parity = c & 1;
+        const uint32_t d_tmem = tmem_base + b * kAccCols;
         // a buffer is reused two chunks later, once both epilogues drained it
-        if (first && c >= 2 && !warp_wait(acc_empty(b), ((c >> 1) - 1) & 1)) {
+        if (c >= 2 && !warp_wait(acc_empty(b), ((c >> 1) - 1) & 1)) {
           fail();
           break;
         }
-        if (!warp_wait(stage_full(s), (kb / kStages) & 1)) {
-          fail();
-          break;
-        }
-        if (lane == 0) {
-          ptx::tc_fence_after();
-          const uint32_t a_cols = tmem_base + kAColBase + s * kACols;
-          const uint64_t bdesc = ptx::sw128_kmajor_desc(sbase + kOffB + s * kBStageBytes);
-          const uint32_t d_tmem = tmem_base + b * kAccCols;
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            // hi and lo products go to the same accumulator; descriptor start
-            // addresses are in 16-byte units (32 bytes = the next 16 K)
-            ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + 2u * k, idesc,
-                                 !(first && k == 0));
-            ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + (kBHalfBytes >> 4) + 2u * k,
-                                 idesc, 1u);
+        for (int j = 0; j < kStages; ++j) {
+          const int kb = c * kChunk + j;
+          if (kb >= num_kb) break;
+          if (!warp_wait(stage_full(j), parity)) {
+            fail();
+            ok_mma = false;
+            break;
           }
-          commit_both(stage_empty(s));
-          if ((kb % kChunk) == kChunk - 1 || kb == num_kb - 1) commit_both(acc_full(b));
+          if (lane == 0) {
+            ptx::tc_fence_after();
+            const uint32_t a_cols = a_cols0 + j * kACols;
+            const uint64_t bdesc = bdesc0 + ((j * kBStageBytes) >> 4);
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              // hi and lo products go to the same accumulator; descriptor
+              // start addresses are in 16-byte units (32 bytes = next 16 K)
+              ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + 2u * k, idesc,
+                                   (j == 0 && k == 0) ? 0u : 1u);
+              ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + (kBHalfBytes >> 4) + 2u * k,
+                                   idesc, 1u);
+            }
+            commit_both(stage_empty(j));
+            if (j == kStages - 1 || kb == num_kb - 1) commit_both(acc_full(b));
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       // no MMA may still be reading or writing tensor memory when it is released
       if (lane == 0) commit_both(mma_done);
