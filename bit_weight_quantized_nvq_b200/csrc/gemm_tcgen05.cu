@@ -32,16 +32,18 @@
 //  2. gemm_kernel: CTA pairs (clusters of 2).  Each CTA owns 128 weight
 //     rows; the pair shares a tile of 128 tokens and the even CTA issues
 //     tcgen05.mma.cta_group::2 (M = 256, N = 128, K = 16) for both:
-//       warp 0    TMA: this CTA's hi and lo rows of 64 of the tokens (two
-//                 64 x 64 fp16 boxes, 128-byte swizzle) into an 8-stage ring;
+//       warp 0    TMA: this CTA's hi and lo rows of 64 of the tokens, for
+//                 the two 64-wide K sub-tiles of a 128-wide stage (four
+//                 64 x 64 fp16 boxes, 128-byte swizzle), into a 4-stage ring;
 //       warp 1    allocates the pair's 512 TMEM columns; in the even CTA it
-//                 waits for each stage and issues 8 pair MMAs (hi and lo of
-//                 4 K-steps into the same accumulator), with A read from
+//                 waits for each stage and issues 16 pair MMAs (hi and lo of
+//                 8 K-steps into the same accumulator), with A read from
 //                 tensor memory and B from both CTAs' shared memory;
-//       warps 2-9 two threads per weight row: cp.async the packed codes and
-//                 scales, decode them to fp16 w' and tcgen05.st them into the
-//                 8-stage A ring in tensor memory (row m in lane m); drain
-//                 finished 512-wide K chunks into fp32 registers; store y;
+//       warps 2-9 two threads per weight row, one per sub-tile: cp.async the
+//                 packed codes and scales, decode them to fp16 w' and
+//                 tcgen05.st them into the 4-stage A ring in tensor memory
+//                 (row m in lane m); drain finished 512-wide K chunks into
+//                 fp32 registers; store y;
 //       warp 10   forwards "this CTA's rows of the stage landed" to the even
 //                 CTA's stage barrier.
 //     Every role runs with its whole warp converged on the waits (a wait in
@@ -67,30 +69,32 @@ namespace {
 constexpr int kBN = 128;            // weight rows per CTA = TMEM lanes
 constexpr int kBT = 128;            // tokens per tile = pair MMA N (hi and lo issued separately)
 constexpr int kBTc = kBT / 2;       // tokens whose hi and lo rows one CTA of the pair loads
-constexpr int kBK = 64;             // K per stage: one 128-byte fp16 swizzle row
-constexpr int kStages = 8;          // pipeline depth: activation ring (shared memory) and
+constexpr int kBK = 128;            // K per stage: two 64-wide sub-tiles
+constexpr int kSubK = 64;           // K per 128-byte fp16 swizzle row (TMA box, MMA tile)
+constexpr int kSubs = kBK / kSubK;
+constexpr int kStages = 4;          // pipeline depth: activation ring (shared memory) and
                                     // expanded-weight ring (tensor memory) advance together
-constexpr int kCStages = 8;         // packed-weight staging (shared memory)
-constexpr int kTPR = 2;             // expansion threads per weight row
+constexpr int kCStages = 6;         // packed-weight staging (shared memory)
+constexpr int kTPR = 2;             // expansion threads per weight row: one per sub-tile
 constexpr int kExpThreads = kTPR * kBN;   // weight expansion + epilogue
 constexpr int kExpWarps = kExpThreads / 32;
 constexpr int kFwdWarp = 2 + kExpWarps;   // forwarder: after the expansion warps
 constexpr int kThreads = 32 * (kFwdWarp + 1);
-constexpr int kEPT = kBK / kTPR;    // K elements one thread expands per stage
-constexpr int kCPT = kEPT / 2;      // their code bytes = TMEM columns
-static_assert(kTPR == 2 || kTPR == 4, "a thread expands one or two 16-element subblocks");
-constexpr int kChunk = 8;           // K stages accumulated per TMEM buffer
+constexpr int kEPT = kBK / kTPR;    // K elements one thread expands per stage (64)
+constexpr int kCPT = kEPT / 2;      // their code bytes = TMEM columns (32)
+static_assert(kTPR == kSubs && kEPT == kSubK, "thread part p expands sub-tile p");
+constexpr int kChunk = 4;           // K stages accumulated per TMEM buffer (512 K)
 constexpr uint32_t kAccCols = kBT;                  // one accumulator: 128 fp32 columns
-constexpr uint32_t kACols = kBK / 2;                // one A stage: 64 fp16 = 32 columns
+constexpr uint32_t kACols = kBK / 2;                // one A stage: 128 fp16 = 64 columns
 constexpr uint32_t kAColBase = 2 * kAccCols;        // A ring after the two accumulators
 constexpr uint32_t kTmemCols = kAColBase + kStages * kACols;   // 512
 static_assert(kTmemCols == 512, "the tile uses all of tensor memory");
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
-constexpr uint32_t kBHalfBytes = kBTc * kBK * 2;        // 8 KB: this CTA's hi (or lo) rows
-constexpr uint32_t kBStageBytes = 2 * kBHalfBytes;      // 16 KB of [hi; lo]
-constexpr uint32_t kCodeStageBytes = kBN * kBK / 2;     // 4 KB of codes
-constexpr uint32_t kScaleStageBytes = kExpThreads * 4;  // the row's 4 scale bytes, per thread
+constexpr uint32_t kBSubBytes = kBTc * kSubK * 2;       // 8 KB: this CTA's hi (or lo) rows of a sub-tile
+constexpr uint32_t kBStageBytes = kSubs * 2 * kBSubBytes;   // 32 KB: [sub0 hi | sub0 lo | sub1 hi | sub1 lo]
+constexpr uint32_t kCodeStageBytes = kBN * kBK / 2;     // 8 KB of codes
+constexpr uint32_t kScaleStageBytes = kExpThreads * 4;  // 4 scale bytes per thread
 constexpr uint32_t kOffB = 0;
 constexpr uint32_t kOffCodes = kOffB + kStages * kBStageBytes;
 constexpr uint32_t kOffScales = kOffCodes + kCStages * kCodeStageBytes;
@@ -233,7 +237,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   const bool leader = rank == 0;
   const int n0 = blockIdx.x * kBN;
   const int m0 = blockIdx.y * kBT;
-  const int num_kb = K / kBK;
+  const int num_kb = (K + kBK - 1) / kBK;   // the last stage may hold one sub-tile
   const int num_chunks = (num_kb + kChunk - 1) / kChunk;
 
   if (threadIdx.x == 0) {
@@ -285,10 +289,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       }
       if (lane == 0) {
         const uint32_t dst = sbase + kOffB + s * kBStageBytes;
-        ptx::mbar_arrive_expect_tx(full_b(s), kBStageBytes);
-        ptx::tma_load_2d(dst, &act_map, kb * kBK, m0 + kBTc * rank, full_b(s));
-        ptx::tma_load_2d(dst + kBHalfBytes, &act_map, kb * kBK, M_pad + m0 + kBTc * rank,
-                         full_b(s));
+        const int nsub = min(kSubs, (K - kb * kBK) / kSubK);
+        ptx::mbar_arrive_expect_tx(full_b(s), nsub * 2 * kBSubBytes);
+        for (int sub = 0; sub < nsub; ++sub) {
+          const uint32_t d0 = dst + sub * 2 * kBSubBytes;
+          const int kx = kb * kBK + sub * kSubK;
+          ptx::tma_load_2d(d0, &act_map, kx, m0 + kBTc * rank, full_b(s));
+          ptx::tma_load_2d(d0 + kBSubBytes, &act_map, kx, M_pad + m0 + kBTc * rank, full_b(s));
+        }
       }
       __syncwarp();
       ++issued;
@@ -320,10 +328,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 0));
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 1));
       };
-      // The warp shares its scheduler with two decoding warps, so every
-      // instruction between MMA bursts is a bubble: a chunk is one pass over
-      // the 8 ring stages, unrolled, so stage indices, first-of-chunk and
-      // end-of-chunk are constants and the descriptors are plain adds.
+      // The issuing thread is paced by the tensor core, so every instruction
+      // between MMA bursts is a bubble (more so as the warp shares its
+      // scheduler with two decoding warps): a chunk is one pass over the
+      // ring, unrolled, so stage indices and flags are constants and the
+      // descriptors are plain adds, and a stage holds 16 MMAs per wait.
+      // (Issuing through a predicate from the converged warp, instead of the
+      // lane-0 branch, measured slower.)
       static_assert(kChunk == kStages, "one chunk = one pass over the ring");
       const uint32_t a_cols0 = tmem_base + kAColBase;
       const uint64_t bdesc0 = ptx::sw128_kmajor_desc(sbase + kOffB);
@@ -350,14 +361,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
             ptx::tc_fence_after();
             const uint32_t a_cols = a_cols0 + j * kACols;
             const uint64_t bdesc = bdesc0 + ((j * kBStageBytes) >> 4);
+            const bool two = kb * kBK + kSubK < K;   // the last stage may hold one sub-tile
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              // hi and lo products go to the same accumulator; descriptor
-              // start addresses are in 16-byte units (32 bytes = next 16 K)
-              ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + 2u * k, idesc,
-                                   (j == 0 && k == 0) ? 0u : 1u);
-              ptx::mma_f16_ts_pair(d_tmem, a_cols + 8u * k, bdesc + (kBHalfBytes >> 4) + 2u * k,
-                                   idesc, 1u);
+            for (int sub = 0; sub < kSubs; ++sub) {
+              if (sub == 1 && !two) break;
+#pragma unroll
+              for (int k = 0; k < kSubK / 16; ++k) {
+                // hi and lo products go to the same accumulator; descriptor
+                // start addresses are in 16-byte units (32 bytes = next 16 K)
+                const uint32_t a = a_cols + sub * (kSubK / 2) + 8u * k;
+                const uint64_t bhi = bdesc + ((sub * 2 * kBSubBytes) >> 4) + 2u * k;
+                ptx::mma_f16_ts_pair(d_tmem, a, bhi, idesc, (j == 0 && sub == 0 && k == 0) ? 0u : 1u);
+                ptx::mma_f16_ts_pair(d_tmem, a, bhi + (kBSubBytes >> 4), idesc, 1u);
+              }
             }
             commit_both(stage_empty(j));
             if (j == kStages - 1 || kb == num_kb - 1) commit_both(acc_full(b));
@@ -374,27 +390,30 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     // ------------------- weight expansion, then the epilogue ------------------
     // A warp may only touch the TMEM lanes of its quarter (warp % 4), so the
     // threads of TMEM lane rt = 32 * (warp % 4) + lane expand weight row
-    // n0 + rt: warp group p = (warp - 2) / 4 takes part p of each 64-wide K
-    // slice (kEPT elements, TMEM columns kCPT * p ..).  In the epilogue the
-    // same threads split the 128 token columns.
+    // n0 + rt: warp group p = (warp - 2) / 4 takes sub-tile p of each
+    // 128-wide K stage (kEPT = 64 elements, TMEM columns kCPT * p ..).  In the
+    // epilogue the same threads split the 128 token columns.
     const int quarter = warp & 3;
     const int p = (warp - 2) >> 2;
     const int rt = quarter * 32 + lane;
     const int row = n0 + rt;
     const bool valid = row < N;
     const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2) + kCPT * p;
-    const uint8_t* srow = scales + static_cast<size_t>(valid ? row : 0) * (K / 16);
-    const uint32_t stg_c = sbase + kOffCodes + 32u * rt + kCPT * p;
+    const uint8_t* srow = scales + static_cast<size_t>(valid ? row : 0) * (K / 16) + 4 * p;
+    const uint32_t stg_c = sbase + kOffCodes + 64u * rt + kCPT * p;
     const int t = threadIdx.x - 64;    // 0 .. kExpThreads - 1
     const uint32_t stg_s = sbase + kOffScales + 4u * t;
     auto issue = [&](int kb) {
       if (kb < num_kb) {
         const uint32_t slot = kb % kCStages;
-        if constexpr (kCPT == 16)
-          ptx::cp_async_16(stg_c + slot * kCodeStageBytes, crow + 32 * kb, valid ? 16u : 0u);
-        else
-          ptx::cp_async_8(stg_c + slot * kCodeStageBytes, crow + 32 * kb, valid ? 8u : 0u);
-        ptx::cp_async_4(stg_s + slot * kScaleStageBytes, srow + 4 * kb, valid ? 4u : 0u);
+        // this thread's sub-tile exists (K is a multiple of 64): else zero fill
+        // from an in-bounds address
+        const bool in = valid && kb * kBK + p * kSubK < K;
+        const uint8_t* c_src = in ? crow + (kBK / 2) * kb : crow;
+        const uint8_t* s_src = in ? srow + (kBK / 16) * kb : srow;
+        ptx::cp_async_16(stg_c + slot * kCodeStageBytes, c_src, in ? 16u : 0u);
+        ptx::cp_async_16(stg_c + slot * kCodeStageBytes + 16, c_src + (in ? 16 : 0), in ? 16u : 0u);
+        ptx::cp_async_4(stg_s + slot * kScaleStageBytes, s_src, in ? 4u : 0u);
       }
       ptx::cp_async_commit();
     };
@@ -448,7 +467,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       }
       ptx::tc_fence_after();
       const int cs = kb % kCStages;
-      const uint8_t* stg = smem + kOffCodes + cs * kCodeStageBytes + 32 * rt + kCPT * p;
+      const uint8_t* stg = smem + kOffCodes + cs * kCodeStageBytes + 64 * rt + kCPT * p;
       const uint32_t sc = *reinterpret_cast<const uint32_t*>(
           smem + kOffScales + cs * kScaleStageBytes + 4 * t);
       // The previous stage's tensor-memory store is waited for (and the
@@ -462,25 +481,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
           if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * ((kb - 1) % kStages));
         }
       };
-      if constexpr (kCPT == 16) {
-        // subblocks 2p and 2p + 1 of the slice
-        const uint4 c = *reinterpret_cast<const uint4*>(stg);
-        const __half2 sp = ue4m3x2_to_half2(sc >> (16 * p));
-        const __half2 s_lo = __low2half2(sp), s_hi = __high2half2(sp);
-        const uint4 e0 = expand8(c.x, s_lo), e1 = expand8(c.y, s_lo);
-        const uint4 e2 = expand8(c.z, s_hi), e3 = expand8(c.w, s_hi);
-        const uint32_t v[16] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w,
-                                e2.x, e2.y, e2.z, e2.w, e3.x, e3.y, e3.z, e3.w};
+      {
+        // sub-tile p: subblocks 0..3 of it, 8 codes per 32-bit word
+        const uint4 c0 = *reinterpret_cast<const uint4*>(stg);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(stg + 16);
+        const __half2 sp01 = ue4m3x2_to_half2(sc & 0xFFFFu);
+        const __half2 sp23 = ue4m3x2_to_half2(sc >> 16);
+        const __half2 s0 = __low2half2(sp01), s1 = __high2half2(sp01);
+        const __half2 s2 = __low2half2(sp23), s3 = __high2half2(sp23);
+        const uint4 e0 = expand8(c0.x, s0), e1 = expand8(c0.y, s0);
+        const uint4 e2 = expand8(c0.z, s1), e3 = expand8(c0.w, s1);
+        const uint4 e4 = expand8(c1.x, s2), e5 = expand8(c1.y, s2);
+        const uint4 e6 = expand8(c1.z, s3), e7 = expand8(c1.w, s3);
+        const uint32_t v[32] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w,
+                                e2.x, e2.y, e2.z, e2.w, e3.x, e3.y, e3.z, e3.w,
+                                e4.x, e4.y, e4.z, e4.w, e5.x, e5.y, e5.z, e5.w,
+                                e6.x, e6.y, e6.z, e6.w, e7.x, e7.y, e7.z, e7.w};
         announce_prev();
-        ptx::tmem_st_16cols(a_dst + s * kACols, v);
-      } else {
-        // subblock p of the slice
-        const uint2 c = *reinterpret_cast<const uint2*>(stg);
-        const __half2 s2 = __low2half2(ue4m3x2_to_half2((sc >> (8 * p)) & 0xFFu));
-        const uint4 e0 = expand8(c.x, s2), e1 = expand8(c.y, s2);
-        const uint32_t v[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-        announce_prev();
-        ptx::tmem_st_8cols(a_dst + s * kACols, v);
+        ptx::tmem_st_32cols(a_dst + s * kACols, v);
       }
       issue(kb + kCStages - 1);
       ++stored;
@@ -614,7 +632,7 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(2 * M_pad)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBTc)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kSubK), static_cast<cuuint32_t>(kBTc)};
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, act, dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
