@@ -1,0 +1,124 @@
+"""Host-side logic of bench.py, on the CPU: the multi-rank timing plumbing
+(barrier and max over ranks) on two gloo ranks, the reference arm launched
+as two ranks, the gating of ncu traffic figures by kernel-source hash, and
+the workload table."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out_dir: str) -> None:
+    os.environ.update(WORLD_SIZE=str(world), RANK=str(rank), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench as b
+    d = b.Dist()
+    d.init("gloo")
+    d.barrier()
+    # every rank reports its own "time"; all must agree on the largest
+    m = d.max(10.0 + 3.5 * rank, "cpu")
+    d.barrier()
+    d.close()
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"rank": rank, "max": m}, f)
+
+
+def test_dist_max_over_two_gloo_ranks(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    got = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(2)]
+    assert [g["max"] for g in got] == [13.5, 13.5]
+
+
+def test_dist_single_rank_is_identity():
+    d = bench.Dist()
+    if d.world != 1:
+        pytest.skip("run outside a launcher")
+    d.init("gloo")
+    d.barrier()
+    assert d.max(2.25, "cpu") == 2.25
+    d.close()
+
+
+def test_reference_arm_under_two_ranks_prints_one_line():
+    """torchrun with 2 ranks: rank 0 times the oracle and prints the JSON
+    line, rank 1 exits 0 without work."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--workload", "gemv_4096", "--steps", "3", "--warmup", "3", "--cpu-seconds", "0.3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 3
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["config"]["workload"] == "gemv_4096"
+
+
+def test_warmup_below_three_is_rejected():
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--warmup", "2"])
+
+
+def _fake_tree(tmp_path, kernel_text: bytes, profile: str):
+    csrc = tmp_path / "bit_weight_quantized_nvq_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_bytes(kernel_text)
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "kern_wl.md").write_text(profile)
+
+
+def test_traffic_is_used_only_for_the_measured_sources(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    _fake_tree(tmp_path, b"kernel v1", "placeholder")
+    h1 = bench.source_hash("k.cu")
+    (tmp_path / "profiles" / "kern_wl.md").write_text(
+        f"# summary\n\nsource_hash: {h1}\ndram_bytes_per_launch: 123456\n")
+    assert bench.profiled_traffic("kern", "wl", h1) == 123456.0
+    # the kernel changed since the counters were taken: no traffic figure
+    (tmp_path / "bit_weight_quantized_nvq_b200" / "csrc" / "k.cu").write_bytes(b"kernel v2")
+    h2 = bench.source_hash("k.cu")
+    assert h2 != h1
+    assert bench.profiled_traffic("kern", "wl", h2) is None
+    # no summary, or a summary without the bytes line
+    assert bench.profiled_traffic("other", "wl", h1) is None
+    (tmp_path / "profiles" / "kern_wl.md").write_text(f"source_hash: {h1}\n")
+    assert bench.profiled_traffic("kern", "wl", h1) is None
+
+
+def test_workload_table():
+    for name, bound in (("decode_sweep", "hbm"), ("gemv_4096", "hbm"), ("small_batch_m8", "hbm"),
+                        ("prefill_m256", "tensor"), ("prefill_m2048", "tensor"),
+                        ("stack_decode", "hbm"), ("stack_prefill", "tensor")):
+        wk = bench.make_workload(name)
+        assert wk.bound == bound, name
+        assert wk.config()["workload"] == name
+    with pytest.raises(SystemExit):
+        bench.make_workload("no_such_workload")
