@@ -259,3 +259,39 @@ def test_planted_fp16_bias_error_is_caught(monkeypatch):
     monkeypatch.setattr(onvq, "fp16_values", lambda: real * 2.0)
     assert not golden_ok(onvq)
     assert not _brute_force_ok(onvq)
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 3, 64), (3, 4, 128)])
+def test_sum_abs_terms_against_exact_subblock_loop(M, N, K):
+    """sum|terms| (the scale of the accuracy bound) against an explicit loop
+    over subblocks in exact rationals: |0.5 * g * s_w * d_a * isum| per
+    subblock, with isum recomputed from the OCP E2M1 list."""
+    rng = np.random.default_rng(7000 + M * 100 + N * 10 + K)
+    codes, scales, g, q, d = random_case(rng, M, N, K)
+    e2m1 = lambda c: (-1 if c & 8 else 1) * OCP_E2M1[c & 7]
+    isum = o.subblock_sums(codes, q)
+    sa = o.sum_abs_terms(isum, scales, g, d)
+    for m in range(M):
+        dv = [struct.unpack("<e", struct.pack("<H", int(b)))[0] for b in d[m]]
+        for n in range(N):
+            total = Fraction(0)
+            for sb in range(K // 16):
+                s = 0
+                for k in range(16 * sb, 16 * sb + 16):
+                    byte = int(codes[n, k // 2])
+                    c = (byte & 0xF) if k % 2 == 0 else (byte >> 4)
+                    s += int(2 * e2m1(c)) * int(q[m, k])
+                term = (Fraction(1, 2) * Fraction(float(g)) * Fraction(E4M3[int(scales[n, sb])])
+                        * Fraction(dv[sb // 2]) * s)
+                total += abs(term)
+            # exact up to the fp64 rounding of the sum (a dropped 0.5 or a
+            # wrong scale index would miss by far more)
+            assert abs(Fraction(float(sa[m, n])) - total) <= Fraction(2.0 ** -50) * total
+
+
+def test_tolerance_is_the_stated_bound():
+    """|y - y_ref| <= 1e-5 * sum|terms| + 1e-6, elementwise."""
+    assert o.tolerance(0.0) == pytest.approx(1e-6, rel=0, abs=1e-18)
+    assert o.tolerance(1.0) == pytest.approx(1e-5 + 1e-6, rel=1e-15)
+    assert np.allclose(o.tolerance(np.array([2.0, 1e3])), [2e-5 + 1e-6, 1e-2 + 1e-6],
+                       rtol=1e-15, atol=0)
