@@ -693,8 +693,8 @@ def run_nvq(args, dist: Dist):
     if args.workload == "decode_sweep" and dist.world == 1 and not args.no_prefill_summary:
         extra["prefill_gemm"] = prefill_summary(device, peaks)
 
-    cpu = None
-    if dist.rank == 0 and not args.no_cpu_baseline:
+    cpu = None   # the oracle's host-core baseline: rank 0 of a 1-GPU run only
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wk, args.cpu_seconds)
 
     h2d, d2h = wk.e2e_bytes()
