@@ -269,9 +269,6 @@ class GemvWorkload:
             c["y_host"] = torch.empty((self.M, N), dtype=torch.float32).pin_memory()
             self.cases.append(c)
 
-    def fused(self, K):
-        return False   # the separate quantiser overlaps the GEMV and is faster here
-
     def config(self):
         act = "fp32 -> Q8_0 on the GPU every step (nvq_quantize_act_q8_0)"
         return {"workload": self.name, "M": self.M,
@@ -293,26 +290,20 @@ class GemvWorkload:
         activations (fp32 when quantised inside the kernel, else Q8_0) and
         the fp32 output."""
         M, K, N = self.M, c["K"], c["N"]
-        act = 4 * M * K if self.fused(K) else M * K * (1 + 2 / 32)
-        return N * K * WEIGHT_BYTES_PER_ELEMENT + act + 4 * M * N
+        return N * K * WEIGHT_BYTES_PER_ELEMENT + M * K * (1 + 2 / 32) + 4 * M * N
 
     def launches_per_step(self):
-        return sum(1 if self.fused(c["K"]) else 2 for c in self.cases)
+        return 2 * len(self.cases)
 
     def step(self, stream, log=None, e2e=False):
         capi = self.capi
         for c in self.cases:
             if e2e:
                 c["x"].copy_(c["x_host"], non_blocking=True)
-            fused = self.fused(c["K"])
-            if not fused:
-                capi.quantize_act_q8_0(c["x"], c["q"], c["d"], stream=stream)
+            capi.quantize_act_q8_0(c["x"], c["q"], c["d"], stream=stream)
             if log is not None:
                 log.begin(stream)
-            if fused:
-                capi.quant_gemv(c["codes"], c["scales"], c["g"], c["x"], c["y"], stream=stream)
-            else:
-                capi.gemv(c["codes"], c["scales"], c["g"], c["q"], c["d"], c["y"], stream=stream)
+            capi.gemv(c["codes"], c["scales"], c["g"], c["q"], c["d"], c["y"], stream=stream)
             if log is not None:
                 log.end(stream, self.kernel_amount(c))
             if e2e:

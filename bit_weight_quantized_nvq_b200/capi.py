@@ -44,14 +44,15 @@ SIGNATURES = {
     "nvq_quantize_act_q8_0": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp]),
     "nvq_gemv": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp]),
-    "nvq_quant_gemv": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp, _vp]),
     "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "nvq_gemm_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                         _c_i64, _vp, _vp]),
-    "nvq_debug_subblock_sums": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _c_i64, _vp,
-                                               _vp]),
+    "nvq_debug_subblock_sums": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp,
+                                               _vp, _c_i64, _vp, _vp, _vp]),
+    "nvq_error_flags": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint), ctypes.c_int]),
+    "nvq_debug_stalled_wait": (ctypes.c_int, [ctypes.c_uint64, _vp, _vp]),
     "nvq_decoder_stack": (ctypes.c_int, [ctypes.POINTER(Linear), _c_i64, _vp, _c_i64,
                                          ctypes.POINTER(_vp), _vp, ctypes.c_size_t, _vp]),
     "nvq_decoder_stack_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Linear), _c_i64]),
@@ -155,24 +156,6 @@ def gemv(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
     return y
 
 
-def quant_gemv_supported(K: int) -> bool:
-    """Whether nvq_quant_gemv handles this K (asked of the library with an
-    empty product, which launches nothing)."""
-    return _lib.nvq_quant_gemv(None, None, 1.0, 0, K, None, None, None) == NVQ_OK
-
-
-def quant_gemv(codes: torch.Tensor, scales: torch.Tensor, g: float, x: torch.Tensor,
-               y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Q8_0 of one fp32 token fused into the decode GEMV: y[1, N] fp32."""
-    N = codes.shape[0]
-    M, K = x.shape
-    if y is None:
-        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    _check("nvq_quant_gemv", _lib.nvq_quant_gemv(
-        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(x), _ptr(y), _stream(stream)))
-    return y
-
-
 def gemm_workspace_size(M: int, N: int, K: int) -> int:
     return int(_lib.nvq_gemm_workspace_size(M, N, K))
 
@@ -209,16 +192,40 @@ def gemm_noalloc(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.T
     return y
 
 
-def debug_subblock_sums(codes: torch.Tensor, q: torch.Tensor,
-                        isum: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Integer per-16 subblock sums of the GEMV: int32 [M, N, K/16]."""
+def debug_subblock_sums(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
+                        d: torch.Tensor, y: torch.Tensor | None = None,
+                        isum: torch.Tensor | None = None, stream=None):
+    """nvq_gemv that also exports its integer per-16 subblock sums:
+    returns (y fp32 [M, N], isum int32 [M, N, K/16])."""
     N = codes.shape[0]
     M, K = q.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=q.device)
     if isum is None:
         isum = torch.empty((M, N, K // 16), dtype=torch.int32, device=q.device)
     _check("nvq_debug_subblock_sums", _lib.nvq_debug_subblock_sums(
-        _ptr(codes), N, K, _ptr(q), M, _ptr(isum), _stream(stream)))
-    return isum
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y), _ptr(isum),
+        _stream(stream)))
+    return y, isum
+
+
+FLAG_GEMV_TIMEOUT = 1
+FLAG_GEMM_TIMEOUT = 2
+
+
+def error_flags(clear: bool = False) -> int:
+    """Device-side error flags of the current device (NVQ_FLAG_* bits);
+    synchronous.  Read them after synchronising the streams used."""
+    v = ctypes.c_uint(0)
+    _check("nvq_error_flags", _lib.nvq_error_flags(ctypes.byref(v), 1 if clear else 0))
+    return int(v.value)
+
+
+def debug_stalled_wait(limit_ns: int, result: torch.Tensor, stream=None) -> None:
+    """Test-only: one bounded pipeline wait that can never complete
+    (nvq_debug_stalled_wait); result is a device int32 [2] tensor."""
+    _check("nvq_debug_stalled_wait", _lib.nvq_debug_stalled_wait(
+        int(limit_ns), _ptr(result), _stream(stream)))
 
 
 class DecoderStack:

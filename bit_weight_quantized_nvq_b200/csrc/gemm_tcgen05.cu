@@ -52,7 +52,6 @@
 //     an error flag and the CTA drains what it issued, and the pair frees
 //     TMEM together after a cluster barrier.
 #include <algorithm>
-#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -564,6 +563,27 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 int64_t padded_tokens(int64_t M) { return (M + kBT - 1) / kBT * kBT; }
 
+// The scratch array's device address in the current context.  Host code may
+// not use the array's name as an address (it names a host-side shadow), so
+// the address is looked up with cudaGetSymbolAddress, with the device
+// current, and cached per device together with the context it was looked up
+// in; a different current context (for example after cudaDeviceReset) makes
+// the next call look it up again.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 }  // namespace
 
 size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
@@ -573,40 +593,40 @@ size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
 
 size_t gemm_noalloc_limit() { return kNoAllocScratchBytes; }
 
-// The scratch array's device address on the current device.  Host code may
-// not use the array's name as an address (it names a host-side shadow), so
-// the address is looked up with cudaGetSymbolAddress, once per device with
-// that device current, and cached.
 cudaError_t gemm_noalloc_scratch(void** out) {
   constexpr int kMaxDevices = 64;
-  static std::atomic<void*> cache[kMaxDevices];
+  struct Entry {
+    CUcontext ctx;
+    void* ptr;
+  };
+  static Entry cache[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  void* p = cache[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(mu);
-    p = cache[dev].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      e = cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch);
-      if (e != cudaSuccess) return e;
-      cache[dev].store(p, std::memory_order_release);
-    }
+  CUcontext ctx = nullptr;
+  if (CtxGetCurrentFn get = ctx_get_current()) get(&ctx);
+  std::lock_guard<std::mutex> lock(mu);
+  Entry& c = cache[dev];
+  if (c.ptr == nullptr || c.ctx != ctx) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_gemm_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    c.ptr = p;
+    c.ctx = ctx;
   }
-  *out = p;
+  *out = c.ptr;
   return cudaSuccess;
 }
 
-unsigned int gemm_error_flags(bool clear) {
-  unsigned int v = 0;
-  cudaMemcpyFromSymbol(&v, g_gemm_error_flags, sizeof(v));
-  if (clear) {
+cudaError_t gemm_error_flags(bool clear, unsigned int* flags) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_gemm_error_flags, sizeof(unsigned int));
+  if (e == cudaSuccess && clear) {
     const unsigned int zero = 0;
-    cudaMemcpyToSymbol(g_gemm_error_flags, &zero, sizeof(zero));
+    e = cudaMemcpyToSymbol(g_gemm_error_flags, &zero, sizeof(zero));
   }
-  return v;
+  return e;
 }
 
 cudaError_t gemm_expand(const int8_t* q, const uint16_t* d, int64_t M, int64_t K,
@@ -640,15 +660,9 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
       CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static SmemAttrOnce attr;
+  cudaError_t e = attr.ensure(gemm_kernel, static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
   // pairs of CTAs along N: an even number of 128-row tiles (an odd last
   // tile gets an all-padding partner)
   const int64_t tiles_n = (N + kBN - 1) / kBN;
@@ -658,14 +672,14 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
+  cudaLaunchAttribute cluster[1];
+  cluster[0].id = cudaLaunchAttributeClusterDimension;
+  cluster[0].val.clusterDim.x = 2;
+  cluster[0].val.clusterDim.y = 1;
+  cluster[0].val.clusterDim.z = 1;
+  cfg.attrs = cluster;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, map, codes, scales, static_cast<int>(N),
+  e = cudaLaunchKernelEx(&cfg, gemm_kernel, map, codes, scales, static_cast<int>(N),
                                      static_cast<int>(K), static_cast<int>(M),
                                      static_cast<int>(M_pad), g, tok_scale, y);
   if (e != cudaSuccess) return e;

@@ -6,45 +6,40 @@
 // Q8_0 row, one scale per 16 weights): per 16-element subblock,
 //   y += g * s_w * d_a * 0.5 * sum(c_w * q_a),   c_w = 2*E2M1 in -12..12.
 //
-// Design (HBM-bound; every weight byte is read exactly once):
-//  * one warp per weight row; lane l of the warp owns the 32-element chunks
-//    l, l+32, l+64, ... of the row.  A chunk is 16 code bytes (one 128-bit
-//    load), two UE4M3 scale bytes (one 16-bit load) and exactly one Q8_0
-//    activation block (32 int8 codes + one fp16 d), so lanes read disjoint,
-//    contiguous, coalesced spans of both weight streams;
-//  * loads of U chunks are issued before any is used, so each warp keeps
-//    U * 512 bytes of weights in flight;
-//  * codes are decoded in registers to signed bytes c = 2*E2M1 with byte
-//    permutes (no shared-memory table); dp4a (s8 x s8) forms the exact
-//    integer subblock sums, so the +12 bias of the x86 unsigned-by-signed
-//    dot is not needed here;
-//  * the two subblock sums of a chunk are rescaled by their UE4M3 scales,
-//    multiplied by the chunk's d and accumulated in fp32; the activation
-//    block is read through L1 (it is shared by every row on the SM);
-//  * one shuffle reduction per row, then y = 0.5*g*acc.
+// Arithmetic shared by every schedule (HBM-bound; every weight byte is read
+// exactly once):
+//  * lane l of a warp owns whole 32-element chunks of a row: 16 code bytes
+//    (one 128-bit load), two UE4M3 scale bytes and exactly one Q8_0
+//    activation block (32 int8 codes + one fp16 d);
+//  * codes are decoded in registers with byte permutes (no shared-memory
+//    table) and the two exact integer subblock sums of a chunk are formed
+//    with dp4a; they are rescaled by their UE4M3 scales, multiplied by the
+//    chunk's d and accumulated in fp32;
+//  * one shuffle reduction per row (and, for rows split over several warps,
+//    a fixed-order sum of the warps' partials), then y = 0.5*g*acc.
+// Every kernel has an ISUM instantiation that also stores the integer
+// subblock sums it formed, isum[m, n, 2c + h] for chunk c, half h, so that
+// nvq_debug_subblock_sums can export the sums of the very code that
+// produces y (the y it writes is the same bit pattern).
 //
-// Three schedules share that arithmetic:
-//  * gemv_m1_kernel (M = 1, K % 256 == 0; the decode path): one CTA per SM
-//    owning a balanced row range; a producer warp streams groups of 16
-//    contiguous rows (whole K, or K segments of at most 5120) into a
-//    4-stage ring of ~46 KB stages with 1-D TMA bulk copies; 16 consumer
-//    warps own one row each.  The activation block of every chunk is staged
-//    once per CTA in shared memory as conflict-free 16-byte vectors (two
-//    halves of the 32 codes, and {d, corr0, corr1}); the weights are decoded
-//    to the +12-biased integer LUT of the "Bias trick" paragraph (9
-//    operations per 8 codes instead of 11) and the bias is removed by
-//    starting each subblock's dp4a chain at corr = -12 * bsum16, precomputed
-//    per activation subblock.  (The register schedule below goes further and
-//    feeds both table halves to dp4a instead of OR-merging them.)  The chunk loop is fully unrolled for 4 or 5
-//    chunks per lane so all shared-memory loads of a stage are in flight
-//    together.  The consumers are instruction-bound, so these savings matter.
-//  * gemv_tma_kernel (K % 256 == 0, every workload shape): persistent CTAs,
-//    one per half SM, each owning a contiguous, balanced range of rows.  A
-//    producer warp streams groups of 8 rows (the whole K, or a K segment of
-//    at most 5120 elements) into a 4-stage shared-memory ring with 1-D TMA
-//    bulk copies; 8 consumer warps each own one row of the group and decode
-//    from shared memory.  Memory-level parallelism comes from the ring (up
-//    to ~90 KB in flight per CTA), not from registers.
+// Schedules:
+//  * gemv_m1_reg_kernel (M = 1, K = 1024 * T for the common T; the decode
+//    path): one CTA per SM owning a balanced row range; a producer thread
+//    streams stages of R whole contiguous rows (two 1-D TMA bulk copies,
+//    <= 46 KB, 4 stages in flight); 16 consumer warps.  Every lane always
+//    handles the same chunk positions of every row, so its activation codes,
+//    d and the bias corrections sit in registers for the whole kernel.  The
+//    weights are decoded to the +12-biased integer LUT of the "Bias trick"
+//    paragraph with sign-replicating byte permutes, and the bias is removed
+//    by starting each subblock's dp4a chain at corr = -12 * bsum16.
+//  * gemv_m1_kernel (M = 1, other K % 256 == 0): the same ring with groups
+//    of 16 rows (whole K, or K segments of at most 5120 elements) and the
+//    activations staged once per CTA in shared memory; biased LUT with an
+//    OR-merge of the two table halves.
+//  * gemv_tma_kernel (M = 2..16, or M = 1 when the shared memory of the M = 1
+//    schedule does not fit; K % 256 == 0): persistent CTAs, two per SM, each
+//    owning a balanced row range; groups of 8 rows through a 4-stage ring;
+//    the signed LUT, decoded once and used for all M tokens.
 //  * gemv_kernel (any K % 64 == 0): one warp per row, loads straight to
 //    registers.
 #include <algorithm>
@@ -58,8 +53,8 @@
 namespace nvq {
 namespace {
 
-constexpr int kWarps = 4;        // rows per CTA
-constexpr int kUnroll = 4;       // chunks per lane in flight
+constexpr int kWarps = 4;        // rows per CTA of gemv_kernel
+constexpr int kUnroll = 4;       // chunks per lane in flight in gemv_kernel
 
 // TMA-staged schedule
 constexpr int kTmaConsumers = 8;                  // consumer warps = rows per group
@@ -68,26 +63,36 @@ constexpr int kTmaThreads = (kTmaConsumers + 1) * 32;
 constexpr int kTmaMaxSeg = 5120;                  // K elements per stage and row
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per pipeline wait
 
-// bit 0: a pipeline wait of the GEMV timed out
+// bit 0 (NVQ_FLAG_GEMV_TIMEOUT): a pipeline wait of a GEMV kernel timed out
 __device__ unsigned int g_gemv_error_flags = 0;
 
-__device__ __forceinline__ float gemv_chunk_dot(const uint4 w, uint32_t s2, const int8_t* q,
-                                                const __half* d, int c) {
-  uint32_t cw[8];
+__device__ __forceinline__ void raise_timeout() { atomicOr(&g_gemv_error_flags, 1u); }
+
+// Store the two subblock sums of chunk c of row n for token m.
+__device__ __forceinline__ void store_isum(int32_t* isum, int64_t m, int N, int n, int K, int c,
+                                           int i0, int i1) {
+  int2* dst = reinterpret_cast<int2*>(isum + (m * N + n) * static_cast<int64_t>(K >> 4));
+  dst[c] = make_int2(i0, i1);
+}
+
+// The two signed-LUT subblock sums of one chunk against token m's block c.
+__device__ __forceinline__ int2 chunk_isums(const uint32_t (&cw)[8], const int8_t* q, int c) {
+  const uint4* qa = reinterpret_cast<const uint4*>(q) + 2 * c;
+  const uint4 q0 = __ldg(qa);
+  const uint4 q1 = __ldg(qa + 1);
+  int2 r;
+  r.x = dev::dp4a(cw[0], q0.x, dev::dp4a(cw[1], q0.y,
+        dev::dp4a(cw[2], q0.z, dev::dp4a(cw[3], q0.w, 0))));
+  r.y = dev::dp4a(cw[4], q1.x, dev::dp4a(cw[5], q1.y,
+        dev::dp4a(cw[6], q1.z, dev::dp4a(cw[7], q1.w, 0))));
+  return r;
+}
+
+__device__ __forceinline__ void decode_chunk_signed(const uint4 w, uint32_t (&cw)[8]) {
   dev::decode_e2m1x8(w.x, cw[0], cw[1]);
   dev::decode_e2m1x8(w.y, cw[2], cw[3]);
   dev::decode_e2m1x8(w.z, cw[4], cw[5]);
   dev::decode_e2m1x8(w.w, cw[6], cw[7]);
-  const float2 s = dev::ue4m3x2_to_float2(s2);
-  const uint4* qa = reinterpret_cast<const uint4*>(q) + 2 * c;
-  const uint4 q0 = __ldg(qa);
-  const uint4 q1 = __ldg(qa + 1);
-  const float dm = __half2float(__ldg(d + c));
-  const int i0 = dev::dp4a(cw[0], q0.x, dev::dp4a(cw[1], q0.y,
-                 dev::dp4a(cw[2], q0.z, dev::dp4a(cw[3], q0.w, 0))));
-  const int i1 = dev::dp4a(cw[4], q1.x, dev::dp4a(cw[5], q1.y,
-                 dev::dp4a(cw[6], q1.z, dev::dp4a(cw[7], q1.w, 0))));
-  return dm * fmaf(s.x, static_cast<float>(i0), s.y * static_cast<float>(i1));
 }
 
 // Shared memory of the TMA schedule: kTmaStages stages of
@@ -101,7 +106,7 @@ __host__ __device__ constexpr uint32_t tma_smem_bytes(int seg) {
 }
 
 // ---------------------------------------------------------------------------
-// M = 1 schedule
+// M = 1 schedule, activations staged in shared memory
 // ---------------------------------------------------------------------------
 constexpr int kM1Consumers = 16;                       // rows per group
 constexpr int kM1Threads = (kM1Consumers + 1) * 32;    // + producer warp
@@ -126,11 +131,12 @@ __host__ __device__ constexpr uint32_t m1_smem_bytes(int K, int seg) {
          2 * kM1Stages * 8 + 16;
 }
 
-template <int NPL>   // chunks per lane per stage (seg / 1024); 0 = any seg
+template <int NPL, bool ISUM>   // NPL: chunks per lane per stage (seg / 1024); 0 = any seg
 __global__ void __launch_bounds__(kM1Threads, 1)
 gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                float half_g, int N, int K, int seg, const int8_t* __restrict__ q,
-               const __half* __restrict__ d, float* __restrict__ y) {
+               const __half* __restrict__ d, float* __restrict__ y,
+               int32_t* __restrict__ isum) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t stage_bytes = m1_stage_bytes(seg);
   const uint32_t codes_bytes = kM1Consumers * (seg / 2);
@@ -187,7 +193,7 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
       const uint32_t ph = (it / kM1Stages) & 1;
       if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
         *abort_flag = 1;
-        atomicOr(&g_gemv_error_flags, 1u);
+        raise_timeout();
         break;
       }
       const int grp = it / nseg, sg = it % nseg;
@@ -229,7 +235,7 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
     const uint32_t ph = (it / kM1Stages) & 1;
     if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
       *abort_flag = 1;
-      atomicOr(&g_gemv_error_flags, 1u);
+      raise_timeout();
       break;
     }
     const int grp = it / nseg, sg = it % nseg;
@@ -240,7 +246,8 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
       const uint4* cw = reinterpret_cast<const uint4*>(st + warp * (seg / 2));
       const uint16_t* sw = reinterpret_cast<const uint16_t*>(st + codes_bytes + warp * (seg / 16));
       const int cbase = sg * nch;
-      auto chunk = [&](const uint4 w, uint32_t s2, const uint4 a, const uint4 b, const ActMeta mt) {
+      auto chunk = [&](const uint4 w, uint32_t s2, const uint4 a, const uint4 b, const ActMeta mt,
+                       int cidx) {
         uint32_t c[8];
         dev::decode_e2m1x8_biased(w.x, c[0], c[1]);
         dev::decode_e2m1x8_biased(w.y, c[2], c[3]);
@@ -250,6 +257,7 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
                        dev::dp4a_us(c[2], a.z, dev::dp4a_us(c[3], a.w, mt.corr0))));
         const int i1 = dev::dp4a_us(c[4], b.x, dev::dp4a_us(c[5], b.y,
                        dev::dp4a_us(c[6], b.z, dev::dp4a_us(c[7], b.w, mt.corr1))));
+        if constexpr (ISUM) store_isum(isum, 0, N, row0 + warp, K, cidx, i0, i1);
         const float2 sf = dev::ue4m3x2_to_float2(s2);
         acc = fmaf(mt.d, fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
       };
@@ -267,11 +275,11 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
           mt[i] = meta[cbase + j];
         }
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) chunk(w[i], s2[i], a[i], b[i], mt[i]);
+        for (int i = 0; i < NPL; ++i) chunk(w[i], s2[i], a[i], b[i], mt[i], cbase + lane + 32 * i);
       } else {
 #pragma unroll 2
         for (int j = lane; j < nch; j += 32)
-          chunk(cw[j], sw[j], qa[cbase + j], qb[cbase + j], meta[cbase + j]);
+          chunk(cw[j], sw[j], qa[cbase + j], qb[cbase + j], meta[cbase + j], cbase + j);
       }
     }
     __syncwarp();
@@ -292,11 +300,7 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
 // Every lane of a consumer warp handles the same NPL chunk positions of
 // every row it ever processes, so the activation data of those chunks (32
 // codes, d and the two bias corrections) is loaded once into registers and
-// held there for the whole kernel.  With XF32 the kernel takes the fp32
-// activations instead and performs the Q8_0 quantisation itself, once per
-// CTA into shared memory (the same IEEE operations as
-// nvq_quantize_act_q8_0, so the codes are identical); every CTA repeats
-// that work, so it pays off only where a launch costs more than it.
+// held there for the whole kernel.
 // A row is split across WPR warps (warp part p owns the p-th contiguous K
 // segment of 1024 * NPL elements); a stage is R = 16/WPR (or fewer, to fit
 // 46 KB) whole, contiguous rows, fetched with two bulk copies.  With
@@ -314,12 +318,10 @@ __host__ __device__ constexpr int reg_rows(int K, int wpr) {
   while (r > 1 && static_cast<uint32_t>(r) * (K / 2 + K / 16) > kRegStageMax) --r;
   return r;
 }
-// stages | row partials [stage][warp] | activation words [K/32][8] |
-// ActMeta [K/32] | barriers
+// stages | row partials [stage][warp] | barriers
 __host__ __device__ constexpr uint32_t reg_smem_bytes(int K, int wpr) {
   return kM1Stages * static_cast<uint32_t>(reg_rows(K, wpr)) * (K / 2 + K / 16) +
-         kM1Stages * kM1Consumers * 4 + static_cast<uint32_t>(K / 32) * 48 +
-         2 * kM1Stages * 8 + 16;
+         kM1Stages * kM1Consumers * 4 + 2 * kM1Stages * 8 + 16;
 }
 
 __device__ __forceinline__ void grid_dependency_wait() {
@@ -329,69 +331,20 @@ __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Stage chunk c of the activation vector: lane j (0..7) of a group of eight
-// handles elements 4j..4j+3, i.e. word j of the chunk's 32 codes.  With
-// XF32 the codes are quantised here exactly as the Q8_0 quantiser does
-// (amax over the block by shuffles, IEEE divisions, rint, clamp, fp16 d).
-template <bool XF32>
-__device__ __forceinline__ void stage_act_chunk(int c, int j, unsigned gmask,
-                                                const float* __restrict__ x,
-                                                const int8_t* __restrict__ q,
-                                                const __half* __restrict__ d,
-                                                uint32_t* words, ActMeta* meta) {
-  uint32_t word;
-  float dval;
-  if constexpr (XF32) {
-    const float4 v = reinterpret_cast<const float4*>(x)[8 * c + j];
-    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-    a = fmaxf(a, __shfl_xor_sync(gmask, a, 1, 8));
-    a = fmaxf(a, __shfl_xor_sync(gmask, a, 2, 8));
-    a = fmaxf(a, __shfl_xor_sync(gmask, a, 4, 8));
-    const float d32 = __fdiv_rn(a, 127.0f);
-    word = 0;
-    if (d32 > 0.0f) {
-      const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        int qi = __float2int_rn(__fdiv_rn(e[i], d32));
-        qi = max(-127, min(127, qi));
-        word |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * i);
-      }
-    }
-    dval = __half2float(__float2half_rn(d32));
-  } else {
-    word = reinterpret_cast<const uint32_t*>(q)[8 * c + j];
-    dval = __half2float(d[c]);
-  }
-  int s = dev::dp4a(word, 0x01010101u, 0);
-  s += __shfl_xor_sync(gmask, s, 1, 8);
-  s += __shfl_xor_sync(gmask, s, 2, 8);   // lanes 0-3: subblock 0, lanes 4-7: subblock 1
-  words[8 * c + j] = word;
-  if (j == 0) {
-    meta[c].d = dval;
-    meta[c].corr0 = -12 * s;
-    meta[c].pad = 0;
-  }
-  if (j == 4) meta[c].corr1 = -12 * s;
-}
-
-template <int NPL, int WPR, bool XF32>
+template <int NPL, int WPR, bool ISUM>
 __global__ void __launch_bounds__(kM1Threads, 1)
 gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                   float half_g, int N, int K, const float* __restrict__ x,
-                   const int8_t* __restrict__ q, const __half* __restrict__ d,
-                   float* __restrict__ y) {
+                   float half_g, int N, int K, const int8_t* __restrict__ q,
+                   const __half* __restrict__ d, float* __restrict__ y,
+                   int32_t* __restrict__ isum) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int R = reg_rows(K, WPR);
   const int active = R * WPR;                      // consumer warps in use
-  const int nchunk = K / 32;
   const uint32_t row_code = K / 2, row_scale = K / 16;
   const uint32_t stage_bytes = static_cast<uint32_t>(R) * (row_code + row_scale);
   const uint32_t codes_bytes = static_cast<uint32_t>(R) * row_code;
   float* part = reinterpret_cast<float*>(smem + kM1Stages * stage_bytes);  // [stage][warp]
-  uint32_t* act_words = reinterpret_cast<uint32_t*>(part + kM1Stages * kM1Consumers);
-  ActMeta* meta = reinterpret_cast<ActMeta*>(act_words + 8 * nchunk);
-  uint64_t* full = reinterpret_cast<uint64_t*>(meta + nchunk);
+  uint64_t* full = reinterpret_cast<uint64_t*>(part + kM1Stages * kM1Consumers);
   uint64_t* empty = full + kM1Stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kM1Stages);
 
@@ -436,7 +389,7 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
       const uint32_t ph = (it / kM1Stages) & 1;
       if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
         *abort_flag = 1;
-        atomicOr(&g_gemv_error_flags, 1u);
+        raise_timeout();
         ok = false;
         break;
       }
@@ -458,7 +411,7 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
         if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + it % kM1Stages),
                                     (it / kM1Stages) & 1, abort_flag, kWaitLimitNs)) {
           *abort_flag = 1;
-          atomicOr(&g_gemv_error_flags, 1u);
+          raise_timeout();
           break;
         }
         finalize(it);
@@ -472,54 +425,33 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
   }
 
   // ------------- consumers: warp w = (row w / WPR, part w % WPR) -------------
+  if (warp >= active) return;
   const int rl = warp / WPR;
   const int p = warp % WPR;
   uint4 qa[NPL], qb[NPL];
   float dd[NPL];
   int c0[NPL], c1[NPL];
-  if constexpr (XF32) {
-    // quantise the fp32 token once per CTA into shared memory (all 16 warps)
-    const unsigned gmask = 0xFFu << (lane & 24);
-    for (int cb = warp * 4; cb < nchunk; cb += kM1Consumers * 4) {
-      const int c = cb + (lane >> 3);
-      if (c < nchunk) stage_act_chunk<true>(c, lane & 7, gmask, x, q, d, act_words, meta);
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kM1Consumers * 32) : "memory");
-    if (warp >= active) return;
+  // each lane loads its own activation chunks straight into registers
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int c = p * (NPL * 32) + lane + 32 * i;   // chunk index in the row
-      qa[i] = reinterpret_cast<const uint4*>(act_words)[2 * c];
-      qb[i] = reinterpret_cast<const uint4*>(act_words)[2 * c + 1];
-      const ActMeta mt = meta[c];
-      dd[i] = mt.d;
-      c0[i] = mt.corr0;
-      c1[i] = mt.corr1;
-    }
-  } else {
-    // Q8_0 input: each lane loads its own chunks straight into registers
-    if (warp >= active) return;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int c = p * (NPL * 32) + lane + 32 * i;
-      const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * c;
-      qa[i] = __ldg(src);
-      qb[i] = __ldg(src + 1);
-      dd[i] = __half2float(__ldg(d + c));
-      const int s0 = dev::dp4a(qa[i].x, 0x01010101u, dev::dp4a(qa[i].y, 0x01010101u,
-                     dev::dp4a(qa[i].z, 0x01010101u, dev::dp4a(qa[i].w, 0x01010101u, 0))));
-      const int s1 = dev::dp4a(qb[i].x, 0x01010101u, dev::dp4a(qb[i].y, 0x01010101u,
-                     dev::dp4a(qb[i].z, 0x01010101u, dev::dp4a(qb[i].w, 0x01010101u, 0))));
-      c0[i] = -12 * s0;
-      c1[i] = -12 * s1;
-    }
+  for (int i = 0; i < NPL; ++i) {
+    const int c = p * (NPL * 32) + lane + 32 * i;
+    const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * c;
+    qa[i] = __ldg(src);
+    qb[i] = __ldg(src + 1);
+    dd[i] = __half2float(__ldg(d + c));
+    const int s0 = dev::dp4a(qa[i].x, 0x01010101u, dev::dp4a(qa[i].y, 0x01010101u,
+                   dev::dp4a(qa[i].z, 0x01010101u, dev::dp4a(qa[i].w, 0x01010101u, 0))));
+    const int s1 = dev::dp4a(qb[i].x, 0x01010101u, dev::dp4a(qb[i].y, 0x01010101u,
+                   dev::dp4a(qb[i].z, 0x01010101u, dev::dp4a(qb[i].w, 0x01010101u, 0))));
+    c0[i] = -12 * s0;
+    c1[i] = -12 * s1;
   }
   for (int it = 0; it < total; ++it) {
     const int s = it % kM1Stages;
     const uint32_t ph = (it / kM1Stages) & 1;
     if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
       *abort_flag = 1;
-      atomicOr(&g_gemv_error_flags, 1u);
+      raise_timeout();
       break;
     }
     const int row0 = r_begin + it * R;
@@ -541,6 +473,8 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
       for (int i = 0; i < NPL; ++i) {
         const int i0 = dev::dot16_biased(w[i].x, w[i].y, qa[i], c0[i]);
         const int i1 = dev::dot16_biased(w[i].z, w[i].w, qb[i], c1[i]);
+        if constexpr (ISUM)
+          store_isum(isum, 0, N, row0 + rl, K, p * (NPL * 32) + lane + 32 * i, i0, i1);
         const float2 sf = dev::ue4m3x2_to_float2(s2[i]);
         acc = fmaf(dd[i], fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
       }
@@ -557,11 +491,15 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
   }
 }
 
-template <int MT>
+// ---------------------------------------------------------------------------
+// M = 2..16 (and fallback M = 1) schedule: persistent CTAs, TMA ring
+// ---------------------------------------------------------------------------
+template <int MT, bool ISUM>
 __global__ void __launch_bounds__(kTmaThreads, 2)
 gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                 float half_g, int N, int K, int seg, const int8_t* __restrict__ q,
-                const __half* __restrict__ d, float* __restrict__ y) {
+                const __half* __restrict__ d, float* __restrict__ y,
+                int32_t* __restrict__ isum) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t stage_bytes = tma_stage_bytes(seg);
   const uint32_t codes_bytes = kTmaConsumers * (seg / 2);
@@ -597,7 +535,7 @@ gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ s
       const uint32_t ph = (it / kTmaStages) & 1;
       if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
         *abort_flag = 1;
-        atomicOr(&g_gemv_error_flags, 1u);
+        raise_timeout();
         break;
       }
       const int grp = it / nseg, sg = it % nseg;
@@ -642,7 +580,7 @@ gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ s
     const uint32_t ph = (it / kTmaStages) & 1;
     if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
       *abort_flag = 1;
-      atomicOr(&g_gemv_error_flags, 1u);
+      raise_timeout();
       break;
     }
     const int grp = it / nseg, sg = it % nseg;
@@ -655,12 +593,17 @@ gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ s
       const int cbase = sg * nch;
 #pragma unroll 4
       for (int j = lane; j < nch; j += 32) {
-        const uint4 w = sc[j];
-        const uint32_t s2 = ss[j];
+        uint32_t cw[8];
+        decode_chunk_signed(sc[j], cw);
+        const float2 sf = dev::ue4m3x2_to_float2(ss[j]);
+        const int c = cbase + j;
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-          acc[m] += gemv_chunk_dot(w, s2, q + static_cast<size_t>(m) * K,
-                                   d + static_cast<size_t>(m) * (K >> 5), cbase + j);
+        for (int m = 0; m < MT; ++m) {
+          const int2 is = chunk_isums(cw, q + static_cast<size_t>(m) * K, c);
+          if constexpr (ISUM) store_isum(isum, m, N, row0 + warp, K, c, is.x, is.y);
+          const float dm = __half2float(__ldg(d + static_cast<size_t>(m) * (K >> 5) + c));
+          acc[m] += dm * fmaf(sf.x, static_cast<float>(is.x), sf.y * static_cast<float>(is.y));
+        }
       }
     }
     __syncwarp();
@@ -679,11 +622,14 @@ gemv_tma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ s
   }
 }
 
-template <int MT>
+// ---------------------------------------------------------------------------
+// any K % 64 == 0: one warp per row, loads straight to registers
+// ---------------------------------------------------------------------------
+template <int MT, bool ISUM>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
             float half_g, int N, int K, const int8_t* __restrict__ q,
-            const __half* __restrict__ d, float* __restrict__ y) {
+            const __half* __restrict__ d, float* __restrict__ y, int32_t* __restrict__ isum) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (row >= N) return;
@@ -711,22 +657,14 @@ gemv_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scale
       const int c = c0 + u * 32 + lane;
       if (c < nchunk) {
         uint32_t cw[8];
-        dev::decode_e2m1x8(wv[u].x, cw[0], cw[1]);
-        dev::decode_e2m1x8(wv[u].y, cw[2], cw[3]);
-        dev::decode_e2m1x8(wv[u].z, cw[4], cw[5]);
-        dev::decode_e2m1x8(wv[u].w, cw[6], cw[7]);
+        decode_chunk_signed(wv[u], cw);
         const float2 s = dev::ue4m3x2_to_float2(sv[u]);
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          const uint4* qa = reinterpret_cast<const uint4*>(q + static_cast<size_t>(m) * K) + 2 * c;
-          const uint4 q0 = __ldg(qa);
-          const uint4 q1 = __ldg(qa + 1);
+          const int2 is = chunk_isums(cw, q + static_cast<size_t>(m) * K, c);
+          if constexpr (ISUM) store_isum(isum, m, N, row, K, c, is.x, is.y);
           const float dm = __half2float(__ldg(d + static_cast<size_t>(m) * (K >> 5) + c));
-          const int i0 = dev::dp4a(cw[0], q0.x, dev::dp4a(cw[1], q0.y,
-                         dev::dp4a(cw[2], q0.z, dev::dp4a(cw[3], q0.w, 0))));
-          const int i1 = dev::dp4a(cw[4], q1.x, dev::dp4a(cw[5], q1.y,
-                         dev::dp4a(cw[6], q1.z, dev::dp4a(cw[7], q1.w, 0))));
-          acc[m] = fmaf(dm, fmaf(s.x, static_cast<float>(i0), s.y * static_cast<float>(i1)), acc[m]);
+          acc[m] = fmaf(dm, fmaf(s.x, static_cast<float>(is.x), s.y * static_cast<float>(is.y)), acc[m]);
         }
       }
     }
@@ -738,36 +676,25 @@ gemv_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scale
   }
 }
 
-// Integer subblock sums through the same decode and dot code, one warp per
-// row: isum[m, n, 2c + h] for chunk c, half h.
-__global__ void __launch_bounds__(kWarps * 32)
-subblock_sums_kernel(const uint8_t* __restrict__ codes, int N, int K,
-                     const int8_t* __restrict__ q, int M, int32_t* __restrict__ isum) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (row >= N) return;
-  const int nchunk = K >> 5;
-  const uint4* wrow = reinterpret_cast<const uint4*>(codes + static_cast<size_t>(row) * (K >> 1));
-  for (int c = lane; c < nchunk; c += 32) {
-    const uint4 w = dev::ld_stream_v4(wrow + c);
-    uint32_t cw[8];
-    dev::decode_e2m1x8(w.x, cw[0], cw[1]);
-    dev::decode_e2m1x8(w.y, cw[2], cw[3]);
-    dev::decode_e2m1x8(w.z, cw[4], cw[5]);
-    dev::decode_e2m1x8(w.w, cw[6], cw[7]);
-    for (int m = 0; m < M; ++m) {
-      const uint4* qa = reinterpret_cast<const uint4*>(q + static_cast<size_t>(m) * K) + 2 * c;
-      const uint4 q0 = __ldg(qa);
-      const uint4 q1 = __ldg(qa + 1);
-      int2 out;
-      out.x = dev::dp4a(cw[0], q0.x, dev::dp4a(cw[1], q0.y,
-              dev::dp4a(cw[2], q0.z, dev::dp4a(cw[3], q0.w, 0))));
-      out.y = dev::dp4a(cw[4], q1.x, dev::dp4a(cw[5], q1.y,
-              dev::dp4a(cw[6], q1.z, dev::dp4a(cw[7], q1.w, 0))));
-      int2* dst = reinterpret_cast<int2*>(isum + (static_cast<size_t>(m) * N + row) * (K >> 4)) + c;
-      *dst = out;
-    }
-  }
+// ---------------------------------------------------------------------------
+// test-only: a pipeline wait that never completes
+// ---------------------------------------------------------------------------
+// One consumer waits, through the same bounded wait as the GEMV pipelines,
+// for a stage whose producer never issues its copy (the barrier's phase can
+// never complete).  The wait gives up after limit_ns, raises the GEMV
+// timeout flag exactly as a stalled GEMV would, and the kernel returns.
+__global__ void __launch_bounds__(32)
+stalled_wait_kernel(uint64_t limit_ns, int* __restrict__ result) {
+  __shared__ __align__(8) uint64_t full;
+  if (threadIdx.x != 0) return;
+  ptx::mbar_init(ptx::smem_addr(&full), 1);
+  ptx::fence_mbar_init();
+  const uint64_t t0 = ptx::globaltimer_ns();
+  const bool got = ptx::mbar_wait_bounded(ptx::smem_addr(&full), 0, nullptr, limit_ns);
+  if (!got) raise_timeout();
+  result[0] = got ? 1 : 0;
+  const uint64_t us = (ptx::globaltimer_ns() - t0) / 1000;
+  result[1] = us > 0x7fffffffull ? 0x7fffffff : static_cast<int>(us);
 }
 
 // K elements per TMA stage and row: the largest multiple of 256 that divides
@@ -780,66 +707,53 @@ int tma_segment(int64_t K) {
   return 0;
 }
 
-template <int NPL>
+template <int NPL, bool ISUM>
 cudaError_t launch_m1(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
                       int64_t K, int seg, const int8_t* q, const uint16_t* d, float* y,
-                      cudaStream_t stream) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_m1_kernel<NPL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemPerCtaMax));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+                      int32_t* isum, cudaStream_t stream) {
+  static SmemAttrOnce attr;
+  cudaError_t e = attr.ensure(gemv_m1_kernel<NPL, ISUM>, static_cast<int>(kSmemPerCtaMax));
+  if (e != cudaSuccess) return e;
   const int64_t ctas = std::min<int64_t>(device_sm_count(), N);
-  gemv_m1_kernel<NPL><<<static_cast<unsigned>(ctas), kM1Threads,
-                        m1_smem_bytes(static_cast<int>(K), seg), stream>>>(
+  gemv_m1_kernel<NPL, ISUM><<<static_cast<unsigned>(ctas), kM1Threads,
+                              m1_smem_bytes(static_cast<int>(K), seg), stream>>>(
       codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), seg, q,
-      reinterpret_cast<const __half*>(d), y);
+      reinterpret_cast<const __half*>(d), y, isum);
   return cudaGetLastError();
 }
 
-template <int NPL, int WPR, bool XF32>
+template <int NPL, int WPR, bool ISUM>
 cudaError_t launch_m1_reg(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
-                          int64_t K, const float* x, const int8_t* q, const uint16_t* d,
-                          float* y, cudaStream_t stream) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  auto kernel = gemv_m1_reg_kernel<NPL, WPR, XF32>;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemPerCtaMax));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+                          int64_t K, const int8_t* q, const uint16_t* d, float* y,
+                          int32_t* isum, cudaStream_t stream) {
+  auto kernel = gemv_m1_reg_kernel<NPL, WPR, ISUM>;
+  static SmemAttrOnce attr;
+  cudaError_t e = attr.ensure(kernel, static_cast<int>(kSmemPerCtaMax));
+  if (e != cudaSuccess) return e;
   const int64_t ctas = std::min<int64_t>(device_sm_count(), N);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kM1Threads);
   cfg.dynamicSmemBytes = reg_smem_bytes(static_cast<int>(K), WPR);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, codes, scales, 0.5f * g, static_cast<int>(N),
-                            static_cast<int>(K), x, q, reinterpret_cast<const __half*>(d), y);
+                            static_cast<int>(K), q, reinterpret_cast<const __half*>(d), y, isum);
 }
 
 // The register schedule covers K = 1024 * NPL * WPR for the (NPL, WPR) pairs
 // instantiated here; returns cudaErrorNotSupported for other K.
-template <bool XF32>
+template <bool ISUM>
 cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, float g,
-                                   int64_t N, int64_t K, const float* x, const int8_t* q,
-                                   const uint16_t* d, float* y, cudaStream_t stream) {
+                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                                   float* y, int32_t* isum, cudaStream_t stream) {
   if (K % 1024 != 0) return cudaErrorNotSupported;
 #define NVQ_REG(npl, wpr) \
-  return launch_m1_reg<npl, wpr, XF32>(codes, scales, g, N, K, x, q, d, y, stream)
+  return launch_m1_reg<npl, wpr, ISUM>(codes, scales, g, N, K, q, d, y, isum, stream)
   switch (K / 1024) {
     case 4: NVQ_REG(4, 1);
     case 5: NVQ_REG(5, 1);
@@ -856,54 +770,47 @@ cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, 
 #undef NVQ_REG
 }
 
-template <int MT>
+template <int MT, bool ISUM>
 cudaError_t launch_gemv_m(const uint8_t* codes, const uint8_t* scales, float g,
                           int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
-                          float* y, cudaStream_t stream) {
+                          float* y, int32_t* isum, cudaStream_t stream) {
   const int seg = tma_segment(K);
   if (MT == 1) {
     const cudaError_t e =
-        launch_m1_reg_dispatch<false>(codes, scales, g, N, K, nullptr, q, d, y, stream);
+        launch_m1_reg_dispatch<ISUM>(codes, scales, g, N, K, q, d, y, isum, stream);
     if (e != cudaErrorNotSupported) return e;
   }
   if (MT == 1 && seg > 0 && m1_smem_bytes(static_cast<int>(K), seg) <= kSmemPerCtaMax) {
-    if (seg == 5120) return launch_m1<5>(codes, scales, g, N, K, seg, q, d, y, stream);
-    if (seg == 4096) return launch_m1<4>(codes, scales, g, N, K, seg, q, d, y, stream);
-    return launch_m1<0>(codes, scales, g, N, K, seg, q, d, y, stream);
+    if (seg == 5120) return launch_m1<5, ISUM>(codes, scales, g, N, K, seg, q, d, y, isum, stream);
+    if (seg == 4096) return launch_m1<4, ISUM>(codes, scales, g, N, K, seg, q, d, y, isum, stream);
+    return launch_m1<0, ISUM>(codes, scales, g, N, K, seg, q, d, y, isum, stream);
   }
   if (seg > 0) {
     const uint32_t smem = tma_smem_bytes(seg);
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(gemv_tma_kernel<MT>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(tma_smem_bytes(kTmaMaxSeg)));
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
-    }
+    static SmemAttrOnce attr;
+    cudaError_t e = attr.ensure(gemv_tma_kernel<MT, ISUM>,
+                                static_cast<int>(tma_smem_bytes(kTmaMaxSeg)));
+    if (e != cudaSuccess) return e;
     const int64_t ctas = std::min<int64_t>(2 * static_cast<int64_t>(device_sm_count()), N);
-    gemv_tma_kernel<MT><<<static_cast<unsigned>(ctas), kTmaThreads, smem, stream>>>(
+    gemv_tma_kernel<MT, ISUM><<<static_cast<unsigned>(ctas), kTmaThreads, smem, stream>>>(
         codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), seg, q,
-        reinterpret_cast<const __half*>(d), y);
+        reinterpret_cast<const __half*>(d), y, isum);
     return cudaGetLastError();
   }
   const unsigned grid = static_cast<unsigned>((N + kWarps - 1) / kWarps);
-  gemv_kernel<MT><<<grid, kWarps * 32, 0, stream>>>(
+  gemv_kernel<MT, ISUM><<<grid, kWarps * 32, 0, stream>>>(
       codes, scales, 0.5f * g, static_cast<int>(N), static_cast<int>(K), q,
-      reinterpret_cast<const __half*>(d), y);
+      reinterpret_cast<const __half*>(d), y, isum);
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
-                        int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
-                        int64_t M, float* y, cudaStream_t stream) {
+template <bool ISUM>
+cudaError_t launch_gemv_any(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                            int64_t K, const int8_t* q, const uint16_t* d, int64_t M, float* y,
+                            int32_t* isum, cudaStream_t stream) {
   switch (M) {
 #define NVQ_GEMV_CASE(mm) \
-    case mm: return launch_gemv_m<mm>(codes, scales, g, N, K, q, d, y, stream);
+    case mm: return launch_gemv_m<mm, ISUM>(codes, scales, g, N, K, q, d, y, isum, stream);
     NVQ_GEMV_CASE(1) NVQ_GEMV_CASE(2) NVQ_GEMV_CASE(3) NVQ_GEMV_CASE(4)
     NVQ_GEMV_CASE(5) NVQ_GEMV_CASE(6) NVQ_GEMV_CASE(7) NVQ_GEMV_CASE(8)
     NVQ_GEMV_CASE(9) NVQ_GEMV_CASE(10) NVQ_GEMV_CASE(11) NVQ_GEMV_CASE(12)
@@ -913,39 +820,32 @@ cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
   }
 }
 
-bool quant_gemv_supported(int64_t K) {
-  if (K % 1024 != 0) return false;
-  switch (K / 1024) {
-    case 4: case 5: case 6: case 8: case 10: case 12: case 15: case 16: case 20: case 25:
-      return true;
-    default:
-      return false;
-  }
+}  // namespace
+
+cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
+                        int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                        int64_t M, float* y, cudaStream_t stream) {
+  return launch_gemv_any<false>(codes, scales, g, N, K, q, d, M, y, nullptr, stream);
 }
 
-cudaError_t launch_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
-                              int64_t N, int64_t K, const float* x, float* y,
-                              cudaStream_t stream) {
-  return launch_m1_reg_dispatch<true>(codes, scales, g, N, K, x, nullptr, nullptr, y, stream);
+cudaError_t launch_gemv_isum(const uint8_t* codes, const uint8_t* scales, float g,
+                             int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                             int64_t M, float* y, int32_t* isum, cudaStream_t stream) {
+  return launch_gemv_any<true>(codes, scales, g, N, K, q, d, M, y, isum, stream);
 }
 
-unsigned int gemv_error_flags(bool clear) {
-  unsigned int v = 0;
-  cudaMemcpyFromSymbol(&v, g_gemv_error_flags, sizeof(v));
-  if (clear) {
-    const unsigned int zero = 0;
-    cudaMemcpyToSymbol(g_gemv_error_flags, &zero, sizeof(zero));
-  }
-  return v;
-}
-
-cudaError_t launch_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
-                                 const int8_t* q, int64_t M, int32_t* isum,
-                                 cudaStream_t stream) {
-  const unsigned grid = static_cast<unsigned>((N + kWarps - 1) / kWarps);
-  subblock_sums_kernel<<<grid, kWarps * 32, 0, stream>>>(
-      codes, static_cast<int>(N), static_cast<int>(K), q, static_cast<int>(M), isum);
+cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream) {
+  stalled_wait_kernel<<<1, 32, 0, stream>>>(limit_ns, result);
   return cudaGetLastError();
+}
+
+cudaError_t gemv_error_flags(bool clear, unsigned int* flags) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_gemv_error_flags, sizeof(unsigned int));
+  if (e == cudaSuccess && clear) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_gemv_error_flags, &zero, sizeof(zero));
+  }
+  return e;
 }
 
 }  // namespace nvq

@@ -137,20 +137,6 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                                       static_cast<cudaStream_t>(stream)));
 }
 
-nvq_status nvq_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
-                          int64_t N, int64_t K, const float* x, float* y, void* stream) {
-  // x plays the part of q (checked for NULL and alignment); d is not used
-  nvq_status st = check_dot_args(codes, scales, N, K, x, x, 1, y, 1, 1, true);
-  if (st != NVQ_OK) return st;
-  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
-  if (!nvq::quant_gemv_supported(K)) return NVQ_ERR_BAD_SHAPE;
-  if (N == 0) return NVQ_OK;
-  st = check_device();
-  if (st != NVQ_OK) return st;
-  return cuda_status(nvq::launch_quant_gemv(codes, scales, g, N, K, x, y,
-                                            static_cast<cudaStream_t>(stream)));
-}
-
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || K <= 0 || N < 0) return 0;
   return nvq::gemm_workspace_size(M, N, K);
@@ -195,17 +181,44 @@ nvq_status nvq_gemm_noalloc(const uint8_t* codes, const uint8_t* scales, float g
                                       static_cast<cudaStream_t>(stream)));
 }
 
-nvq_status nvq_debug_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
-                                   const int8_t* q, int64_t M, int32_t* isum,
-                                   void* stream) {
-  nvq_status st = check_dot_args(codes, nullptr, N, K, q, nullptr, M, isum, 1, 16,
-                                 false);
+nvq_status nvq_debug_subblock_sums(const uint8_t* codes, const uint8_t* scales, float g,
+                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                                   int64_t M, float* y, int32_t* isum, void* stream) {
+  nvq_status st = check_dot_args(codes, scales, N, K, q, d, M, y, 1, 16, true);
   if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
   if (N == 0 || M == 0) return NVQ_OK;
+  if (!isum) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(isum)) return NVQ_ERR_MISALIGNED;
   st = check_device();
   if (st != NVQ_OK) return st;
-  return cuda_status(nvq::launch_subblock_sums(codes, N, K, q, M, isum,
-                                               static_cast<cudaStream_t>(stream)));
+  return cuda_status(nvq::launch_gemv_isum(codes, scales, g, N, K, q, d, M, y, isum,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+nvq_status nvq_error_flags(unsigned int* flags, int clear) {
+  if (!flags) return NVQ_ERR_INVALID_ARG;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  unsigned int gemv = 0, gemm = 0;
+  cudaError_t e = nvq::gemv_error_flags(clear != 0, &gemv);
+  if (e == cudaSuccess) e = nvq::gemm_error_flags(clear != 0, &gemm);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  *flags = (gemv ? NVQ_FLAG_GEMV_TIMEOUT : 0u) | (gemm ? NVQ_FLAG_GEMM_TIMEOUT : 0u);
+  return NVQ_OK;
+}
+
+nvq_status nvq_debug_stalled_wait(uint64_t limit_ns, int* result, void* stream) {
+  if (!result) return NVQ_ERR_INVALID_ARG;
+  if (limit_ns < 1000 || limit_ns > 1000000000ull) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(result)) return NVQ_ERR_MISALIGNED;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_stalled_wait(limit_ns, result,
+                                              static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

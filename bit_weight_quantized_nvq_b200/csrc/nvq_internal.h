@@ -2,6 +2,7 @@
 // Launchers assume validated arguments (the C ABI layer checks them).
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -18,22 +19,21 @@ cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                         int64_t N, int64_t K, const int8_t* q,
                         const uint16_t* d, int64_t M, float* y,
                         cudaStream_t stream);
+// The same dispatch and kernels, instantiated to also store the integer
+// subblock sums they form (isum int32 [M, N, K/16]).
+cudaError_t launch_gemv_isum(const uint8_t* codes, const uint8_t* scales, float g,
+                             int64_t N, int64_t K, const int8_t* q,
+                             const uint16_t* d, int64_t M, float* y, int32_t* isum,
+                             cudaStream_t stream);
 
-// Q8_0 quantisation of one fp32 token fused into the decode GEMV (M = 1);
-// supported for K = 1024 * T, T in {4, 5, 6, 8, 10, 12, 15, 16, 20, 25}.
-bool quant_gemv_supported(int64_t K);
-cudaError_t launch_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
-                              int64_t N, int64_t K, const float* x, float* y,
-                              cudaStream_t stream);
+// Test-only: a pipeline wait that can never complete, bounded by limit_ns;
+// result[0] = 1 if the wait completed (never), result[1] = microseconds waited.
+cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream);
 
-// Error flags raised by GEMV kernels (bit 0: a pipeline wait timed out);
-// synchronous read, optionally clearing them.
-unsigned int gemv_error_flags(bool clear);
-
-// Integer per-16 subblock sums through the GEMV's decode/dot code.
-cudaError_t launch_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
-                                 const int8_t* q, int64_t M, int32_t* isum,
-                                 cudaStream_t stream);
+// Error flags raised by the kernels when a bounded pipeline wait times out,
+// read synchronously on the current device (optionally clearing them).
+cudaError_t gemv_error_flags(bool clear, unsigned int* flags);
+cudaError_t gemm_error_flags(bool clear, unsigned int* flags);
 
 // Prefill GEMM (tcgen05) and the size of its activation workspace.
 size_t gemm_workspace_size(int64_t M, int64_t N, int64_t K);
@@ -52,17 +52,34 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
 
 // The allocation-free GEMM: bytes of its library-owned scratch, and the
 // scratch's device address on the current device (looked up once per
-// device, on first use).
+// device and context, on first use).
 size_t gemm_noalloc_limit();
 cudaError_t gemm_noalloc_scratch(void** out);
-
-// Error flags raised by the GEMM kernel (bit 0: a pipeline wait timed out).
-unsigned int gemm_error_flags(bool clear);
 
 // Record the CUDA error reported by nvq_last_cuda_error() on this thread.
 void set_last_cuda_error(cudaError_t e);
 
 // Number of streaming multiprocessors of the current device (cached).
 int device_sm_count();
+
+// Sets a kernel's dynamic shared-memory limit once per device.  Safe when
+// several host threads make their first calls at the same time (the
+// attribute call is idempotent; the flag only skips repeats).
+struct SmemAttrOnce {
+  static constexpr int kMaxDevices = 64;
+  std::atomic<bool> done[kMaxDevices] = {};
+
+  template <typename Kernel>
+  cudaError_t ensure(Kernel kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool cacheable = dev >= 0 && dev < kMaxDevices;
+    if (cacheable && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && cacheable) done[dev].store(true, std::memory_order_release);
+    return e;
+  }
+};
 
 }  // namespace nvq

@@ -102,19 +102,14 @@ extern "C" nvq_status nvq_decoder_stack(const nvq_linear* linears, int64_t n_lay
   const bool decode = M <= 16;
 
   cudaError_t err = cudaSuccess;
-  // the fused quantise-in-GEMV repeats the quantisation in every CTA; at the
-  // widths of a dense decoder a separate (overlapped) quantiser is faster
-  const bool fused = false;
   auto quantize = [&](const float* in, int64_t K) {
-    if (err != cudaSuccess || (fused && nvq::quant_gemv_supported(K))) return;
+    if (err != cudaSuccess) return;
     err = nvq::launch_quantize_q8_0(in, M, K, qa, da, st);
     if (err == cudaSuccess && !decode) err = nvq::gemm_expand(qa, da, M, K, gws, st);
   };
-  auto dot = [&](const nvq_linear& W, const float* in, float* y) {
+  auto dot = [&](const nvq_linear& W, float* y) {
     if (err != cudaSuccess) return;
-    if (fused && nvq::quant_gemv_supported(W.K))
-      err = nvq::launch_quant_gemv(W.codes, W.scales, W.g, W.N, W.K, in, y, st);
-    else if (decode)
+    if (decode)
       err = nvq::launch_gemv(W.codes, W.scales, W.g, W.N, W.K, qa, da, M, y, st);
     else
       err = nvq::gemm_main(W.codes, W.scales, W.g, W.N, W.K, M, y, gws, st);
@@ -122,16 +117,16 @@ extern "C" nvq_status nvq_decoder_stack(const nvq_linear* linears, int64_t n_lay
   for (int64_t l = 0; l < n_layers && err == cudaSuccess; ++l) {
     const nvq_linear* L = linears + NVQ_STACK_LINEARS * l;
     quantize(x, L[kQ].K);
-    dot(L[kQ], x, outs[kQ]);
-    dot(L[kK], x, outs[kK]);
-    dot(L[kV], x, outs[kV]);
+    dot(L[kQ], outs[kQ]);
+    dot(L[kK], outs[kK]);
+    dot(L[kV], outs[kV]);
     quantize(outs[kV], L[kO].K);
-    dot(L[kO], outs[kV], outs[kO]);
+    dot(L[kO], outs[kO]);
     quantize(outs[kO], L[kUp].K);
-    dot(L[kUp], outs[kO], outs[kUp]);
-    dot(L[kGate], outs[kO], outs[kGate]);
+    dot(L[kUp], outs[kUp]);
+    dot(L[kGate], outs[kGate]);
     quantize(outs[kUp], L[kDown].K);
-    dot(L[kDown], outs[kUp], outs[kDown]);
+    dot(L[kDown], outs[kDown]);
   }
   if (err != cudaSuccess) {
     nvq::set_last_cuda_error(err);

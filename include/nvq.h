@@ -135,22 +135,6 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                     int64_t M, float* y, void* stream);
 
 /*
- * nvq_quant_gemv - decode GEMV of one fp32 token with its Q8_0 quantisation
- * fused in: y[1, N] = Q8_0(x)[1, K] . W[N, K]^T.
- *
- * x  device float [1, K] (finite).  The kernel quantises x exactly as
- * nvq_quantize_act_q8_0 does (same IEEE operations, so the codes and scales
- * are identical) and then runs the nvq_gemv product, so y is bit-identical
- * to nvq_quantize_act_q8_0 followed by nvq_gemv; it saves one launch and
- * one round trip of the activations.  Supported for K = 1024 * T with T in
- * {4, 5, 6, 8, 10, 12, 15, 16, 20, 25} (NVQ_ERR_BAD_SHAPE otherwise).
- * Errors: as nvq_gemv.
- */
-nvq_status nvq_quant_gemv(const uint8_t* codes, const uint8_t* scales, float g,
-                          int64_t N, int64_t K, const float* x, float* y,
-                          void* stream);
-
-/*
  * nvq_gemm_workspace_size - bytes of device workspace nvq_gemm needs for
  * M tokens of K features (0 when M == 0).  It holds the activations
  * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q.
@@ -200,7 +184,9 @@ nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
  * should use nvq_gemm with a caller workspace.
  * Set-up: the first call on a device looks up the scratch's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.
+ * before any stream capture.  The address is cached per device and context;
+ * a call made in another context (for example after cudaDeviceReset) looks
+ * it up again, so that call too must come before any capture.
  * Sharing: every call, on every stream and host thread, uses the same
  * array, so calls whose work overlaps on the GPU race and corrupt each
  * other's results; serialise them (one stream, or events).  The array keeps
@@ -213,15 +199,59 @@ nvq_status nvq_gemm_noalloc(const uint8_t* codes, const uint8_t* scales, float g
                             int64_t M, float* y, void* stream);
 
 /*
- * nvq_debug_subblock_sums - the integer per-16 subblock sums the GEMV forms,
- * exported for bit-exact checking:
- * isum[m, n, sb] = sum_{k in sb} (2*E2M1(code[n,k])) * q[m,k], int32
- * [M, N, K/16] (|isum| <= 16*12*127).  Uses the GEMV's own decode and dp4a
- * code.  Errors: as nvq_gemv (M = 1..16).
+ * nvq_debug_subblock_sums - nvq_gemv that also exports the integer per-16
+ * subblock sums it forms, for bit-exact checking ("HANDOFF: flint CPU
+ * optimization (Q4_1 + NVFP4)", section 3: the row dot forms one integer sum
+ * per 16-element subblock; "Bias trick": the decode path stores the codes
+ * +12-biased and removes the bias with -12*bsum16).
+ *
+ * Arguments as nvq_gemv, plus
+ * isum  device int32 [M, N, K/16]:
+ *       isum[m, n, sb] = sum_{k in sb} (2*E2M1(code[n,k])) * q[m,k]
+ *       (|isum| <= 16*12*127), 16-byte aligned.
+ * The call dispatches exactly as nvq_gemv does and runs the same schedule,
+ * decode (biased or signed LUT) and dp4a code, instantiated to also store
+ * the sums; y receives the same values nvq_gemv writes.
+ * Errors: as nvq_gemv; NVQ_ERR_INVALID_ARG / NVQ_ERR_MISALIGNED for isum.
  */
-nvq_status nvq_debug_subblock_sums(const uint8_t* codes, int64_t N, int64_t K,
-                                   const int8_t* q, int64_t M, int32_t* isum,
-                                   void* stream);
+nvq_status nvq_debug_subblock_sums(const uint8_t* codes, const uint8_t* scales, float g,
+                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                                   int64_t M, float* y, int32_t* isum, void* stream);
+
+/* Bits of nvq_error_flags. */
+#define NVQ_FLAG_GEMV_TIMEOUT 1u  /* a GEMV pipeline wait gave up (4 s)  */
+#define NVQ_FLAG_GEMM_TIMEOUT 2u  /* a GEMM pipeline wait gave up (4 s)  */
+
+/*
+ * nvq_error_flags - device-side error flags of the current device.
+ *
+ * Every pipeline wait inside the kernels (a consumer waiting for a copy, a
+ * producer for a free stage, the tensor-core issuer for its operands) is
+ * bounded: after 4 s without progress the kernel raises a flag, stops
+ * issuing, lets the copies it issued land, frees its tensor memory and
+ * returns instead of hanging.  The outputs of a call whose kernel timed out
+ * are not valid, and the call itself has already returned NVQ_OK (it only
+ * enqueued work), so callers that need the guarantee read the flags after
+ * synchronising the streams they used.
+ * flags  host uint32 out: NVQ_FLAG_* bits raised since the last clear.
+ * clear  nonzero: reset the flags after reading them.
+ * The read is synchronous (a device-to-host copy on the legacy stream).
+ * Errors: NVQ_ERR_INVALID_ARG (flags NULL), NVQ_ERR_UNSUPPORTED_DEVICE,
+ * NVQ_ERR_CUDA.
+ */
+nvq_status nvq_error_flags(unsigned int* flags, int clear);
+
+/*
+ * nvq_debug_stalled_wait - test-only: run one pipeline wait that can never
+ * complete (a stage whose copy is never issued), through the same bounded
+ * wait as the GEMV kernels, with a limit of limit_ns (1 us .. 1 s).  The
+ * kernel gives up after the limit, raises NVQ_FLAG_GEMV_TIMEOUT and returns.
+ * result  device int32 [2] (16-byte aligned): result[0] = 1 if the wait
+ *         completed (it cannot), result[1] = microseconds spent waiting.
+ * Errors: NVQ_ERR_INVALID_ARG (NULL, limit out of range),
+ * NVQ_ERR_MISALIGNED, NVQ_ERR_UNSUPPORTED_DEVICE, NVQ_ERR_CUDA.
+ */
+nvq_status nvq_debug_stalled_wait(uint64_t limit_ns, int* result, void* stream);
 
 /* One NVFP4 weight matrix W[N, K] in device memory (caller-owned). */
 typedef struct nvq_linear {

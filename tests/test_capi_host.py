@@ -85,8 +85,20 @@ def test_host_validation_status_codes():
     assert lib.nvq_gemm_workspace_size(0, 8, 64) == 0
 
     sums = lib.nvq_debug_subblock_sums
-    assert sums(codes, 8, 64, q, 17, y, None) == capi.NVQ_ERR_BAD_SHAPE
-    assert sums(codes, 8, 32, q, 1, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    isum = p()
+    assert sums(codes, scales, 1.0, 8, 64, q, d, 17, y, isum, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert sums(codes, scales, 1.0, 8, 32, q, d, 1, y, isum, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert sums(codes, scales, 1.0, 8, 64, q, d, 1, y, None, None) == capi.NVQ_ERR_INVALID_ARG
+    assert sums(codes, scales, 1.0, 8, 64, q, d, 1, y, p(off=4), None) == capi.NVQ_ERR_MISALIGNED
+    assert sums(None, None, 1.0, 8, 64, None, None, 0, None, None, None) == capi.NVQ_OK
+
+    flags = lib.nvq_error_flags
+    assert flags(None, 0) == capi.NVQ_ERR_INVALID_ARG
+    stalled = lib.nvq_debug_stalled_wait
+    assert stalled(10, p(), None) == capi.NVQ_ERR_INVALID_ARG
+    assert stalled(2 * 10**9, p(), None) == capi.NVQ_ERR_INVALID_ARG
+    assert stalled(10**6, None, None) == capi.NVQ_ERR_INVALID_ARG
+    assert stalled(10**6, p(off=4), None) == capi.NVQ_ERR_MISALIGNED
 
 
 def test_pack_rejects_bad_arguments():
