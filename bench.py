@@ -2,19 +2,21 @@
 """Benchmark of the NVFP4 x Q8_0 kernels on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl nvq|reference]
+                    [--impl nvq|reference] [--no-sub]
 
 Prints ONE JSON line on rank 0.
 
-Workloads (``--workload``):
-  decode_sweep (default)  one step quantises one token's activations (Q8_0)
+Workloads (``--workload``; the line's headline is this one, default
+``decode_sweep``, and unless ``--no-sub`` the line also carries every other
+workload under ``"workloads"``, each measured the same way):
+  decode_sweep            one step quantises one token's activations (Q8_0)
                           and runs the decode GEMV for each of the four
                           linear shapes of a 27B-class dense decoder,
                           (K, N) = (5120, 5120), (5120, 25600), (25600, 5120),
                           (5120, 152064).  Metric: weight GB/s (NVFP4 weight
                           bytes N*K*0.5625 streamed per second).
   gemv_4096               M=1, K=N=4096.
-  small_batch_m{2,4,8,16} decode GEMV at M tokens, (5120, 25600), (25600, 5120).
+  small_batch_m{2,4,8,16} M tokens, (5120, 25600), (25600, 5120).
   prefill_m{256,2048}     Q8_0 + tcgen05 GEMM over (5120, 5120), (5120, 25600),
                           (25600, 5120).  Metric: algorithmic TFLOP/s 2*M*N*K.
   stack_decode            all 448 linears of a 64-layer dense decoder (17.9 GB
@@ -23,30 +25,44 @@ Workloads (``--workload``):
   stack_prefill           the same stack for 2048 tokens.
 
 Timing: W untimed eager warm-up steps; the K timed steps are captured once
-into a CUDA graph (the public entry points are graph-capturable: they only
-enqueue work) and replayed inside the timed region, bracketed by a barrier
-and a device synchronize and timed with CUDA events on the launching stream;
-the time is the max over ranks.  The dominant kernel of every step is
-bracketed by its own (graph-recorded) events for the roofline entry.  One
-step's weights exceed the 126 MB L2 in every workload (600 MB for the decode
-sweep), so no L2 flush is inserted.  ``e2e`` runs the same K steps through
-the public Python API eagerly, with each step's activations copied from
-pinned host memory and its outputs copied back inside the timed region (the
-weights are resident model parameters).
+into a CUDA graph (the public entry points only enqueue work) and replayed
+inside the timed region, bracketed by a barrier and a device synchronize and
+timed with CUDA events on the launching stream; the time is the max over
+ranks.  One step's inputs exceed the 126 MB L2 in every workload (600 MB of
+weights for the decode sweep), so no L2 flush is inserted.
+
+Roofline of the dominant kernel (``roofline``): for the GEMV and GEMM
+workloads each shape's dominant launch (nvq_gemv; nvq_gemm) is timed alone in
+its own event-free CUDA graph of back-to-back launches that rotate through
+enough copies of the weights (at least 4x the L2 size) that no launch finds
+its weights in L2; achieved = algorithmic bytes (or flops) of one launch of
+every shape / the sum of their launch times, with the per-shape rates
+listed.  ``step_achieved`` divides the same amount by the whole step (which
+also holds the quantiser launches).  For the stack the unit is the whole
+pass (its launches are the step).
+
+``e2e`` runs the same K steps through the public Python API eagerly, with each
+step's activations copied from pinned host memory and its outputs copied back
+inside the timed region (the weights are resident model parameters).
+
+``cpu_baseline`` times the plain CPU oracle on a bounded sample of the same
+workload: on one host core, and (``all_cores``) spread over every core of the
+host in a pool of spawned worker processes, one numpy thread each.
 
 Multi-GPU (``torchrun --nproc-per-node N``): every rank runs the same
 workload on its own GPU with no data exchange (independent replicas; the
 only collectives are the timing barrier and max).  ``value`` is the units of
 all ranks divided by the max time; ``scaling`` is "weak".
 
-``--impl reference`` times the plain CPU oracle on the host (rank 0 only),
-each step a bounded sample of the same workload, on the same metric.
+``--impl reference`` times the plain CPU oracle on the host cores (rank 0
+only), each step a bounded sample of the same workload, on the same metric.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -64,6 +80,10 @@ if ROOT not in sys.path:
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 WEIGHT_BYTES_PER_ELEMENT = 0.5625       # 4-bit code + one UE4M3 byte per 16
+L2_BYTES = 126e6
+SUB_WORKLOADS = ["gemv_4096", "small_batch_m2", "small_batch_m4", "small_batch_m8",
+                 "small_batch_m16", "prefill_m256", "prefill_m2048", "stack_decode",
+                 "stack_prefill"]
 
 
 # ---------------------------------------------------------------------------
@@ -172,7 +192,9 @@ class ClockSampler:
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
         window = "timed region"
         if not inside:
-            inside, window = self.samples, "whole run (timed region shorter than one sample)"
+            # the timed region was shorter than one sample: the nearest ones
+            near = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            inside, window = near, "nearest samples (timed region shorter than one sample)"
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         reasons = sorted({r for s in inside for r in s[4]})
@@ -205,31 +227,124 @@ def profiled_traffic(kernel: str, workload: str, src_hash: str):
     return float(m_bytes.group(1))
 
 
-class EventLog:
-    """Start/stop events around the dominant kernel of each step; created
-    external so that they become timestamp nodes when captured in a graph."""
+def replay_ms(graph, stream) -> float:
+    """Device time of one replay of a captured graph (CUDA events on the
+    launching stream, synchronised on both sides)."""
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    graph.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+def l2_copies(nbytes: float) -> int:
+    """Weight copies to rotate through so that a launch never finds its
+    weights in L2 (at least 4x L2 in total, at least 2)."""
+    return max(2, math.ceil(4 * L2_BYTES / max(nbytes, 1.0)))
+
+
+# ---------------------------------------------------------------------------
+# oracle tasks (CPU baseline): quantise a row sample's activations and take
+# the fp64 dequantise-then-dot of a block of weight rows
+# ---------------------------------------------------------------------------
+
+def oracle_task(task):
+    """Run one oracle task, (codes, scales, g, x, reps, units) -> units: the
+    oracle's Q8_0 quantisation of x, then its fp64 dequantise-then-dot of the
+    weight block, `reps` times."""
+    import oracle as o
+    codes, scales, g, x, reps, units = task
+    q, d = o.quantize_q8_0(x)
+    for _ in range(reps):
+        o.dot_fp64(codes, scales, g, q, d)
+    return units
+
+
+def _pool_init():
+    import oracle  # noqa: F401  (imported once per worker, outside the timing)
+
+
+def _noop(_):
+    return 0
+
+
+def split_tasks(tasks, parts: int):
+    """Split every task's repetitions into about `parts` tasks (units in
+    proportion)."""
+    out = []
+    for codes, scales, g, x, reps, units in tasks:
+        k = max(1, min(parts, reps))
+        bounds = np.linspace(0, reps, k + 1).astype(int)
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            if b > a:
+                out.append((codes, scales, g, x, int(b - a), units * (b - a) / reps))
+    return out
+
+
+class OraclePool:
+    """Worker processes (spawned, one numpy thread each) over all host cores."""
 
     def __init__(self):
-        self.pairs = []
-        self._open = None
+        import concurrent.futures as cf
+        import multiprocessing as mp
+        try:
+            self.cores = len(os.sched_getaffinity(0))
+        except AttributeError:
+            self.cores = os.cpu_count() or 1
+        self.cores = max(1, min(self.cores, 128))
+        saved = {k: os.environ.get(k) for k in
+                 ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        try:
+            self.ex = cf.ProcessPoolExecutor(self.cores, mp_context=mp.get_context("spawn"),
+                                             initializer=_pool_init)
+            list(self.ex.map(_noop, range(self.cores * 2)))   # start every worker
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
 
-    def begin(self, stream):
-        import torch
-        ev = torch.cuda.Event(enable_timing=True, external=True)
-        ev.record(stream)
-        self._open = ev
+    def run(self, tasks) -> float:
+        parts = split_tasks(tasks, self.cores)
+        return float(sum(self.ex.map(oracle_task, parts)))
 
-    def end(self, stream, amount):
-        import torch
-        ev = torch.cuda.Event(enable_timing=True, external=True)
-        ev.record(stream)
-        self.pairs.append((self._open, ev, amount))
-        self._open = None
+    def close(self):
+        self.ex.shutdown(wait=True, cancel_futures=True)
 
-    def totals(self):
-        ms = sum(a.elapsed_time(b) for a, b, _ in self.pairs)
-        amount = sum(x for _, _, x in self.pairs)
-        return ms, amount, len(self.pairs)
+
+def run_tasks_serial(tasks) -> float:
+    return float(sum(oracle_task(t) for t in tasks))
+
+
+# The oracle packs a small base block of each matrix's rows once (its packer
+# is far slower than its dot product); a sample of any size runs the oracle's
+# dot over that block repeatedly.  The dot costs the same whatever the values.
+ORACLE_BASE_ROWS = 64
+_ORACLE_BASE = {}
+
+
+def oracle_base(key, make):
+    """(codes, scales, g, x) of a base block, packed by the oracle, cached."""
+    if key not in _ORACLE_BASE:
+        import oracle as o
+        W, x = make()
+        codes, scales, g = o.pack_nvfp4(W)
+        _ORACLE_BASE[key] = (codes, scales, g, x)
+    return _ORACLE_BASE[key]
+
+
+def sample_task(base, rows: int, units_per_row: float):
+    """A task that runs the oracle over `rows` weight rows as repetitions of
+    the base block (rows rounded up to whole blocks)."""
+    codes, scales, g, x = base
+    reps = max(1, -(-rows // codes.shape[0]))
+    return (codes, scales, g, x, reps, units_per_row * reps * codes.shape[0])
 
 
 # ---------------------------------------------------------------------------
@@ -246,8 +361,9 @@ class GemvWorkload:
     metric = "nvfp4_q8_0_gemv_weight_GBps"
     unit = "GB/s"
 
-    def __init__(self, name, shapes, M, make_case):
-        self.name, self.shapes, self.M, self.make_case = name, shapes, M, make_case
+    def __init__(self, name, shapes, M, make_case, oracle_rows):
+        self.name, self.shapes, self.M = name, shapes, M
+        self.make_case, self.oracle_rows = make_case, oracle_rows
 
     def setup(self, device):
         import torch
@@ -270,11 +386,10 @@ class GemvWorkload:
             self.cases.append(c)
 
     def config(self):
-        act = "fp32 -> Q8_0 on the GPU every step (nvq_quantize_act_q8_0)"
         return {"workload": self.name, "M": self.M,
                 "shapes_KN": [list(s) for s in self.shapes],
                 "weights": "NVFP4 (E2M1 + UE4M3 per 16 + fp32 g), N(0,0.02^2)",
-                "activations": act,
+                "activations": "fp32 -> Q8_0 on the GPU every step (nvq_quantize_act_q8_0)",
                 "l2": "inputs larger than L2 (weights of one step %.0f MB > 126 MB)"
                       % (self.weight_bytes() / 1e6),
                 "parallelism": "replicas"}
@@ -285,27 +400,25 @@ class GemvWorkload:
     def units_per_step(self):
         return self.weight_bytes() / 1e9          # GB
 
-    def kernel_amount(self, c):
-        """Algorithmic bytes of one GEMV launch: NVFP4 weights, the
-        activations (fp32 when quantised inside the kernel, else Q8_0) and
-        the fp32 output."""
-        M, K, N = self.M, c["K"], c["N"]
+    def kernel_amount(self, K, N):
+        """Algorithmic bytes of one GEMV launch: NVFP4 weights, the Q8_0
+        activations and the fp32 output."""
+        M = self.M
         return N * K * WEIGHT_BYTES_PER_ELEMENT + M * K * (1 + 2 / 32) + 4 * M * N
 
     def launches_per_step(self):
         return 2 * len(self.cases)
 
-    def step(self, stream, log=None, e2e=False):
+    def dominant(self, c, codes, scales, stream):
+        self.capi.gemv(codes, scales, c["g"], c["q"], c["d"], c["y"], stream=stream)
+
+    def step(self, stream, e2e=False):
         capi = self.capi
         for c in self.cases:
             if e2e:
                 c["x"].copy_(c["x_host"], non_blocking=True)
             capi.quantize_act_q8_0(c["x"], c["q"], c["d"], stream=stream)
-            if log is not None:
-                log.begin(stream)
-            capi.gemv(c["codes"], c["scales"], c["g"], c["q"], c["d"], c["y"], stream=stream)
-            if log is not None:
-                log.end(stream, self.kernel_amount(c))
+            self.dominant(c, c["codes"], c["scales"], stream)
             if e2e:
                 c["y_host"].copy_(c["y"], non_blocking=True)
 
@@ -313,34 +426,49 @@ class GemvWorkload:
         return (sum(c["x"].numel() * 4 for c in self.cases),
                 sum(c["y"].numel() * 4 for c in self.cases))
 
+    def shape_timings(self, stream, reps):
+        """Per shape: the dominant launch alone, back to back in an event-free
+        graph, rotating through weight copies that defeat L2."""
+        import torch
+        out = []
+        for c in self.cases:
+            K, N = c["K"], c["N"]
+            ncopy = l2_copies(N * K * WEIGHT_BYTES_PER_ELEMENT)
+            copies = [(c["codes"], c["scales"])] + [
+                (c["codes"].clone(), c["scales"].clone()) for _ in range(ncopy - 1)]
+            for cc, ss in copies[:2]:
+                self.dominant(c, cc, ss, stream)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                s = torch.cuda.current_stream()
+                for i in range(reps):
+                    cc, ss = copies[i % ncopy]
+                    self.dominant(c, cc, ss, s)
+            graph.replay()
+            ms = replay_ms(graph, stream)
+            del graph, copies
+            torch.cuda.empty_cache()
+            out.append({"K": K, "N": N, "us_per_launch": ms * 1e3 / reps,
+                        "amount": self.kernel_amount(K, N), "weight_copies": ncopy})
+        return out
+
     # --- CPU oracle sample ---------------------------------------------------
-    def oracle_prepare(self, size):
-        import oracle as o
-        self.o = o
-        self.samples = []
+    def oracle_tasks(self, rows):
+        tasks = []
         for K, N in self.shapes:
-            W, x = self.make_case(K, N)
-            g = o.nvfp4_tensor_scale(W)
-            r = min(size, N)
-            codes, scales, _ = o.pack_nvfp4(W[:r], g=g)
-            del W
-            self.samples.append((K, r, codes, scales, g, x))
+            base = oracle_base(("gemv", self.name, K, N),
+                               lambda: self.oracle_rows(K, N, ORACLE_BASE_ROWS))
+            tasks.append(sample_task(base, rows, K * WEIGHT_BYTES_PER_ELEMENT / 1e9))
+        return tasks
 
-    def oracle_step(self):
-        o = self.o
-        gb = 0.0
-        for K, r, codes, scales, g, x in self.samples:
-            q, d = o.quantize_q8_0(x)
-            o.dot_fp64(codes, scales, g, q, d)
-            gb += r * K * WEIGHT_BYTES_PER_ELEMENT / 1e9
-        return gb
-
-    def oracle_sample_desc(self, size):
-        return (f"first {size} rows of each of the {len(self.shapes)} shapes, M={self.M}: "
-                "oracle Q8_0 quantisation + fp64 dequantise-then-dot")
+    def oracle_sample_desc(self, rows):
+        return (f"{rows} weight rows of each of the {len(self.shapes)} shapes (the first "
+                f"{ORACLE_BASE_ROWS} rows, oracle-packed, run repeatedly), M={self.M}: oracle Q8_0 "
+                "quantisation + fp64 dequantise-then-dot")
 
 
-class GemmWorkload:
+class GemmWorkload(GemvWorkload):
     """Prefill: Q8_0 of M tokens and the tcgen05 GEMM for each shape."""
 
     kernel = "gemm"
@@ -350,30 +478,15 @@ class GemmWorkload:
     unit = "TFLOP/s"
 
     def __init__(self, name, shapes, M):
-        self.name, self.shapes, self.M = name, shapes, M
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        super().__init__(name, shapes, M, lambda K, N: wl.prefill_case(M, K, N), None)
 
     def setup(self, device):
         import torch
-        from bit_weight_quantized_nvq_b200 import capi, workloads as wl
-        self.capi = capi
-        self.cases = []
-        M = self.M
-        for K, N in self.shapes:
-            W, x = wl.prefill_case(M, K, N)
-            codes, scales, g = capi.pack_nvfp4(W)
-            del W
-            c = {"K": K, "N": N, "g": g,
-                 "codes": torch.from_numpy(codes).to(device),
-                 "scales": torch.from_numpy(scales).to(device),
-                 "x": torch.from_numpy(x).to(device),
-                 "x_host": torch.from_numpy(x).pin_memory(),
-                 "q": torch.empty((M, K), dtype=torch.int8, device=device),
-                 "d": torch.empty((M, K // 32), dtype=torch.float16, device=device),
-                 "y": torch.empty((M, N), dtype=torch.float32, device=device),
-                 "ws": torch.empty(capi.gemm_workspace_size(M, N, K), dtype=torch.uint8,
-                                   device=device)}
-            c["y_host"] = torch.empty((M, N), dtype=torch.float32).pin_memory()
-            self.cases.append(c)
+        super().setup(device)
+        for c in self.cases:
+            c["ws"] = torch.empty(self.capi.gemm_workspace_size(self.M, c["N"], c["K"]),
+                                  dtype=torch.uint8, device=device)
 
     def config(self):
         return {"workload": self.name, "M": self.M,
@@ -383,64 +496,36 @@ class GemmWorkload:
                 "l2": "inputs larger than L2 (activations and weights of one step > 126 MB)",
                 "parallelism": "replicas"}
 
-    def flops(self, c):
-        return 2.0 * self.M * c["N"] * c["K"]
-
     def units_per_step(self):
         return sum(2.0 * self.M * N * K for K, N in self.shapes) / 1e12   # TFLOP
 
-    def kernel_amount(self, c):
-        return self.flops(c)
+    def kernel_amount(self, K, N):
+        return 2.0 * self.M * N * K
 
     def launches_per_step(self):
         return 3 * len(self.cases)       # quantise, expand, tcgen05 GEMM
 
-    def step(self, stream, log=None, e2e=False):
-        capi = self.capi
-        for c in self.cases:
-            if e2e:
-                c["x"].copy_(c["x_host"], non_blocking=True)
-            capi.quantize_act_q8_0(c["x"], c["q"], c["d"], stream=stream)
-            if log is not None:
-                log.begin(stream)
-            capi.gemm(c["codes"], c["scales"], c["g"], c["q"], c["d"], c["y"], c["ws"],
-                      stream=stream)
-            if log is not None:
-                log.end(stream, self.kernel_amount(c))
-            if e2e:
-                c["y_host"].copy_(c["y"], non_blocking=True)
+    def dominant(self, c, codes, scales, stream):
+        self.capi.gemm(codes, scales, c["g"], c["q"], c["d"], c["y"], c["ws"], stream=stream)
 
-    def e2e_bytes(self):
-        return (sum(c["x"].numel() * 4 for c in self.cases),
-                sum(c["y"].numel() * 4 for c in self.cases))
-
-    def oracle_prepare(self, size):
-        import oracle as o
+    def oracle_tasks(self, rows):
         from bit_weight_quantized_nvq_b200 import workloads as wl
-        self.o = o
-        self.samples = []
-        toks = max(1, min(self.M, size // 64))
+        toks = max(1, min(self.M, 16))
+        tasks = []
         for K, N in self.shapes:
-            W, x = wl.prefill_case(self.M, K, N)
-            g = o.nvfp4_tensor_scale(W)
-            r = min(size, N)
-            codes, scales, _ = o.pack_nvfp4(W[:r], g=g)
-            del W
-            self.samples.append((K, r, codes, scales, g, x[:toks]))
+            base = oracle_base(
+                ("gemm", self.name, K, N),
+                lambda: (wl.weight_rows("prefill", "W", N, K, ORACLE_BASE_ROWS),
+                         wl.activations("prefill", "x", self.M, K, "normal",
+                                        outliers=True)[:toks]))
+            tasks.append(sample_task(base, rows, 2.0 * toks * K / 1e12))
+        return tasks
 
-    def oracle_step(self):
-        o = self.o
-        tf = 0.0
-        for K, r, codes, scales, g, x in self.samples:
-            q, d = o.quantize_q8_0(x)
-            o.dot_fp64(codes, scales, g, q, d)
-            tf += 2.0 * x.shape[0] * r * K / 1e12
-        return tf
-
-    def oracle_sample_desc(self, size):
-        toks = max(1, min(self.M, size // 64))
-        return (f"{toks} tokens x first {size} rows of each of the {len(self.shapes)} shapes: "
-                "oracle Q8_0 + fp64 dequantise-then-dot")
+    def oracle_sample_desc(self, rows):
+        toks = max(1, min(self.M, 16))
+        return (f"{toks} tokens x {rows} weight rows of each of the {len(self.shapes)} shapes "
+                f"(the first {ORACLE_BASE_ROWS} rows, oracle-packed, run repeatedly): oracle Q8_0 + "
+                "fp64 dequantise-then-dot")
 
 
 class StackWorkload:
@@ -462,15 +547,15 @@ class StackWorkload:
         import torch
         from bit_weight_quantized_nvq_b200 import capi, workloads as wl
         self.capi = capi
-        self.layer_host = []
+        layer_host = []
         for name, W in wl.stack_layer_weights():
             codes, scales, g = capi.pack_nvfp4(W)
-            self.layer_host.append((codes, scales, g))
+            layer_host.append((codes, scales, g))
             del W
         layers = []
         for _ in range(wl.STACK_LAYERS):
             layers.append([(torch.from_numpy(c).to(device), torch.from_numpy(s).to(device), g)
-                           for c, s, g in self.layer_host])
+                           for c, s, g in layer_host])
         self.stack = capi.DecoderStack(layers, self.M, device=device)
         x = wl.stack_input(self.M)
         self.x = torch.from_numpy(x).to(device)
@@ -495,70 +580,62 @@ class StackWorkload:
     def units_per_step(self):
         return float(self.M)                        # tokens
 
-    def kernel_amount(self, _=None):
-        return self.weight_bytes() if self.bound == "hbm" else self.flops()
-
     def launches_per_step(self):
         per_layer = 4 + 7 + (4 if self.M > 16 else 0)
         return per_layer * self.n_layers
 
-    def step(self, stream, log=None, e2e=False):
+    def step(self, stream, e2e=False):
         if e2e:
             self.x.copy_(self.x_host, non_blocking=True)
-        if log is not None:
-            log.begin(stream)
         self.stack.forward(self.x, stream=stream)
-        if log is not None:
-            log.end(stream, self.kernel_amount())
         if e2e:
             self.y_host.copy_(self.stack.outs[6], non_blocking=True)
 
     def e2e_bytes(self):
         return self.x.numel() * 4, self.stack.outs[6].numel() * 4
 
-    def oracle_prepare(self, size):
-        import oracle as o
-        from bit_weight_quantized_nvq_b200 import workloads as wl
-        self.o = o
-        self.samples = []
-        toks = max(1, min(self.M, size // 256))
-        for name, W in wl.stack_layer_weights():
-            g = o.nvfp4_tensor_scale(W)
-            r = min(size, W.shape[0])
-            codes, scales, _ = o.pack_nvfp4(W[:r], g=g)
-            self.samples.append((W.shape[1], W.shape[0], r, codes, scales, g))
-        self.x_s = wl.stack_input(self.M)[:toks]
+    def shape_timings(self, stream, reps):
+        return None
 
-    def oracle_step(self):
-        """One layer's 7 products on a row sample; returns tokens of the
+    def oracle_tasks(self, rows):
+        """One layer's 7 products on a row sample; units = tokens of the
         64-layer pass that this much work is worth (row fraction x layers)."""
-        o = self.o
-        frac = 0.0
-        rng = np.random.default_rng(0)
-        for K, N, r, codes, scales, g in self.samples:
-            x = rng.standard_normal((self.x_s.shape[0], K)).astype(np.float32)
-            q, d = o.quantize_q8_0(x)
-            o.dot_fp64(codes, scales, g, q, d)
-            frac += r * K / sum(KK * NN for _, KK, NN in self.linears)
-        return self.x_s.shape[0] * frac / self.n_layers
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        toks = max(1, min(self.M, 4))
+        total = sum(K * N for _, K, N in self.linears)
+        tasks = []
+        for i, (name, K, N) in enumerate(self.linears):
+            def make(name=name, K=K, N=N, i=i):
+                rng = np.random.default_rng(i)
+                return (wl.weight_rows("stack", name, N, K, ORACLE_BASE_ROWS),
+                        rng.standard_normal((toks, K)).astype(np.float32))
+            base = oracle_base(("stack", self.name, K, N, name), make)
+            tasks.append(sample_task(base, rows, toks * (K / total) / self.n_layers))
+        return tasks
 
-    def oracle_sample_desc(self, size):
-        toks = max(1, min(self.M, size // 256))
-        return (f"{toks} token(s) x first {size} rows of each of the 7 linears of one layer "
-                "(random activations), scaled to the 64-layer pass by the fraction of weights "
-                "processed")
+    def oracle_sample_desc(self, rows):
+        toks = max(1, min(self.M, 4))
+        return (f"{toks} token(s) x {rows} weight rows of each of the 7 linears of one layer "
+                f"(the first {ORACLE_BASE_ROWS} rows, oracle-packed, run repeatedly; random "
+                "activations), scaled to the 64-layer pass by the fraction of weights processed")
 
 
 def make_workload(name: str):
     from bit_weight_quantized_nvq_b200 import workloads as wl
     if name == "decode_sweep":
-        return GemvWorkload(name, wl.DECODE_SHAPES, 1, lambda K, N: wl.decode_case(K, N))
+        return GemvWorkload(name, wl.DECODE_SHAPES, 1, lambda K, N: wl.decode_case(K, N),
+                            lambda K, N, r: (wl.weight_rows("decode_sweep", "W", N, K, r, True),
+                                             wl.activations("decode_sweep", "x", 1, K)))
     if name == "gemv_4096":
-        return GemvWorkload(name, [(4096, 4096)], 1, lambda K, N: wl.gemv_4096_case())
+        return GemvWorkload(name, [(4096, 4096)], 1, lambda K, N: wl.gemv_4096_case(),
+                            lambda K, N, r: (wl.weight_rows("gemv_4096", "W", N, K, r),
+                                             wl.activations("gemv_4096", "x", 1, K)))
     if name.startswith("small_batch_m"):
         M = int(name[len("small_batch_m"):])
-        return GemvWorkload(name, wl.SMALL_BATCH_SHAPES, M,
-                            lambda K, N: wl.small_batch_case(M, K, N))
+        return GemvWorkload(
+            name, wl.SMALL_BATCH_SHAPES, M, lambda K, N: wl.small_batch_case(M, K, N),
+            lambda K, N, r: (wl.weight_rows("small_batch", "W", N, K, r, True),
+                             wl.activations("small_batch", "x", M, K, "student_t4")))
     if name.startswith("prefill_m"):
         return GemmWorkload(name, wl.PREFILL_SHAPES, int(name[len("prefill_m"):]))
     if name == "stack_decode":
@@ -569,96 +646,81 @@ def make_workload(name: str):
 
 
 # ---------------------------------------------------------------------------
-# timing
+# measurement
 # ---------------------------------------------------------------------------
 
-def capture_steps(wk, steps: int, stream, events: bool):
-    """A CUDA graph of `steps` steps, optionally with an event pair around
-    the dominant kernel of every step."""
-    import torch
-    log = EventLog() if events else None
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        s = torch.cuda.current_stream()
-        for _ in range(steps):
-            wk.step(s, log)
-    return graph, log
-
-
-def roofline_entry(wk, log, peaks):
-    """The dominant kernel's achieved rate.  Its launch durations come from a
-    replay whose graph has an event pair around every such launch; an event
-    record node adds a little latency to the launch it brackets, so this is
-    a conservative figure.  `step_achieved` divides the same algorithmic
-    amount by the event-free step time instead (it also charges the other
-    kernels of the step to the dominant one: a lower bound too)."""
-    kernel_ms, amount, n = log.totals()
-    src_hash = source_hash(*wk.sources)
-    traffic = profiled_traffic(wk.kernel, wk.name, src_hash)
+def roofline_entry(wk, shapes, ms_per_step, peaks):
+    """The dominant kernel's achieved rate against the measured peak."""
     if wk.bound == "hbm":
-        achieved = amount / (kernel_ms / 1e3) / 1e9
-        peak, unit, src = peaks["hbm_gbs"], "GB/s", "hbm_gbs (copy)"
+        scale, peak, unit, src = 1e9, peaks["hbm_gbs"], "GB/s", "hbm_gbs (copy)"
     else:
-        achieved = amount / (kernel_ms / 1e3) / 1e12
-        peak, unit, src = peaks["bf16_tflops"], "TFLOP/s", "bf16_tflops (burst; fp16 runs at the bf16 rate)"
+        scale, peak, unit, src = 1e12, peaks["bf16_tflops"], "TFLOP/s", \
+            "bf16_tflops (burst; fp16 runs at the bf16 rate)"
+    if shapes:
+        amount = sum(s["amount"] for s in shapes)
+        us = sum(s["us_per_launch"] for s in shapes)
+        per_shape = [{"K": s["K"], "N": s["N"], "us": round(s["us_per_launch"], 3),
+                      "achieved": round(s["amount"] / (s["us_per_launch"] / 1e6) / scale, 2),
+                      "frac": round(s["amount"] / (s["us_per_launch"] / 1e6) / scale / peak, 4),
+                      "weight_copies": s["weight_copies"]} for s in shapes]
+        timing = ("each shape's dominant launch alone, back to back in an event-free CUDA "
+                  "graph rotating through weight copies (>= 4x L2); sum of launch times "
+                  f"{us:.2f} us per step vs the step's {ms_per_step * 1e3:.2f} us")
+        launches = len(shapes)
+        traffic = profiled_traffic(wk.kernel, wk.name, source_hash(*wk.sources))
+    else:
+        amount = wk.weight_bytes() if wk.bound == "hbm" else wk.flops()
+        us = ms_per_step * 1e3
+        per_shape = None
+        timing = "one pass of the whole stack (the step) per unit"
+        launches = 1
+        traffic = None
+    achieved = amount / (us / 1e6) / scale
     entry = {"bound": wk.bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-             "frac": round(achieved / peak, 4), "traffic": traffic,
-             "kernel": wk.kernel, "launches": n,
-             "avg_launch_us": round(kernel_ms * 1e3 / max(1, n), 3),
-             "algorithmic_per_launch": amount / max(1, n),
-             "peak_source": f"{peaks['source']} MEASURED_PEAKS.json {src}"}
+             "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": wk.kernel,
+             "launches_per_step": launches, "avg_launch_us": round(us / launches, 3),
+             "algorithmic_per_launch": amount / launches,
+             "peak_source": f"{peaks['source']} MEASURED_PEAKS.json {src}",
+             "step_achieved": round(amount / (ms_per_step / 1e3) / scale, 2),
+             "step_frac": round(amount / (ms_per_step / 1e3) / scale / peak, 4),
+             "timing": timing}
+    if per_shape is not None:
+        entry["per_shape"] = per_shape
     if wk.bound == "tensor" and wk.kernel == "gemm":
         entry["issued_frac"] = round(2 * achieved / peak, 4)   # hi and lo halves
-    entry["timing"] = ("launch durations from a second replay of the same steps with an "
-                       "event pair around every dominant-kernel launch")
     return entry
 
 
-def run_nvq(args, dist: Dist):
+def measure(wk, args, dist: Dist, peaks, device, sampler):
+    """Set up one workload, time its K steps, its dominant kernel per shape
+    and its e2e path; returns the entry (times are maxima over ranks)."""
     import torch
-    torch.cuda.set_device(dist.local_rank)
-    device = torch.device("cuda", dist.local_rank)
-    dist.init("nccl")
-    peaks = load_peaks()
-    wk = make_workload(args.workload)
     wk.setup(device)
-    # graphs are captured on a side stream; everything runs on it
-    stream = torch.cuda.Stream(device)
-    torch.cuda.set_stream(stream)
-
+    stream = torch.cuda.current_stream(device)
     for _ in range(args.warmup):
         wk.step(stream)
     torch.cuda.synchronize()
-    graph, _ = capture_steps(wk, args.steps, stream, events=False)
-    graph_ev, log = capture_steps(wk, args.steps, stream, events=True)
-    graph.replay()                        # untimed replays (graph upload)
-    graph_ev.replay()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        s = torch.cuda.current_stream()
+        for _ in range(args.steps):
+            wk.step(s)
+    graph.replay()                        # untimed replay (graph upload)
     torch.cuda.synchronize()
-
-    sampler = ClockSampler(dist.local_rank)
-    sampler.start()
-    time.sleep(0.35)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
-    torch.cuda.synchronize()
     t_wall0 = time.time()
-    start.record(stream)
-    graph.replay()
-    end.record(stream)
-    torch.cuda.synchronize()
+    ms = replay_ms(graph, stream)
     t_wall1 = time.time()
     dist.barrier()
-    ms = start.elapsed_time(end)
-    graph_ev.replay()                     # the dominant kernel's launch durations
-    torch.cuda.synchronize()
-    t_wall2 = time.time()
-    roofline = roofline_entry(wk, log, peaks)
-    roofline["step_achieved"] = round(
-        log.totals()[1] / (ms / 1e3) / (1e9 if wk.bound == "hbm" else 1e12), 2)
-    time.sleep(0.25)
-    sampler.stop()
-    clocks = sampler.summary(t_wall0 - 0.1, t_wall2 + 0.1)
-    del graph, graph_ev
+    clocks = sampler.summary(t_wall0 - 0.05, t_wall1 + 0.05)
+    del graph
+    shapes = wk.shape_timings(stream, max(args.steps, 20))
+    ms_max = dist.max(ms, device)
+    ms_per_step = ms_max / args.steps
+    if shapes:
+        for s in shapes:
+            s["us_per_launch"] = dist.max(s["us_per_launch"], device)
+    roofline = roofline_entry(wk, shapes, ms_per_step, peaks)
 
     # e2e: the same K steps through the public API, eagerly, with copies
     for _ in range(max(1, args.warmup // 2)):
@@ -672,126 +734,146 @@ def run_nvq(args, dist: Dist):
     e_end.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
-    e2e_ms = e_start.elapsed_time(e_end)
+    e2e_ms = dist.max(e_start.elapsed_time(e_end), device)
 
-    ms_max = dist.max(ms, device)
-    e2e_ms_max = dist.max(e2e_ms, device)
     units = wk.units_per_step() * args.steps * dist.world
-    value = units / (ms_max / 1e3)
-    e2e_value = units / (e2e_ms_max / 1e3)
-
-    extra = {}
-    if args.workload == "decode_sweep" and dist.world == 1 and not args.no_prefill_summary:
-        extra["prefill_gemm"] = prefill_summary(device, peaks)
-
-    cpu = None   # the oracle's host-core baseline: rank 0 of a 1-GPU run only
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wk, args.cpu_seconds)
-
     h2d, d2h = wk.e2e_bytes()
-    line = {
-        "metric": wk.metric, "value": round(value, 3), "unit": wk.unit,
-        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_max / args.steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4 x q8_0 (int32 subblock sums / exact fp16 operands, fp32 accumulate)",
-        "data": "synthetic (seeded; shapes and distributions of the workload)",
+    return {
+        "metric": wk.metric, "value": round(units / (ms_max / 1e3), 3), "unit": wk.unit,
+        "ms_per_step": round(ms_per_step, 5),
         "config": wk.config(),
-        "impl": "nvq",
-        "timing": ("CUDA graph of the K steps replayed once, events on the launching stream "
-                   "before and after; no event nodes inside that replay"),
-        "e2e": {"value": round(e2e_value, 3), "unit": wk.unit,
+        "e2e": {"value": round(units / (e2e_ms / 1e3), 3), "unit": wk.unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "eager public API calls with pinned-host copies"},
         "gpu_launches": wk.launches_per_step() * args.steps,
         "roofline": roofline,
-        "cpu_baseline": cpu,
         "clocks": clocks,
     }
-    line.update(extra)
+
+
+def cpu_baseline(wk, seconds: float, pool):
+    """The oracle on a bounded sample of the workload: one host core, and
+    every host core through the pool (when given)."""
+    import threadpoolctl
+    rows = 64
+    with threadpoolctl.threadpool_limits(1):
+        tasks = wk.oracle_tasks(rows)
+        t0 = time.perf_counter()
+        run_tasks_serial(tasks)
+        t_small = time.perf_counter() - t0
+        rows = int(max(64, rows * seconds / max(t_small, 1e-3)))
+        tasks = wk.oracle_tasks(rows)
+        t0 = time.perf_counter()
+        units = run_tasks_serial(tasks)
+        t = time.perf_counter() - t0
+    entry = {"value": round(units / t, 6), "unit": wk.unit, "cores": 1, "kind": "oracle",
+             "sample": wk.oracle_sample_desc(rows), "seconds": round(t, 2)}
+    if pool is not None:
+        rows_all = int(rows * max(1, pool.cores * 3 // 4))
+        tasks = wk.oracle_tasks(rows_all)
+        t0 = time.perf_counter()
+        units = pool.run(tasks)
+        t = time.perf_counter() - t0
+        entry["all_cores"] = {"value": round(units / t, 6), "unit": wk.unit,
+                              "cores": pool.cores, "kind": "oracle",
+                              "sample": wk.oracle_sample_desc(rows_all),
+                              "seconds": round(t, 2),
+                              "how": "row blocks over a pool of spawned processes, one "
+                                     "numpy thread each"}
+    return entry
+
+
+def run_nvq(args, dist: Dist):
+    import gc
+
+    import torch
+    pool = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        pool = OraclePool()           # spawned before the first GPU call
+    torch.cuda.set_device(dist.local_rank)
+    device = torch.device("cuda", dist.local_rank)
+    dist.init("nccl")
+    peaks = load_peaks()
+    # everything runs on one side stream (graphs are captured on it)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
+    sampler = ClockSampler(dist.local_rank)
+    sampler.start()
+    time.sleep(0.3)
+
+    names = [args.workload]
+    if not args.no_sub:
+        names += [n for n in SUB_WORKLOADS if n != args.workload]
+    entries = {}
+    for name in names:
+        wk = make_workload(name)
+        entry = measure(wk, args, dist, peaks, device, sampler)
+        if pool is not None:
+            entry["cpu_baseline"] = cpu_baseline(
+                wk, args.cpu_seconds if name == args.workload else args.cpu_seconds / 4, pool)
+        else:
+            entry["cpu_baseline"] = None
+        entries[name] = entry
+        del wk
+        gc.collect()
+        torch.cuda.empty_cache()
+    time.sleep(0.2)
+    sampler.stop()
+    if pool is not None:
+        pool.close()
+
+    main = entries.pop(args.workload)
+    line = {
+        "metric": main["metric"], "value": main["value"], "unit": main["unit"],
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": main["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 x q8_0 (int32 subblock sums / exact fp16 operands, fp32 accumulate)",
+        "data": "synthetic (seeded; shapes and distributions of the workload)",
+        "config": main["config"],
+        "impl": "nvq",
+        "timing": ("CUDA graph of the K steps replayed once, events on the launching stream "
+                   "before and after; no event nodes inside that replay"),
+        "e2e": main["e2e"],
+        "gpu_launches": main["gpu_launches"] + sum(e["gpu_launches"] for e in entries.values()),
+        "gpu_launches_headline": main["gpu_launches"],
+        "roofline": main["roofline"],
+        "cpu_baseline": main["cpu_baseline"],
+        "clocks": main["clocks"],
+    }
+    if entries:
+        line["workloads"] = entries
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()
-
-
-def prefill_summary(device, peaks):
-    """The prefill GEMM at 2048 tokens, timed the same way (graph replay),
-    reported next to the decode line."""
-    import torch
-    wk = make_workload("prefill_m2048")
-    wk.setup(device)
-    stream = torch.cuda.current_stream(device)   # the side stream set by run_nvq
-    for _ in range(3):
-        wk.step(stream)
-    torch.cuda.synchronize()
-    steps = 10
-    graph, _ = capture_steps(wk, steps, stream, events=False)
-    graph_ev, log = capture_steps(wk, steps, stream, events=True)
-    graph.replay()
-    graph_ev.replay()
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    graph.replay()
-    end.record(stream)
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    graph_ev.replay()
-    torch.cuda.synchronize()
-    roof = roofline_entry(wk, log, peaks)
-    roof["step_achieved"] = round(log.totals()[1] / (ms / 1e3) / 1e12, 2)
-    out = {"workload": "prefill_m2048", "shapes_KN": [list(s) for s in wk.shapes],
-           "step_TFLOPs": round(wk.units_per_step() * steps / (ms / 1e3), 2),
-           "roofline": roof}
-    del graph, graph_ev, wk
-    torch.cuda.empty_cache()
-    return out
-
-
-def cpu_baseline(wk, seconds: float):
-    """The oracle, timed on one host core on a bounded sample of the workload."""
-    import threadpoolctl
-    size = 64
-    with threadpoolctl.threadpool_limits(1):
-        wk.oracle_prepare(size)
-        t0 = time.perf_counter()
-        wk.oracle_step()
-        t_small = time.perf_counter() - t0
-        size = int(max(64, min(65536, size * seconds / max(t_small, 1e-3))))
-        wk.oracle_prepare(size)
-        t0 = time.perf_counter()
-        units = wk.oracle_step()
-        t = time.perf_counter() - t0
-    return {"value": round(units / t, 6), "unit": wk.unit, "cores": 1, "kind": "oracle",
-            "sample": wk.oracle_sample_desc(size), "seconds": round(t, 2)}
 
 
 def run_reference(args, dist: Dist):
     """The oracle as the reference arm: rank 0 only, on the host cores."""
     if dist.rank != 0:
         return
-    import threadpoolctl
     wk = make_workload(args.workload)
+    pool = OraclePool()
     # size the per-step sample so that warm-up + timed steps take about
     # 6 * --cpu-seconds in total (a few minutes at most)
     budget = 6 * args.cpu_seconds / (args.steps + args.warmup)
-    size = 64
-    with threadpoolctl.threadpool_limits(1):
-        wk.oracle_prepare(size)
-        t0 = time.perf_counter()
-        wk.oracle_step()
-        t_small = time.perf_counter() - t0
-        size = int(max(8, min(65536, size * budget / max(t_small, 1e-4))))
-        wk.oracle_prepare(size)
-        for _ in range(args.warmup):
-            wk.oracle_step()
-        t0 = time.perf_counter()
-        units = 0.0
-        for _ in range(args.steps):
-            units += wk.oracle_step()
-        t = time.perf_counter() - t0
+    rows = 64
+    tasks = wk.oracle_tasks(rows)
+    t0 = time.perf_counter()
+    pool.run(tasks)
+    t_small = time.perf_counter() - t0
+    rows = int(max(64, rows * budget / max(t_small, 1e-4)))
+    tasks = wk.oracle_tasks(rows)
+    for _ in range(args.warmup):
+        pool.run(tasks)
+    t0 = time.perf_counter()
+    units = 0.0
+    for _ in range(args.steps):
+        units += pool.run(tasks)
+    t = time.perf_counter() - t0
+    pool.close()
     value = units / t
-    desc = wk.oracle_sample_desc(size)
+    desc = wk.oracle_sample_desc(rows)
     line = {
         "metric": wk.metric, "value": round(value, 6), "unit": wk.unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -801,7 +883,7 @@ def run_reference(args, dist: Dist):
         "data": "synthetic (seeded; a bounded sample of the workload per step)",
         "config": dict(wk.config(), sample_per_step=desc),
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 6), "unit": wk.unit, "cores": 1,
+        "cpu_baseline": {"value": round(value, 6), "unit": wk.unit, "cores": pool.cores,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 6), "unit": wk.unit,
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -814,14 +896,15 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode_sweep")
     ap.add_argument("--impl", choices=["nvq", "reference"], default="nvq")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="target duration of the oracle CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="target duration of the headline's oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill-summary", action="store_true")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="measure only --workload (no other workloads in the line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

@@ -113,6 +113,23 @@ def weights(workload: str, tensor: str, N: int, K: int,
     return out
 
 
+def weight_rows(workload: str, tensor: str, N: int, K: int, rows: int,
+                boost_columns: bool = False) -> np.ndarray:
+    """The first `rows` rows of weights(workload, tensor, N, K, ...), drawn
+    without generating the rest of the matrix (row blocks have their own
+    seed sequences)."""
+    rows = min(rows, N)
+    ss = seed_sequence(workload, tensor, N, K)
+    nblocks = (rows + ROW_BLOCK - 1) // ROW_BLOCK
+    out = np.empty((nblocks * ROW_BLOCK, K), dtype=np.float32)
+    for b in range(nblocks):
+        _fill_rows(ss, out, b, WEIGHT_STD)
+    out = out[:rows]
+    if boost_columns:
+        out[:, boosted_columns(workload, tensor, K)] *= np.float32(COLUMN_BOOST)
+    return out
+
+
 def activations(workload: str, tensor: str, M: int, K: int,
                 dist: str = "normal", outliers: bool = False) -> np.ndarray:
     """fp32 x[M, K]: N(0, 1) or Student-t(nu=4); optionally 0.1 % of the

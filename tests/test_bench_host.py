@@ -77,7 +77,9 @@ def test_reference_arm_under_two_ranks_prints_one_line():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 3
     assert line["value"] > 0 and line["higher_is_better"] is True
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    cores = len(os.sched_getaffinity(0))
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] == min(cores, 128)
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["config"]["workload"] == "gemv_4096"
 
@@ -122,3 +124,29 @@ def test_workload_table():
         assert wk.config()["workload"] == name
     with pytest.raises(SystemExit):
         bench.make_workload("no_such_workload")
+
+
+def test_oracle_tasks_split_over_workers_keep_their_units():
+    """The all-cores oracle baseline splits each sample's repetitions over
+    the pool without losing or double-counting work."""
+    wk = bench.make_workload("gemv_4096")
+    tasks = wk.oracle_tasks(300)
+    (codes, scales, g, x, reps, units), = tasks
+    assert reps == 5 and codes.shape[0] == bench.ORACLE_BASE_ROWS      # 300 rows -> 5 x 64
+    assert abs(units - 5 * 64 * 4096 * 0.5625 / 1e9) < 1e-12
+    parts = bench.split_tasks(tasks, 3)
+    assert sum(p[4] for p in parts) == reps
+    assert abs(sum(p[5] for p in parts) - units) < 1e-12
+    assert abs(bench.run_tasks_serial(parts) - bench.run_tasks_serial(tasks)) < 1e-15
+
+
+def test_cpu_baseline_reports_one_core_and_all_cores():
+    wk = bench.make_workload("gemv_4096")
+    pool = bench.OraclePool()
+    try:
+        cb = bench.cpu_baseline(wk, 0.2, pool)
+    finally:
+        pool.close()
+    assert cb["cores"] == 1 and cb["kind"] == "oracle" and cb["value"] > 0
+    assert cb["all_cores"]["cores"] == pool.cores and cb["all_cores"]["value"] > 0
+    assert "64 rows" in cb["sample"]

@@ -87,3 +87,10 @@ def test_workload_cases_follow_the_recipe():
     assert np.array_equal(x[:, ch], plain[:, ch] * 50)
     assert [name for name, _, _ in wl.STACK_LINEARS] == ["q", "k", "v", "o", "up", "gate", "down"]
     assert sum(K * N for _, K, N in wl.STACK_LINEARS) * wl.STACK_LAYERS * 0.5625 / 1e9 == pytest.approx(17.93, abs=0.01)
+
+
+def test_weight_rows_equal_the_leading_rows_of_the_full_matrix():
+    full = wl.weights("wl_test", "W", 2500, 128, boost_columns=True)
+    for rows in (1, 1024, 1500, 2500, 9999):
+        part = wl.weight_rows("wl_test", "W", 2500, 128, rows, boost_columns=True)
+        assert np.array_equal(part, full[:rows])
