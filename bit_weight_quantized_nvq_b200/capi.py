@@ -44,6 +44,10 @@ SIGNATURES = {
     "nvq_quantize_act_q8_0": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp]),
     "nvq_gemv": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp]),
+    "nvq_gemv_requant": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp, _vp,
+                                        _vp, _vp, _vp, _vp]),
+    "nvq_gemv_grouped": (ctypes.c_int, [ctypes.POINTER(Linear), _c_i64, _vp, _vp, _c_i64,
+                                        ctypes.POINTER(_vp), _vp]),
     "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
@@ -154,6 +158,44 @@ def gemv(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
         _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), M, _ptr(y),
         _stream(stream)))
     return y
+
+
+def gemv_requant(codes: torch.Tensor, scales: torch.Tensor, g: float, q: torch.Tensor,
+                 d: torch.Tensor, counters: torch.Tensor, y: torch.Tensor | None = None,
+                 q_out: torch.Tensor | None = None, d_out: torch.Tensor | None = None,
+                 stream=None):
+    """One token's GEMV that also emits Q8_0 of y (nvq_gemv_requant):
+    returns (y fp32 [1, N], q_out int8 [1, N], d_out float16 [1, N/32]).
+    counters: device int32 [N/32], zero before the first call."""
+    N = codes.shape[0]
+    M, K = q.shape
+    if y is None:
+        y = torch.empty((1, N), dtype=torch.float32, device=q.device)
+    if q_out is None:
+        q_out = torch.empty((1, N), dtype=torch.int8, device=q.device)
+    if d_out is None:
+        d_out = torch.empty((1, N // 32), dtype=torch.float16, device=q.device)
+    _check("nvq_gemv_requant", _lib.nvq_gemv_requant(
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(q), _ptr(d), _ptr(y), _ptr(q_out),
+        _ptr(d_out), _ptr(counters), _stream(stream)))
+    return y, q_out, d_out
+
+
+def gemv_grouped(mats, q: torch.Tensor, d: torch.Tensor, ys=None, stream=None):
+    """nvq_gemv of several (codes, scales, g) with the same K against one
+    activation: returns the list of y [M, N_i]."""
+    M, K = q.shape
+    arr = (Linear * len(mats))()
+    for i, (codes, scales, g) in enumerate(mats):
+        arr[i] = Linear(codes.data_ptr(), scales.data_ptr(), float(g), codes.shape[0],
+                        codes.shape[1] * 2)
+    if ys is None:
+        ys = [torch.empty((M, c.shape[0]), dtype=torch.float32, device=q.device)
+              for c, _, _ in mats]
+    ptrs = (_vp * len(mats))(*[t.data_ptr() for t in ys])
+    _check("nvq_gemv_grouped", _lib.nvq_gemv_grouped(arr, len(mats), _ptr(q), _ptr(d), M, ptrs,
+                                                     _stream(stream)))
+    return ys
 
 
 def gemm_workspace_size(M: int, N: int, K: int) -> int:

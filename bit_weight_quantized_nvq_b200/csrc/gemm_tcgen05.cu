@@ -105,42 +105,13 @@ constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + slack to align to 1
 static_assert(kOffCodes % 1024 == 0, "swizzled tiles need 1 KB alignment");
 static_assert(kSmemBytes <= 232448, "over the opt-in shared memory of one CTA");
 
-// fp16 high bytes of the E2M1 values: 0, .5, 1, 1.5, 2, 3, 4, 6 are 0x0000,
-// 0x3800, 0x3C00, 0x3E00, 0x4000, 0x4200, 0x4400, 0x4600 (low bytes zero);
-// codes 8..15 carry the sign bit 0x80.
-constexpr uint32_t kHbPosLo = 0x3E3C3800u;
-constexpr uint32_t kHbPosHi = 0x46444240u;
-constexpr uint32_t kHbNegLo = 0xBEBCB880u;
-constexpr uint32_t kHbNegHi = 0xC6C4C2C0u;
-
 // bit 0: a pipeline wait of the GEMM timed out
 __device__ unsigned int g_gemm_error_flags = 0;
 
-__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ __half2 bits_h2(uint32_t u) {
-  return *reinterpret_cast<__half2*>(&u);
-}
-
-// Eight codes (one word) -> eight fp16 w' = E2M1 * s, as one 16-byte chunk.
-__device__ __forceinline__ uint4 expand8(uint32_t w, __half2 s2) {
-  uint32_t lo, hi;
-  dev::lut16_x8<kHbPosLo, kHbPosHi, kHbNegLo, kHbNegHi>(w, lo, hi);
-  uint4 r;
-  r.x = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x1404)), s2));
-  r.y = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x3424)), s2));
-  r.z = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x1404)), s2));
-  r.w = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x3424)), s2));
-  return r;
-}
-
-__device__ __forceinline__ __half2 ue4m3x2_to_half2(uint32_t two_bytes) {
-  uint32_t h2;
-  const uint16_t in = static_cast<uint16_t>(two_bytes);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  return bits_h2(h2);
-}
+using dev::bits_h2;
+using dev::expand8;
+using dev::h2_bits;
+using dev::ue4m3x2_to_half2;
 
 // ---------------------------------------------------------------------------
 // 1. activation expansion
@@ -587,6 +558,7 @@ CtxGetCurrentFn ctx_get_current() {
 }  // namespace
 
 size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
+  if (gemm_small_supported(M, K)) return gemm_small_workspace_size(M, K);
   const int64_t mp = padded_tokens(M);
   return static_cast<size_t>(4 * mp * K + 4 * mp);
 }
@@ -629,15 +601,19 @@ cudaError_t gemm_error_flags(bool clear, unsigned int* flags) {
   return e;
 }
 
+cudaError_t expand_activations(const int8_t* q, const uint16_t* d, int64_t M, int64_t M_pad,
+                               int64_t K, void* act, float* tok_scale, cudaStream_t stream) {
+  expand_act_kernel<<<static_cast<unsigned>(M_pad), 256, 0, stream>>>(
+      q, reinterpret_cast<const __half*>(d), static_cast<int>(M), static_cast<int>(K),
+      static_cast<int>(M_pad), static_cast<__half*>(act), tok_scale);
+  return cudaGetLastError();
+}
+
 cudaError_t gemm_expand(const int8_t* q, const uint16_t* d, int64_t M, int64_t K,
                         void* workspace, cudaStream_t stream) {
   const int64_t M_pad = padded_tokens(M);
-  __half* act = static_cast<__half*>(workspace);
   float* tok_scale = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + 4 * M_pad * K);
-  expand_act_kernel<<<static_cast<unsigned>(M_pad), 256, 0, stream>>>(
-      q, reinterpret_cast<const __half*>(d), static_cast<int>(M), static_cast<int>(K),
-      static_cast<int>(M_pad), act, tok_scale);
-  return cudaGetLastError();
+  return expand_activations(q, d, M, M_pad, K, workspace, tok_scale, stream);
 }
 
 cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
@@ -689,6 +665,8 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
 cudaError_t launch_gemm(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
                         int64_t K, const int8_t* q, const uint16_t* d, int64_t M, float* y,
                         void* workspace, cudaStream_t stream) {
+  if (gemm_small_supported(M, K))
+    return launch_gemm_small(codes, scales, g, N, K, q, d, M, y, workspace, stream);
   cudaError_t e = gemm_expand(q, d, M, K, workspace, stream);
   if (e != cudaSuccess) return e;
   return gemm_main(codes, scales, g, N, K, M, y, workspace, stream);

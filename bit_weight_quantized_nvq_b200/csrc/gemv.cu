@@ -31,7 +31,12 @@
 //    d and the bias corrections sit in registers for the whole kernel.  The
 //    weights are decoded to the +12-biased integer LUT of the "Bias trick"
 //    paragraph with sign-replicating byte permutes, and the bias is removed
-//    by starting each subblock's dp4a chain at corr = -12 * bsum16.
+//    by starting each subblock's dp4a chain at corr = -12 * bsum16.  One
+//    launch may cover up to three matrices that read the same activations
+//    (their rows concatenated, so the row ranges stay balanced), and a matrix
+//    may also emit the Q8_0 quantisation of its output: the CTA that stores
+//    the last of a 32-row block's outputs (per-block arrival counters)
+//    quantises that block, with the activation quantiser's IEEE operations.
 //  * gemv_m1_kernel (M = 1, other K % 256 == 0): the same ring with groups
 //    of 16 rows (whole K, or K segments of at most 5120 elements) and the
 //    activations staged once per CTA in shared memory; biased LUT with an
@@ -312,6 +317,7 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
 // one (griddepcontrol) before it reads any global input, so launch latency
 // and prologue overlap the previous kernel's tail without changing results.
 constexpr uint32_t kRegStageMax = 46080;
+constexpr int kMaxGroup = 3;       // matrices per register-schedule launch
 
 __host__ __device__ constexpr int reg_rows(int K, int wpr) {
   int r = kM1Consumers / wpr;
@@ -331,12 +337,80 @@ __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The matrices of one register-schedule launch: up to kMaxGroup weight
+// matrices with the same K that read the same activations (q, k, v of a
+// layer; up and gate), their rows concatenated; each may also emit the Q8_0
+// quantisation of its output (the requantisation that feeds the next
+// product), which the CTA completing a 32-row block carries out.
+struct RegMat {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  float* y;
+  int8_t* rq_q;      // Q8_0 codes of y [N] (nullptr: no requantisation)
+  __half* rq_d;      // Q8_0 scales of y [N / 32]
+  int* rq_cnt;       // per 32-row block: rows written so far (0 between launches)
+  float half_g;
+  int N;
+  int row_off;       // first row of this matrix among the concatenated rows
+};
+struct RegGroup {
+  RegMat m[kMaxGroup];
+  int count;
+  int rows;          // concatenated rows
+};
+
+// Q8_0 of the 32 outputs of block b, one lane per output: the same IEEE
+// operations as the activation quantiser (amax, d32 = amax/127, q =
+// rint(y/d32) clamped to +-127, d = fp16(d32)), so the codes are those the
+// quantiser would produce from y.
+__device__ __forceinline__ void requant_block_warp(const RegMat& m, int b, int lane) {
+  const float v = __ldcg(m.y + 32 * b + lane);
+  float a = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  const float d32 = __fdiv_rn(a, 127.0f);
+  int qi = 0;
+  if (d32 > 0.0f) qi = max(-127, min(127, __float2int_rn(__fdiv_rn(v, d32))));
+  m.rq_q[32 * b + lane] = static_cast<int8_t>(qi);
+  if (lane == 0) m.rq_d[b] = __float2half_rn(d32);
+}
+// The same by one thread.
+__device__ __forceinline__ void requant_block_thread(const RegMat& m, int b) {
+  float a = 0.0f;
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(__ldcg(m.y + 32 * b + i)));
+  const float d32 = __fdiv_rn(a, 127.0f);
+  for (int i = 0; i < 32; ++i) {
+    int qi = 0;
+    if (d32 > 0.0f) qi = max(-127, min(127, __float2int_rn(__fdiv_rn(__ldcg(m.y + 32 * b + i), d32))));
+    m.rq_q[32 * b + i] = static_cast<int8_t>(qi);
+  }
+  m.rq_d[b] = __float2half_rn(d32);
+}
+// Row `row` of m has been stored (by this thread): count it in its block and
+// report whether this thread completed the block (classic fence + counter
+// protocol: the store is visible device-wide before the count).
+__device__ __forceinline__ bool arrive_row(const RegMat& m, int row) {
+  __threadfence();
+  const bool last = atomicAdd(m.rq_cnt + (row >> 5), 1) == 31;
+  if (last) __threadfence();
+  return last;
+}
+
+// The next stage of a CTA's concatenated row range: at most R rows, all of
+// one matrix.
+__device__ __forceinline__ void next_stage(const RegGroup& grp, int& gr, int r_end, int R,
+                                           int& mi, int& row0, int& nrows) {
+  mi = 0;
+  while (mi + 1 < grp.count && gr >= grp.m[mi + 1].row_off) ++mi;
+  row0 = gr - grp.m[mi].row_off;
+  nrows = min(R, min(r_end - gr, grp.m[mi].N - row0));
+  gr += nrows;
+}
+
 template <int NPL, int WPR, bool ISUM>
 __global__ void __launch_bounds__(kM1Threads, 1)
-gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                   float half_g, int N, int K, const int8_t* __restrict__ q,
-                   const __half* __restrict__ d, float* __restrict__ y,
-                   int32_t* __restrict__ isum) {
+gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __restrict__ q,
+                   const __half* __restrict__ d, int32_t* __restrict__ isum) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int R = reg_rows(K, WPR);
   const int active = R * WPR;                      // consumer warps in use
@@ -351,9 +425,8 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x;
-  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
-  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
-  const int total = (r_end - r_begin + R - 1) / R;   // stages = row groups
+  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * grp.rows / G);
+  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * grp.rows / G);
 
   grid_dependents_launch();
   if (threadIdx.x == 0) {
@@ -370,21 +443,27 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
   if (warp == kM1Consumers) {
     // ------------- producer: bulk copies, and the sum of row partials --------
     if (lane != 0) return;
+    int smi[kM1Stages] = {}, srow[kM1Stages] = {}, snr[kM1Stages] = {};   // stages in flight
     auto finalize = [&](int it) {   // rows of stage `it`, once its slot is empty
       if (WPR == 1) return;
       const int s = it % kM1Stages;
-      const int row0 = r_begin + it * R;
-      const int nrows = min(R, r_end - row0);
-      for (int r = 0; r < nrows; ++r) {
+      const RegMat& m = grp.m[smi[s]];
+      for (int r = 0; r < snr[s]; ++r) {
         float v = 0.0f;
 #pragma unroll
         for (int p = 0; p < WPR; ++p) v += part[s * kM1Consumers + r * WPR + p];
-        y[row0 + r] = v * half_g;
+        const int row = srow[s] + r;
+        m.y[row] = v * m.half_g;
+        if (m.rq_q != nullptr && arrive_row(m, row)) {
+          requant_block_thread(m, row >> 5);
+          atomicExch(m.rq_cnt + (row >> 5), 0);
+        }
       }
     };
     int issued = 0;
     bool ok = true;
-    for (int it = 0; it < total; ++it) {
+    int gr = r_begin;
+    for (int it = 0; gr < r_end; ++it) {
       const int s = it % kM1Stages;
       const uint32_t ph = (it / kM1Stages) & 1;
       if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
@@ -394,20 +473,24 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
         break;
       }
       if (it >= kM1Stages) finalize(it - kM1Stages);
-      const int row0 = r_begin + it * R;
-      const int nrows = min(R, r_end - row0);
+      int mi, row0, nrows;
+      next_stage(grp, gr, r_end, R, mi, row0, nrows);
+      smi[s] = mi;
+      srow[s] = row0;
+      snr[s] = nrows;
+      const RegMat& m = grp.m[mi];
       const uint32_t bar = ptx::smem_addr(full + s);
       uint8_t* st = smem + s * stage_bytes;
       ptx::mbar_arrive_expect_tx(bar, nrows * (row_code + row_scale));
-      ptx::bulk_load(ptx::smem_addr(st), codes + static_cast<size_t>(row0) * row_code,
+      ptx::bulk_load(ptx::smem_addr(st), m.codes + static_cast<size_t>(row0) * row_code,
                      nrows * row_code, bar);
       ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
-                     scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
+                     m.scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
       ++issued;
     }
     if (ok) {
       // the last stages: wait until consumed, then add their partials
-      for (int it = max(0, total - kM1Stages); it < total; ++it) {
+      for (int it = max(0, issued - kM1Stages); it < issued; ++it) {
         if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + it % kM1Stages),
                                     (it / kM1Stages) & 1, abort_flag, kWaitLimitNs)) {
           *abort_flag = 1;
@@ -446,18 +529,20 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
     c0[i] = -12 * s0;
     c1[i] = -12 * s1;
   }
-  for (int it = 0; it < total; ++it) {
+  int gr = r_begin;
+  for (int it = 0; gr < r_end; ++it) {
     const int s = it % kM1Stages;
     const uint32_t ph = (it / kM1Stages) & 1;
+    int mi, row0, nrows;
+    next_stage(grp, gr, r_end, R, mi, row0, nrows);
     if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
       *abort_flag = 1;
       raise_timeout();
       break;
     }
-    const int row0 = r_begin + it * R;
-    const int nrows = min(R, r_end - row0);
     float acc = 0.0f;
     if (rl < nrows) {
+      const RegMat& m = grp.m[mi];
       const uint8_t* st = smem + s * stage_bytes;
       const uint4* cw = reinterpret_cast<const uint4*>(st + rl * row_code) + p * (NPL * 32);
       const uint16_t* sw =
@@ -474,16 +559,24 @@ gemv_m1_reg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict_
         const int i0 = dev::dot16_biased(w[i].x, w[i].y, qa[i], c0[i]);
         const int i1 = dev::dot16_biased(w[i].z, w[i].w, qb[i], c1[i]);
         if constexpr (ISUM)
-          store_isum(isum, 0, N, row0 + rl, K, p * (NPL * 32) + lane + 32 * i, i0, i1);
+          store_isum(isum, 0, m.N, row0 + rl, K, p * (NPL * 32) + lane + 32 * i, i0, i1);
         const float2 sf = dev::ue4m3x2_to_float2(s2[i]);
         acc = fmaf(dd[i], fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
       }
       acc = dev::warp_sum(acc);
-      if (lane == 0) {
-        if (WPR == 1)
-          y[row0 + rl] = acc * half_g;
-        else
-          part[s * kM1Consumers + warp] = acc;
+      if (WPR == 1) {
+        const int row = row0 + rl;
+        bool last = false;
+        if (lane == 0) {
+          m.y[row] = acc * m.half_g;
+          if (m.rq_q != nullptr) last = arrive_row(m, row);
+        }
+        if (m.rq_q != nullptr && __shfl_sync(0xffffffffu, last, 0)) {
+          requant_block_warp(m, row >> 5, lane);
+          if (lane == 0) atomicExch(m.rq_cnt + (row >> 5), 0);
+        }
+      } else if (lane == 0) {
+        part[s * kM1Consumers + warp] = acc;
       }
     }
     __syncwarp();
@@ -723,14 +816,13 @@ cudaError_t launch_m1(const uint8_t* codes, const uint8_t* scales, float g, int6
 }
 
 template <int NPL, int WPR, bool ISUM>
-cudaError_t launch_m1_reg(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
-                          int64_t K, const int8_t* q, const uint16_t* d, float* y,
+cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const uint16_t* d,
                           int32_t* isum, cudaStream_t stream) {
   auto kernel = gemv_m1_reg_kernel<NPL, WPR, ISUM>;
   static SmemAttrOnce attr;
   cudaError_t e = attr.ensure(kernel, static_cast<int>(kSmemPerCtaMax));
   if (e != cudaSuccess) return e;
-  const int64_t ctas = std::min<int64_t>(device_sm_count(), N);
+  const int64_t ctas = std::min<int64_t>(device_sm_count(), grp.rows);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kM1Threads);
@@ -741,19 +833,27 @@ cudaError_t launch_m1_reg(const uint8_t* codes, const uint8_t* scales, float g, 
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, codes, scales, 0.5f * g, static_cast<int>(N),
-                            static_cast<int>(K), q, reinterpret_cast<const __half*>(d), y, isum);
+  return cudaLaunchKernelEx(&cfg, kernel, grp, static_cast<int>(K), q,
+                            reinterpret_cast<const __half*>(d), isum);
 }
 
 // The register schedule covers K = 1024 * NPL * WPR for the (NPL, WPR) pairs
 // instantiated here; returns cudaErrorNotSupported for other K.
+bool reg_supported(int64_t K) {
+  if (K % 1024 != 0) return false;
+  switch (K / 1024) {
+    case 4: case 5: case 6: case 8: case 10: case 12: case 15: case 16: case 20: case 25:
+      return true;
+    default:
+      return false;
+  }
+}
+
 template <bool ISUM>
-cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, float g,
-                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
-                                   float* y, int32_t* isum, cudaStream_t stream) {
-  if (K % 1024 != 0) return cudaErrorNotSupported;
-#define NVQ_REG(npl, wpr) \
-  return launch_m1_reg<npl, wpr, ISUM>(codes, scales, g, N, K, q, d, y, isum, stream)
+cudaError_t launch_m1_reg_group(const RegGroup& grp, int64_t K, const int8_t* q,
+                                const uint16_t* d, int32_t* isum, cudaStream_t stream) {
+  if (!reg_supported(K)) return cudaErrorNotSupported;
+#define NVQ_REG(npl, wpr) return launch_m1_reg<npl, wpr, ISUM>(grp, K, q, d, isum, stream)
   switch (K / 1024) {
     case 4: NVQ_REG(4, 1);
     case 5: NVQ_REG(5, 1);
@@ -768,6 +868,27 @@ cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, 
     default: return cudaErrorNotSupported;
   }
 #undef NVQ_REG
+}
+
+RegMat reg_mat(const uint8_t* codes, const uint8_t* scales, float g, int64_t N, float* y) {
+  RegMat m = {};
+  m.codes = codes;
+  m.scales = scales;
+  m.y = y;
+  m.half_g = 0.5f * g;
+  m.N = static_cast<int>(N);
+  return m;
+}
+
+template <bool ISUM>
+cudaError_t launch_m1_reg_dispatch(const uint8_t* codes, const uint8_t* scales, float g,
+                                   int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
+                                   float* y, int32_t* isum, cudaStream_t stream) {
+  RegGroup grp = {};
+  grp.m[0] = reg_mat(codes, scales, g, N, y);
+  grp.count = 1;
+  grp.rows = static_cast<int>(N);
+  return launch_m1_reg_group<ISUM>(grp, K, q, d, isum, stream);
 }
 
 template <int MT, bool ISUM>
@@ -832,6 +953,43 @@ cudaError_t launch_gemv_isum(const uint8_t* codes, const uint8_t* scales, float 
                              int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
                              int64_t M, float* y, int32_t* isum, cudaStream_t stream) {
   return launch_gemv_any<true>(codes, scales, g, N, K, q, d, M, y, isum, stream);
+}
+
+cudaError_t launch_gemv_group(const GemvTarget* t, int n, int64_t K, const int8_t* q,
+                              const uint16_t* d, cudaStream_t stream) {
+  int done = 0;
+  while (done < n) {
+    // one launch for up to kMaxGroup matrices of the register schedule
+    if (reg_supported(K)) {
+      RegGroup grp = {};
+      int rows = 0;
+      const int cnt = std::min(kMaxGroup, n - done);
+      for (int i = 0; i < cnt; ++i) {
+        const GemvTarget& x = t[done + i];
+        RegMat m = reg_mat(x.codes, x.scales, x.g, x.N, x.y);
+        m.rq_q = x.rq_q;
+        m.rq_d = reinterpret_cast<__half*>(x.rq_d);
+        m.rq_cnt = x.rq_cnt;
+        m.row_off = rows;
+        rows += static_cast<int>(x.N);
+        grp.m[i] = m;
+      }
+      grp.count = cnt;
+      grp.rows = rows;
+      const cudaError_t e = launch_m1_reg_group<false>(grp, K, q, d, nullptr, stream);
+      if (e != cudaSuccess) return e;
+      done += cnt;
+      continue;
+    }
+    // other K: the product, then the quantiser on its output
+    const GemvTarget& x = t[done];
+    cudaError_t e = launch_gemv(x.codes, x.scales, x.g, x.N, K, q, d, 1, x.y, stream);
+    if (e == cudaSuccess && x.rq_q != nullptr)
+      e = launch_quantize_q8_0(x.y, 1, x.N, x.rq_q, x.rq_d, stream);
+    if (e != cudaSuccess) return e;
+    ++done;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream) {

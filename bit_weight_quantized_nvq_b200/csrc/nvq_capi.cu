@@ -137,6 +137,65 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                                       static_cast<cudaStream_t>(stream)));
 }
 
+nvq_status nvq_gemv_requant(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                            int64_t K, const int8_t* q, const uint16_t* d, float* y,
+                            int8_t* q_out, uint16_t* d_out, int32_t* counters, void* stream) {
+  nvq_status st = check_dot_args(codes, scales, N, K, q, d, 1, y, 1, 1, true);
+  if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
+  if (N % 32 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (N == 0) return NVQ_OK;
+  if (!q_out || !d_out || !counters) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(q_out) || !aligned16(d_out) || !aligned16(counters)) return NVQ_ERR_MISALIGNED;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  nvq::GemvTarget t = {codes, scales, g, N, y, q_out, d_out, counters};
+  return cuda_status(nvq::launch_gemv_group(&t, 1, K, q, d, static_cast<cudaStream_t>(stream)));
+}
+
+nvq_status nvq_gemv_grouped(const nvq_linear* linears, int64_t count, const int8_t* q,
+                            const uint16_t* d, int64_t M, float* const* ys, void* stream) {
+  if (count < 0 || M < 0) return NVQ_ERR_INVALID_ARG;
+  if (count == 0 || M == 0) return NVQ_OK;
+  if (!linears || !ys) return NVQ_ERR_INVALID_ARG;
+  const int64_t K = linears[0].K;
+  int64_t rows = 0;
+  for (int64_t i = 0; i < count; ++i) {
+    const nvq_linear& L = linears[i];
+    if (L.K != K) return NVQ_ERR_BAD_SHAPE;
+    nvq_status st = check_dot_args(L.codes, L.scales, L.N, L.K, q, d, M, ys[i], 1, 16, true);
+    if (st != NVQ_OK) return st;
+    if (!(L.g == L.g)) return NVQ_ERR_INVALID_ARG;
+    rows += L.N;
+  }
+  if (rows > (int64_t{1} << 30)) return NVQ_ERR_BAD_SHAPE;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M == 1) {
+    constexpr int kBatch = 16;
+    nvq::GemvTarget t[kBatch];
+    for (int64_t i0 = 0; i0 < count; i0 += kBatch) {
+      int n = 0;
+      for (int64_t i = i0; i < count && n < kBatch; ++i) {
+        if (linears[i].N == 0) continue;
+        t[n++] = {linears[i].codes, linears[i].scales, linears[i].g, linears[i].N, ys[i],
+                  nullptr, nullptr, nullptr};
+      }
+      st = cuda_status(nvq::launch_gemv_group(t, n, K, q, d, s));
+      if (st != NVQ_OK) return st;
+    }
+    return NVQ_OK;
+  }
+  for (int64_t i = 0; i < count; ++i) {
+    const nvq_linear& L = linears[i];
+    if (L.N == 0) continue;
+    st = cuda_status(nvq::launch_gemv(L.codes, L.scales, L.g, L.N, K, q, d, M, ys[i], s));
+    if (st != NVQ_OK) return st;
+  }
+  return NVQ_OK;
+}
+
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || K <= 0 || N < 0) return 0;
   return nvq::gemm_workspace_size(M, N, K);
@@ -200,9 +259,11 @@ nvq_status nvq_error_flags(unsigned int* flags, int clear) {
   if (!flags) return NVQ_ERR_INVALID_ARG;
   nvq_status st = check_device();
   if (st != NVQ_OK) return st;
-  unsigned int gemv = 0, gemm = 0;
+  unsigned int gemv = 0, gemm = 0, gemm_small = 0;
   cudaError_t e = nvq::gemv_error_flags(clear != 0, &gemv);
   if (e == cudaSuccess) e = nvq::gemm_error_flags(clear != 0, &gemm);
+  if (e == cudaSuccess) e = nvq::gemm_small_error_flags(clear != 0, &gemm_small);
+  gemm |= gemm_small;
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_status(e);

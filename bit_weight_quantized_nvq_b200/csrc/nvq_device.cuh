@@ -125,6 +125,45 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
+// ---- fp16 operand expansion (tensor-core paths) ------------------------------
+// fp16 high bytes of the E2M1 values: 0, .5, 1, 1.5, 2, 3, 4, 6 are 0x0000,
+// 0x3800, 0x3C00, 0x3E00, 0x4000, 0x4200, 0x4400, 0x4600 (low bytes zero);
+// codes 8..15 carry the sign bit 0x80.
+constexpr uint32_t kHbPosLo = 0x3E3C3800u;
+constexpr uint32_t kHbPosHi = 0x46444240u;
+constexpr uint32_t kHbNegLo = 0xBEBCB880u;
+constexpr uint32_t kHbNegHi = 0xC6C4C2C0u;
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) {
+  return *reinterpret_cast<__half2*>(&u);
+}
+
+// Eight codes (one word, element i in nibble i) -> eight fp16
+// w' = E2M1 * s as four half2 words (element 2i in the low half of word i).
+// E2M1 * s has at most 6 significant bits and lies in 2^-10 .. 2688, so the
+// fp16 product is exact.
+__device__ __forceinline__ uint4 expand8(uint32_t w, __half2 s2) {
+  uint32_t lo, hi;
+  lut16_x8<kHbPosLo, kHbPosHi, kHbNegLo, kHbNegHi>(w, lo, hi);
+  uint4 r;
+  r.x = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x1404)), s2));
+  r.y = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x3424)), s2));
+  r.z = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x1404)), s2));
+  r.w = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x3424)), s2));
+  return r;
+}
+
+// Two UE4M3 scale bytes (low byte = first subblock) to an exact half2.
+__device__ __forceinline__ __half2 ue4m3x2_to_half2(uint32_t two_bytes) {
+  uint32_t h2;
+  const uint16_t in = static_cast<uint16_t>(two_bytes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return bits_h2(h2);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

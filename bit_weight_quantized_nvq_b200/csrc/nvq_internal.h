@@ -26,6 +26,25 @@ cudaError_t launch_gemv_isum(const uint8_t* codes, const uint8_t* scales, float 
                              const uint16_t* d, int64_t M, float* y, int32_t* isum,
                              cudaStream_t stream);
 
+// One token's GEMV through several matrices with the same K that read the
+// same Q8_0 activations, as few launches as the register schedule allows;
+// a target with rq_q set also receives the Q8_0 quantisation of its output
+// (rq_q [N] codes, rq_d [N/32] fp16 scales, N % 32 == 0), bit-identical to
+// launch_quantize_q8_0 of y.  rq_cnt: N/32 ints that are 0 before the launch
+// and are left 0.
+struct GemvTarget {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  float g;
+  int64_t N;
+  float* y;
+  int8_t* rq_q;
+  uint16_t* rq_d;
+  int* rq_cnt;
+};
+cudaError_t launch_gemv_group(const GemvTarget* targets, int n, int64_t K, const int8_t* q,
+                              const uint16_t* d, cudaStream_t stream);
+
 // Test-only: a pipeline wait that can never complete, bounded by limit_ns;
 // result[0] = 1 if the wait completed (never), result[1] = microseconds waited.
 cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream);
@@ -41,7 +60,19 @@ cudaError_t launch_gemm(const uint8_t* codes, const uint8_t* scales, float g,
                         int64_t N, int64_t K, const int8_t* q,
                         const uint16_t* d, int64_t M, float* y,
                         void* workspace, cudaStream_t stream);
-// The two halves of launch_gemm: expand Q8_0 activations into the
+// Q8_0 activations -> the exact fp16 pairs [hi rows 0..M_pad-1 | lo rows
+// M_pad..2*M_pad-1] x K in `act` (rows >= M zero) and M_pad token scales.
+cudaError_t expand_activations(const int8_t* q, const uint16_t* d, int64_t M, int64_t M_pad,
+                               int64_t K, void* act, float* tok_scale, cudaStream_t stream);
+// The small-token tensor-core schedule (M = 1..16, K % 256 == 0), which
+// launch_gemm and gemm_workspace_size select by themselves.
+bool gemm_small_supported(int64_t M, int64_t K);
+size_t gemm_small_workspace_size(int64_t M, int64_t K);
+cudaError_t launch_gemm_small(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                              int64_t K, const int8_t* q, const uint16_t* d, int64_t M, float* y,
+                              void* workspace, cudaStream_t stream);
+cudaError_t gemm_small_error_flags(bool clear, unsigned int* flags);
+// The two halves of launch_gemm for the large-token schedule: expand Q8_0 activations into the
 // workspace, then run the tensor-core GEMM on an expanded workspace (which
 // several weight matrices with the same K may share).
 cudaError_t gemm_expand(const int8_t* q, const uint16_t* d, int64_t M, int64_t K,

@@ -1,7 +1,16 @@
 // nvq_decoder_stack: the linear layers of a dense decoder stack enqueued
 // from native code (7 products and 4 Q8_0 quantisations per layer), so a
-// 64-layer token pass issues its 700-odd launches without crossing back
-// into Python.  The dataflow of a layer is documented in include/nvq.h.
+// 64-layer token pass issues its launches without crossing back into
+// Python.  The dataflow of a layer is documented in include/nvq.h.
+//
+// One token (M = 1) takes five launches per layer: the quantiser of x; one
+// GEMV over q, k and v together (they read the same activations) that also
+// emits Q8_0(y_v); the o GEMV that emits Q8_0(y_o); one GEMV over up and gate
+// that emits Q8_0(y_up); the down GEMV.  The requantisations write the other
+// of two activation buffers than the one the launch reads.  Other token
+// counts run the quantiser and the products separately (GEMV for M <= 16,
+// the tensor-core GEMM above, whose fp16 expansion of the activations is
+// shared by the products that read it).
 #include <algorithm>
 #include <cstdint>
 
@@ -34,16 +43,24 @@ bool layer_shapes_ok(const nvq_linear* L) {
          L[kUp].K == L[kO].N && L[kGate].K == L[kO].N && L[kDown].K == L[kUp].N;
 }
 
+// Workspace: two Q8_0 activation buffers (codes, scales), the requantisation
+// block counters of v, o and up (one token), and the GEMM's expansion.
 struct Layout {
-  size_t q_off, d_off, gemm_off, total;
+  size_t q_off[2], d_off[2], cnt_off, cnt_bytes, gemm_off, total;
 };
 
 Layout workspace_layout(const nvq_linear* L, int64_t M) {
   const int64_t km = max_k(L);
+  const size_t qb = round256(static_cast<size_t>(M * km));
+  const size_t db = round256(static_cast<size_t>(M * (km / 32) * 2));
   Layout w;
-  w.q_off = 0;
-  w.d_off = round256(static_cast<size_t>(M * km));
-  w.gemm_off = w.d_off + round256(static_cast<size_t>(M * (km / 32) * 2));
+  w.q_off[0] = 0;
+  w.d_off[0] = qb;
+  w.q_off[1] = qb + db;
+  w.d_off[1] = 2 * qb + db;
+  w.cnt_off = 2 * (qb + db);
+  w.cnt_bytes = M == 1 ? round256(static_cast<size_t>((L[kV].N + L[kO].N + L[kUp].N) / 32) * 4) : 0;
+  w.gemm_off = w.cnt_off + w.cnt_bytes;
   w.total = w.gemm_off + (M > 16 ? nvq::gemm_workspace_size(M, 0, km) : 0);
   return w;
 }
@@ -96,37 +113,76 @@ extern "C" nvq_status nvq_decoder_stack(const nvq_linear* linears, int64_t n_lay
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int8_t* qa = reinterpret_cast<int8_t*>(ws + lay.q_off);
-  uint16_t* da = reinterpret_cast<uint16_t*>(ws + lay.d_off);
+  int8_t* qa[2] = {reinterpret_cast<int8_t*>(ws + lay.q_off[0]),
+                   reinterpret_cast<int8_t*>(ws + lay.q_off[1])};
+  uint16_t* da[2] = {reinterpret_cast<uint16_t*>(ws + lay.d_off[0]),
+                     reinterpret_cast<uint16_t*>(ws + lay.d_off[1])};
   void* gws = ws + lay.gemm_off;
-  const bool decode = M <= 16;
-
   cudaError_t err = cudaSuccess;
-  auto quantize = [&](const float* in, int64_t K) {
-    if (err != cudaSuccess) return;
-    err = nvq::launch_quantize_q8_0(in, M, K, qa, da, st);
-    if (err == cudaSuccess && !decode) err = nvq::gemm_expand(qa, da, M, K, gws, st);
-  };
-  auto dot = [&](const nvq_linear& W, float* y) {
-    if (err != cudaSuccess) return;
-    if (decode)
-      err = nvq::launch_gemv(W.codes, W.scales, W.g, W.N, W.K, qa, da, M, y, st);
-    else
-      err = nvq::gemm_main(W.codes, W.scales, W.g, W.N, W.K, M, y, gws, st);
-  };
-  for (int64_t l = 0; l < n_layers && err == cudaSuccess; ++l) {
-    const nvq_linear* L = linears + NVQ_STACK_LINEARS * l;
-    quantize(x, L[kQ].K);
-    dot(L[kQ], outs[kQ]);
-    dot(L[kK], outs[kK]);
-    dot(L[kV], outs[kV]);
-    quantize(outs[kV], L[kO].K);
-    dot(L[kO], outs[kO]);
-    quantize(outs[kO], L[kUp].K);
-    dot(L[kUp], outs[kUp]);
-    dot(L[kGate], outs[kGate]);
-    quantize(outs[kUp], L[kDown].K);
-    dot(L[kDown], outs[kDown]);
+
+  if (M == 1) {
+    // block counters start at zero; every launch leaves them at zero
+    int* cnt = reinterpret_cast<int*>(ws + lay.cnt_off);
+    int* cnt_v = cnt;
+    int* cnt_o = cnt_v + L0[kV].N / 32;
+    int* cnt_up = cnt_o + L0[kO].N / 32;
+    err = cudaMemsetAsync(cnt, 0, lay.cnt_bytes, st);
+    auto target = [&](const nvq_linear& W, float* y, int b, int* c) {
+      nvq::GemvTarget t = {W.codes, W.scales, W.g, W.N, y, nullptr, nullptr, nullptr};
+      if (b >= 0) {
+        t.rq_q = qa[b];
+        t.rq_d = da[b];
+        t.rq_cnt = c;
+      }
+      return t;
+    };
+    for (int64_t l = 0; l < n_layers && err == cudaSuccess; ++l) {
+      const nvq_linear* L = linears + NVQ_STACK_LINEARS * l;
+      err = nvq::launch_quantize_q8_0(x, 1, L[kQ].K, qa[0], da[0], st);
+      if (err != cudaSuccess) break;
+      const nvq::GemvTarget qkv[3] = {target(L[kQ], outs[kQ], -1, nullptr),
+                                      target(L[kK], outs[kK], -1, nullptr),
+                                      target(L[kV], outs[kV], 1, cnt_v)};
+      err = nvq::launch_gemv_group(qkv, 3, L[kQ].K, qa[0], da[0], st);
+      if (err != cudaSuccess) break;
+      const nvq::GemvTarget o = target(L[kO], outs[kO], 0, cnt_o);
+      err = nvq::launch_gemv_group(&o, 1, L[kO].K, qa[1], da[1], st);
+      if (err != cudaSuccess) break;
+      const nvq::GemvTarget ug[2] = {target(L[kUp], outs[kUp], 1, cnt_up),
+                                     target(L[kGate], outs[kGate], -1, nullptr)};
+      err = nvq::launch_gemv_group(ug, 2, L[kUp].K, qa[0], da[0], st);
+      if (err != cudaSuccess) break;
+      const nvq::GemvTarget dn = target(L[kDown], outs[kDown], -1, nullptr);
+      err = nvq::launch_gemv_group(&dn, 1, L[kDown].K, qa[1], da[1], st);
+    }
+  } else {
+    const bool decode = M <= 16;
+    auto quantize = [&](const float* in, int64_t K) {
+      if (err != cudaSuccess) return;
+      err = nvq::launch_quantize_q8_0(in, M, K, qa[0], da[0], st);
+      if (err == cudaSuccess && !decode) err = nvq::gemm_expand(qa[0], da[0], M, K, gws, st);
+    };
+    auto dot = [&](const nvq_linear& W, float* y) {
+      if (err != cudaSuccess) return;
+      if (decode)
+        err = nvq::launch_gemv(W.codes, W.scales, W.g, W.N, W.K, qa[0], da[0], M, y, st);
+      else
+        err = nvq::gemm_main(W.codes, W.scales, W.g, W.N, W.K, M, y, gws, st);
+    };
+    for (int64_t l = 0; l < n_layers && err == cudaSuccess; ++l) {
+      const nvq_linear* L = linears + NVQ_STACK_LINEARS * l;
+      quantize(x, L[kQ].K);
+      dot(L[kQ], outs[kQ]);
+      dot(L[kK], outs[kK]);
+      dot(L[kV], outs[kV]);
+      quantize(outs[kV], L[kO].K);
+      dot(L[kO], outs[kO]);
+      quantize(outs[kO], L[kUp].K);
+      dot(L[kUp], outs[kUp]);
+      dot(L[kGate], outs[kGate]);
+      quantize(outs[kUp], L[kDown].K);
+      dot(L[kDown], outs[kDown]);
+    }
   }
   if (err != cudaSuccess) {
     nvq::set_last_cuda_error(err);

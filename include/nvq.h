@@ -135,6 +135,57 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                     int64_t M, float* y, void* stream);
 
 /*
+ * nvq_gemv_requant - one token's GEMV (nvq_gemv with M = 1) whose epilogue
+ * also emits the Q8_0 quantisation of its output, the activation format the
+ * next product of a decoder layer reads (y is a layer's output, Q8_0(y) the
+ * next layer's input: "HANDOFF: flint CPU optimization (Q4_1 + NVFP4)",
+ * section 7 "Open items / next steps", item 2, on the per-32 costs around
+ * the NVFP4 x Q8_0 accumulation; the GGML type table of the spke.com 2-bit
+ * GGUF tutorial for Q8_0).
+ *
+ * y       device float [N]: as nvq_gemv.
+ * q_out   device int8 [N], d_out device uint16 (fp16 bits) [N/32]: Q8_0 of y,
+ *         bit-identical to nvq_quantize_act_q8_0 applied to this y.
+ * counters device int32 [N/32], 16-byte aligned: block arrival counters.
+ *         They must be zero before the first call; every call that completes
+ *         leaves them zero (a call that timed out may not: zero them again).
+ *         Calls that overlap on the GPU need their own counters.
+ * The block of 32 outputs is quantised by whichever CTA stores its last
+ * output.  Requires N % 32 == 0.  For K outside the register schedule (K =
+ * 1024 * T, T in {4,5,6,8,10,12,15,16,20,25}) the call runs nvq_gemv and
+ * then the quantiser (two launches, same results).
+ * Errors: as nvq_gemv; NVQ_ERR_BAD_SHAPE when N % 32 != 0.
+ */
+nvq_status nvq_gemv_requant(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                            int64_t K, const int8_t* q, const uint16_t* d, float* y,
+                            int8_t* q_out, uint16_t* d_out, int32_t* counters, void* stream);
+
+/* One NVFP4 weight matrix W[N, K] in device memory (caller-owned). */
+typedef struct nvq_linear {
+  const uint8_t* codes;   /* device uint8 [N, K/2]  */
+  const uint8_t* scales;  /* device uint8 [N, K/16] */
+  float g;                /* per-tensor scale       */
+  int64_t N;
+  int64_t K;
+} nvq_linear;
+
+/*
+ * nvq_gemv_grouped - nvq_gemv of several weight matrices with the same K
+ * against the same Q8_0 activations (the q, k and v projections of a layer;
+ * up and gate), ys[i][M, N_i] = A . W_i^T.
+ *
+ * linears  host array of `count` descriptors (read during the call).
+ * ys       host array of `count` device float pointers.
+ * For one token the matrices share launches of the register schedule, up to
+ * three per launch with their rows concatenated, so the row ranges of the
+ * SMs stay balanced over the group; other M run one nvq_gemv per matrix.
+ * Results are those of nvq_gemv on each matrix.
+ * Errors: as nvq_gemv; NVQ_ERR_BAD_SHAPE when the K differ.
+ */
+nvq_status nvq_gemv_grouped(const nvq_linear* linears, int64_t count, const int8_t* q,
+                            const uint16_t* d, int64_t M, float* const* ys, void* stream);
+
+/*
  * nvq_gemm_workspace_size - bytes of device workspace nvq_gemm needs for
  * M tokens of K features (0 when M == 0).  It holds the activations
  * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q.
@@ -142,8 +193,9 @@ nvq_status nvq_gemv(const uint8_t* codes, const uint8_t* scales, float g,
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
- * nvq_gemm - prefill GEMM, y[M, N] = A[M, K] . W[N, K]^T for any M >= 1
- * (tuned for M >= 256) on the tcgen05 tensor cores.
+ * nvq_gemm - y[M, N] = A[M, K] . W[N, K]^T for any M >= 1 on the tcgen05
+ * tensor cores: the prefill GEMM, and for M <= 16 with K % 256 == 0 a
+ * small-token schedule (the small-batch decode of several sequences).
  *
  * The activations are expanded once into `workspace` as fp16 pairs
  * hi = fp16(d*q), lo = fp16(d*q - hi), exact (hi + lo == d*q).  Weight tiles
@@ -252,15 +304,6 @@ nvq_status nvq_error_flags(unsigned int* flags, int clear);
  * NVQ_ERR_MISALIGNED, NVQ_ERR_UNSUPPORTED_DEVICE, NVQ_ERR_CUDA.
  */
 nvq_status nvq_debug_stalled_wait(uint64_t limit_ns, int* result, void* stream);
-
-/* One NVFP4 weight matrix W[N, K] in device memory (caller-owned). */
-typedef struct nvq_linear {
-  const uint8_t* codes;   /* device uint8 [N, K/2]  */
-  const uint8_t* scales;  /* device uint8 [N, K/16] */
-  float g;                /* per-tensor scale       */
-  int64_t N;
-  int64_t K;
-} nvq_linear;
 
 /* Linears per decoder layer, in execution order. */
 #define NVQ_STACK_LINEARS 7

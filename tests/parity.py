@@ -9,6 +9,8 @@ codes are compared bit for bit before any output is compared.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -67,6 +69,11 @@ def reference(P: Packed, q_ref, d_ref):
     return y, sa, isum
 
 
+#: (test id, max err/tol) of every tolerance comparison in this session,
+#: summarised at the end of the run (tests/conftest.py)
+MARGINS: list[tuple[str, float]] = []
+
+
 def assert_within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, sa: np.ndarray):
     """|y_gpu - y_ref| <= 1e-5 * sum|terms| + 1e-6 per element, plus the
     false-pass guard: the reference is not identically zero."""
@@ -81,7 +88,10 @@ def assert_within_tolerance(y_gpu: np.ndarray, y_ref: np.ndarray, sa: np.ndarray
         raise AssertionError(
             f"{bad.sum()} of {bad.size} outside tolerance; first at {tuple(i)}: "
             f"gpu={y_gpu[tuple(i)]!r} ref={y_ref[tuple(i)]!r} tol={tol[tuple(i)]!r}")
-    return float((err / np.maximum(tol, 1e-300)).max())
+    ratio = float((err / np.maximum(tol, 1e-300)).max())
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    MARGINS.append((test, ratio))
+    return ratio
 
 
 # ---------------------------------------------------------------------------

@@ -92,6 +92,23 @@ def test_host_validation_status_codes():
     assert sums(codes, scales, 1.0, 8, 64, q, d, 1, y, p(off=4), None) == capi.NVQ_ERR_MISALIGNED
     assert sums(None, None, 1.0, 8, 64, None, None, 0, None, None, None) == capi.NVQ_OK
 
+    rq = lib.nvq_gemv_requant
+    qo, do, cnt = p(), p(), p()
+    assert rq(codes, scales, 1.0, 48, 64, q, d, y, qo, do, cnt, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert rq(codes, scales, 1.0, 64, 64, q, d, y, qo, do, None, None) == capi.NVQ_ERR_INVALID_ARG
+    assert rq(codes, scales, 1.0, 64, 64, q, d, y, p(off=2), do, cnt, None) == capi.NVQ_ERR_MISALIGNED
+    assert rq(codes, scales, 1.0, 64, 96, q, d, y, qo, do, cnt, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert rq(codes, scales, 1.0, 0, 64, q, d, y, None, None, None, None) == capi.NVQ_OK
+
+    grouped = lib.nvq_gemv_grouped
+    arr = (capi.Linear * 2)(capi.Linear(codes, scales, 1.0, 8, 64),
+                            capi.Linear(codes, scales, 1.0, 8, 128))
+    ys = (ctypes.c_void_p * 2)(y, y)
+    assert grouped(arr, 2, q, d, 1, ys, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert grouped(arr, 1, q, d, 17, ys, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert grouped(arr, 0, None, None, 1, None, None) == capi.NVQ_OK
+    assert grouped(None, 2, q, d, 1, ys, None) == capi.NVQ_ERR_INVALID_ARG
+
     flags = lib.nvq_error_flags
     assert flags(None, 0) == capi.NVQ_ERR_INVALID_ARG
     stalled = lib.nvq_debug_stalled_wait
