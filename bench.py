@@ -16,7 +16,8 @@ workload under ``"workloads"``, each measured the same way):
                           (5120, 152064).  Metric: weight GB/s (NVFP4 weight
                           bytes N*K*0.5625 streamed per second).
   gemv_4096               M=1, K=N=4096.
-  small_batch_m{2,4,8,16} M tokens, (5120, 25600), (25600, 5120).
+  small_batch_m{2,4,8,16} M tokens, (5120, 25600), (25600, 5120), through
+                          nvq_gemm (its small-token tensor-core schedule).
   prefill_m{256,2048}     Q8_0 + tcgen05 GEMM over (5120, 5120), (5120, 25600),
                           (25600, 5120).  Metric: algorithmic TFLOP/s 2*M*N*K.
   stack_decode            all 448 linears of a 64-layer dense decoder (17.9 GB
@@ -468,6 +469,33 @@ class GemvWorkload:
                 "quantisation + fp64 dequantise-then-dot")
 
 
+class SmallGemmWorkload(GemvWorkload):
+    """Small-batch decode: Q8_0 of M <= 16 tokens and nvq_gemm, which runs
+    the small-token tensor-core schedule; metric as the GEMV (weight GB/s)."""
+
+    kernel = "gemm_small"
+    sources = ("gemm_small.cu", "gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+
+    def setup(self, device):
+        import torch
+        super().setup(device)
+        for c in self.cases:
+            c["ws"] = torch.empty(self.capi.gemm_workspace_size(self.M, c["N"], c["K"]),
+                                  dtype=torch.uint8, device=device)
+
+    def config(self):
+        cfg = super().config()
+        cfg["path"] = "nvq_gemm small-token tcgen05 schedule"
+        return cfg
+
+    def launches_per_step(self):
+        # quantise, expand, tcgen05 kernel, and the fixed-order sum of split tiles
+        return 4 * len(self.cases)
+
+    def dominant(self, c, codes, scales, stream):
+        self.capi.gemm(codes, scales, c["g"], c["q"], c["d"], c["y"], c["ws"], stream=stream)
+
+
 class GemmWorkload(GemvWorkload):
     """Prefill: Q8_0 of M tokens and the tcgen05 GEMM for each shape."""
 
@@ -632,7 +660,7 @@ def make_workload(name: str):
                                              wl.activations("gemv_4096", "x", 1, K)))
     if name.startswith("small_batch_m"):
         M = int(name[len("small_batch_m"):])
-        return GemvWorkload(
+        return SmallGemmWorkload(
             name, wl.SMALL_BATCH_SHAPES, M, lambda K, N: wl.small_batch_case(M, K, N),
             lambda K, N, r: (wl.weight_rows("small_batch", "W", N, K, r, True),
                              wl.activations("small_batch", "x", M, K, "student_t4")))

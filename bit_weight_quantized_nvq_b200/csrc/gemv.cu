@@ -386,14 +386,29 @@ __device__ __forceinline__ void requant_block_thread(const RegMat& m, int b) {
   }
   m.rq_d[b] = __float2half_rn(d32);
 }
-// Row `row` of m has been stored (by this thread): count it in its block and
-// report whether this thread completed the block (classic fence + counter
-// protocol: the store is visible device-wide before the count).
-__device__ __forceinline__ bool arrive_row(const RegMat& m, int row) {
+// Row `row` of m (concatenated row `grow`) has been stored by this thread.
+// Returns 0, or the way its 32-row block became complete: 1 = every row of
+// the block belongs to this CTA and this was the last of them; 2 = the block
+// is shared with a neighbouring CTA and this CTA's rows arrived last.  Rows
+// are first counted per CTA in shared memory (a CTA-scope fence before the
+// count makes the store visible to the warp that completes the block); only
+// a CTA's share of a block that straddles two CTAs goes through the global
+// counter (device-scope fence, one atomic per CTA and block).
+__device__ __forceinline__ int arrive_row(const RegMat& m, int row, int grow, int r_begin,
+                                          int r_end, int* scnt) {
+  const int bstart = grow & ~31;
+  const int mine = min(r_end, bstart + 32) - max(r_begin, bstart);
+  __threadfence_block();
+  if (atomicAdd(scnt + ((grow >> 5) - (r_begin >> 5)), 1) + 1 != mine) return 0;
+  if (mine == 32) return 1;
   __threadfence();
-  const bool last = atomicAdd(m.rq_cnt + (row >> 5), 1) == 31;
-  if (last) __threadfence();
-  return last;
+  return atomicAdd(m.rq_cnt + (row >> 5), mine) + mine == 32 ? 2 : 0;
+}
+
+// Shared-memory block counters a CTA needs: its row range covers at most
+// ceil(rows / G) rows, i.e. this many 32-row blocks.
+__host__ __device__ __forceinline__ int reg_block_slots(int rows, int G) {
+  return (rows + G - 1) / G / 32 + 2;
 }
 
 // The next stage of a CTA's concatenated row range: at most R rows, all of
@@ -421,6 +436,7 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
   uint64_t* full = reinterpret_cast<uint64_t*>(part + kM1Stages * kM1Consumers);
   uint64_t* empty = full + kM1Stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kM1Stages);
+  int* scnt = reinterpret_cast<int*>(empty + kM1Stages + 2);   // block counters of this CTA
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -429,6 +445,7 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
   const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * grp.rows / G);
 
   grid_dependents_launch();
+  for (int i = threadIdx.x; i < reg_block_slots(grp.rows, G); i += blockDim.x) scnt[i] = 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kM1Stages; ++i) {
       ptx::mbar_init(ptx::smem_addr(full + i), 1);
@@ -454,9 +471,13 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
         for (int p = 0; p < WPR; ++p) v += part[s * kM1Consumers + r * WPR + p];
         const int row = srow[s] + r;
         m.y[row] = v * m.half_g;
-        if (m.rq_q != nullptr && arrive_row(m, row)) {
-          requant_block_thread(m, row >> 5);
-          atomicExch(m.rq_cnt + (row >> 5), 0);
+        if (m.rq_q != nullptr) {
+          const int how = arrive_row(m, row, m.row_off + row, r_begin, r_end, scnt);
+          if (how != 0) {
+            if (how == 1) __threadfence_block(); else __threadfence();
+            requant_block_thread(m, row >> 5);
+            if (how == 2) atomicExch(m.rq_cnt + (row >> 5), 0);
+          }
         }
       }
     };
@@ -566,14 +587,18 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
       acc = dev::warp_sum(acc);
       if (WPR == 1) {
         const int row = row0 + rl;
-        bool last = false;
+        int how = 0;
         if (lane == 0) {
           m.y[row] = acc * m.half_g;
-          if (m.rq_q != nullptr) last = arrive_row(m, row);
+          if (m.rq_q != nullptr) how = arrive_row(m, row, m.row_off + row, r_begin, r_end, scnt);
         }
-        if (m.rq_q != nullptr && __shfl_sync(0xffffffffu, last, 0)) {
-          requant_block_warp(m, row >> 5, lane);
-          if (lane == 0) atomicExch(m.rq_cnt + (row >> 5), 0);
+        if (m.rq_q != nullptr) {
+          how = __shfl_sync(0xffffffffu, how, 0);
+          if (how != 0) {
+            if (how == 1) __threadfence_block(); else __threadfence();
+            requant_block_warp(m, row >> 5, lane);
+            if (how == 2 && lane == 0) atomicExch(m.rq_cnt + (row >> 5), 0);
+          }
         }
       } else if (lane == 0) {
         part[s * kM1Consumers + warp] = acc;
@@ -823,10 +848,13 @@ cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const
   cudaError_t e = attr.ensure(kernel, static_cast<int>(kSmemPerCtaMax));
   if (e != cudaSuccess) return e;
   const int64_t ctas = std::min<int64_t>(device_sm_count(), grp.rows);
+  const uint32_t smem = reg_smem_bytes(static_cast<int>(K), WPR) +
+                        4u * reg_block_slots(grp.rows, static_cast<int>(ctas));
+  if (smem > kSmemPerCtaMax) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kM1Threads);
-  cfg.dynamicSmemBytes = reg_smem_bytes(static_cast<int>(K), WPR);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -963,7 +991,15 @@ cudaError_t launch_gemv_group(const GemvTarget* t, int n, int64_t K, const int8_
     if (reg_supported(K)) {
       RegGroup grp = {};
       int rows = 0;
-      const int cnt = std::min(kMaxGroup, n - done);
+      // a requantised matrix must start on a 32-row block of the
+      // concatenated rows (its blocks are counted there)
+      int cnt = 0;
+      while (cnt < kMaxGroup && done + cnt < n &&
+             (t[done + cnt].rq_q == nullptr || rows % 32 == 0)) {
+        rows += static_cast<int>(t[done + cnt].N);
+        ++cnt;
+      }
+      rows = 0;
       for (int i = 0; i < cnt; ++i) {
         const GemvTarget& x = t[done + i];
         RegMat m = reg_mat(x.codes, x.scales, x.g, x.N, x.y);

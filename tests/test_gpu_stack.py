@@ -82,6 +82,33 @@ def test_small_stack_last_layer_matches_oracle_chain(M):
         assert np.any(y_ref != 0)
 
 
+def test_one_token_stack_with_grouped_requantising_launches():
+    """One token through shapes that the register schedule covers (K = 4096
+    for q/k/v/o/up/gate, 8192 for down): q, k, v in one launch that also
+    emits Q8_0(y_v), o emitting Q8_0(y_o), up and gate in one launch emitting
+    Q8_0(y_up), down alone; every output of the last layer against the
+    oracle chain, and a second pass gives identical outputs (the block
+    counters are left at zero)."""
+    h, f = 4096, 8192
+    stack, packed = build_stack(2, h, f, 1, "grouped")
+    x = wl.activations("stack_test", "xg", 1, h, "student_t4")
+    xd = torch.from_numpy(x).cuda()
+    outs = [t.clone() for t in stack.forward(xd)]
+    torch.cuda.synchronize()
+    ref = oracle_chain(packed, x)
+    for i, name in enumerate(ORDER):
+        y = outs[i].cpu().numpy().astype(np.float64)
+        y_ref, tol = ref[name]
+        err = np.abs(y - y_ref)
+        assert np.all(err <= tol), (name, float((err / tol).max()))
+        assert np.any(y_ref != 0)
+    outs2 = stack.forward(xd)
+    torch.cuda.synchronize()
+    for a, b in zip(outs, outs2):
+        assert torch.equal(a, b)
+    assert capi.error_flags() == 0
+
+
 def test_stack_validates_shapes_and_workspace():
     h, f = 256, 512
     stack, _ = build_stack(1, h, f, 2, "val")
