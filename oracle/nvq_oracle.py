@@ -27,6 +27,9 @@ What it computes, and the passages it follows
            * product: per 16-subblock y += g*s_w*d_a*0.5*sum(c_w*q_a) with the
              integer LUT value c_w = 2*E2M1 in -12..12;
            * accuracy: |y - y_ref| <= 1e-5*sum|terms| + 1e-6 per element.
+[ROOF]     "Roofline-First Decoding: results": a fused 4-bit dequantise-plus-
+           GEMV for batch-1 decoding on fp16 activations (W4A16); here the
+           4-bit weights are NVFP4 and the activations binary16 values.
 [OCP-MX]   OCP Microscaling Formats (MX) v1.0: the E2M1 element type (1 sign,
            2 exponent bits with bias 1, 1 mantissa bit; max 6) and the E4M3
            type (4 exponent bits with bias 7, 3 mantissa bits, max 448, S.1111.111
@@ -65,6 +68,7 @@ __all__ = [
     "unpack_codes", "dequantize_weights", "dequantize_activations",
     "dot_fp64", "subblock_sums", "subblock_sums_biased", "bsum16",
     "y_from_subblock_sums", "sum_abs_terms", "tolerance",
+    "dot_fp64_f16", "sum_abs_terms_f16",
     "ACC_REL_TOL", "ACC_ABS_TOL",
 ]
 
@@ -394,3 +398,44 @@ def sum_abs_terms(isum, scales, g, d) -> np.ndarray:
 def tolerance(sum_abs) -> np.ndarray:
     """Per-element bound 1e-5 * sum|terms| + 1e-6 on |y_fp32 - y_ref|."""
     return ACC_REL_TOL * np.asarray(sum_abs, dtype=np.float64) + ACC_ABS_TOL
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 weights x fp16 activations (W4A16) [ROOF]
+# ---------------------------------------------------------------------------
+
+def dot_fp64_f16(codes, scales, g, x_bits, row_chunk: int = 4096) -> np.ndarray:
+    """y[m, n] = sum_k w[n, k] * fp16(x_bits[m, k]) in fp64, fp64 [M, N].
+
+    The plain definition for fp16 activations: dequantise the weights and
+    decode the binary16 activations (both exact in fp64), then take their
+    dot product (a library matrix product).
+    Pinned by tests/test_oracle_w4a16.py (exact rational brute force, the
+    reduction to dot_fp64 when every activation is a Q8_0 value).
+    """
+    a = fp16_values()[np.asarray(x_bits, dtype=np.uint16)]
+    N = np.asarray(codes).shape[0]
+    y = np.empty((a.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, row_chunk):
+        n1 = min(N, n0 + row_chunk)
+        w = dequantize_weights(codes[n0:n1], scales[n0:n1], g)
+        y[:, n0:n1] = a @ w.T
+    return y
+
+
+def sum_abs_terms_f16(codes, scales, g, x_bits, row_chunk: int = 1024) -> np.ndarray:
+    """sum|terms|[m, n] = sum over 16-element subblocks sb of
+    |sum_{k in sb} w[n, k] * x[m, k]|, fp64 [M, N]: the per-element scale of
+    the accuracy bound for fp16 activations (the subblock partial sums play
+    the part of the Q8_0 path's per-subblock terms)."""
+    a = fp16_values()[np.asarray(x_bits, dtype=np.uint16)]
+    M, K = a.shape
+    N = np.asarray(codes).shape[0]
+    out = np.empty((M, N), dtype=np.float64)
+    for n0 in range(0, N, row_chunk):
+        n1 = min(N, n0 + row_chunk)
+        w = dequantize_weights(codes[n0:n1], scales[n0:n1], g)
+        part = np.einsum("nsj,msj->mns", w.reshape(n1 - n0, K // 16, 16),
+                         a.reshape(M, K // 16, 16))
+        out[:, n0:n1] = np.abs(part).sum(axis=2)
+    return out
