@@ -314,8 +314,10 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
 // it recycles the stage, so results are deterministic.
 // The kernel is launched with programmatic stream serialisation: it lets
 // the next kernel of the stream launch early and waits for the previous
-// one (griddepcontrol) before it reads any global input, so launch latency
-// and prologue overlap the previous kernel's tail without changing results.
+// one (griddepcontrol) before it reads the activations or writes anything,
+// so launch latency, prologue and the first weight copies (the weights are
+// never written by the kernels before it) overlap the previous kernel's tail
+// without changing results.
 constexpr uint32_t kRegStageMax = 46080;
 constexpr int kMaxGroup = 3;       // matrices per register-schedule launch
 
@@ -455,11 +457,14 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
     ptx::fence_mbar_init();
   }
   __syncthreads();
-  grid_dependency_wait();   // inputs written by the previous kernel are visible
 
   if (warp == kM1Consumers) {
     // ------------- producer: bulk copies, and the sum of row partials --------
+    // The weights are not written by the kernels before this one, so the
+    // first ring stages are requested before waiting for them; everything
+    // the producer writes (row sums, requantisation) comes after the wait.
     if (lane != 0) return;
+    bool waited = false;
     int smi[kM1Stages] = {}, srow[kM1Stages] = {}, snr[kM1Stages] = {};   // stages in flight
     auto finalize = [&](int it) {   // rows of stage `it`, once its slot is empty
       if (WPR == 1) return;
@@ -487,6 +492,10 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
     for (int it = 0; gr < r_end; ++it) {
       const int s = it % kM1Stages;
       const uint32_t ph = (it / kM1Stages) & 1;
+      if (it == kM1Stages) {
+        grid_dependency_wait();
+        waited = true;
+      }
       if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
         *abort_flag = 1;
         raise_timeout();
@@ -509,6 +518,7 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
                      m.scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
       ++issued;
     }
+    if (!waited) grid_dependency_wait();
     if (ok) {
       // the last stages: wait until consumed, then add their partials
       for (int it = max(0, issued - kM1Stages); it < issued; ++it) {
@@ -530,6 +540,7 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
 
   // ------------- consumers: warp w = (row w / WPR, part w % WPR) -------------
   if (warp >= active) return;
+  grid_dependency_wait();   // the activations (and y's readers) of the previous kernel
   const int rl = warp / WPR;
   const int p = warp % WPR;
   uint4 qa[NPL], qb[NPL];
