@@ -90,6 +90,19 @@ __host__ __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t W, int
   return c * W / G;
 }
 
+// Slot and phase of a ring of `depth` stages, advanced one stage at a time.
+struct Ring {
+  int depth;
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void advance() {
+    if (++slot == depth) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 // Iterates the (tile, stage range) pieces of a CTA's unit range.
 struct Pieces {
   int64_t u, u_end, Ks;
@@ -117,7 +130,7 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 }
 
 template <int NT>   // MMA N = 2 * padded tokens (16 or 32)
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(112)   // 18 warps x 112 registers fill the register file
 gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
                   const __grid_constant__ CUtensorMap scale_map,
                   const __grid_constant__ CUtensorMap act_map, int N, int K, int M,
@@ -194,46 +207,49 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
     // ------------------------------ TMA producer -------------------------------
     Pieces pc{u0, u1, Ks};
     int t, j0, j1;
-    int64_t i = 0;
+    Ring sm{kSmemStages};
+    int issued = 0;
     bool ok = true;
     while (ok && pc.next(t, j0, j1)) {
-      for (int j = j0; j < j1; ++j, ++i) {
-        const int s = static_cast<int>(i % kSmemStages);
-        if (!warp_wait(empty(s), static_cast<uint32_t>(((i / kSmemStages) & 1) ^ 1))) {
+      for (int j = j0; j < j1; ++j, sm.advance()) {
+        if (!warp_wait(empty(sm.slot), sm.phase ^ 1u)) {
           fail();
           ok = false;
           break;
         }
         if (lane == 0) {
-          const uint32_t dst = slot_addr(s);
-          ptx::mbar_arrive_expect_tx(full(s), slot_bytes(NT));
-          ptx::tma_load_2d(dst, &code_map, j * (kStageK / 2), t * kRows, full(s));
+          const uint32_t dst = slot_addr(sm.slot);
+          const uint32_t bar = full(sm.slot);
+          ptx::mbar_arrive_expect_tx(bar, slot_bytes(NT));
+          ptx::tma_load_2d(dst, &code_map, j * (kStageK / 2), t * kRows, bar);
+#pragma unroll
           for (int sub = 0; sub < kSubs; ++sub)
             ptx::tma_load_2d(dst + kCodeBytes + sub * act_sub_bytes(NT), &act_map,
-                             j * kStageK + sub * kSubK, 0, full(s));
+                             j * kStageK + sub * kSubK, 0, bar);
           ptx::tma_load_2d(dst + kCodeBytes + kSubs * act_sub_bytes(NT), &scale_map,
-                           j * (kStageK / 16), t * kRows, full(s));
+                           j * (kStageK / 16), t * kRows, bar);
         }
         __syncwarp();
+        ++issued;
       }
     }
     if (!ok) {
       // let this CTA's copies in flight land before it can leave
-      for (int64_t k = std::max<int64_t>(0, i - kSmemStages); k < i; ++k)
-        ptx::mbar_wait_bounded(full(static_cast<int>(k % kSmemStages)),
-                               static_cast<uint32_t>((k / kSmemStages) & 1), nullptr,
-                               kWaitLimitNs);
+      for (int k = max(0, issued - kSmemStages); k < issued; ++k)
+        ptx::mbar_wait_bounded(full(k % kSmemStages), static_cast<uint32_t>((k / kSmemStages) & 1),
+                               nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------- MMA issuer --------------------------------
     constexpr uint32_t idesc = ptx::idesc_f16_f32(kRows, NT);
     Pieces pc{u0, u1, Ks};
     int t, j0, j1;
-    int64_t i = 0, ch = 0;
+    Ring sm{kSmemStages}, ar{kAStages};
+    int ch = 0;
     bool ok = true;
     while (ok && pc.next(t, j0, j1)) {
       for (int jc = j0; jc < j1 && ok; jc += kChunkStages, ++ch) {
-        const int b = static_cast<int>(ch & 1);
+        const int b = ch & 1;
         if (ch >= 2 && !warp_wait(acc_empty(b), static_cast<uint32_t>(((ch >> 1) - 1) & 1))) {
           fail();
           ok = false;
@@ -241,19 +257,16 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
         }
         const uint32_t d_tmem = tmem_base + kAccCol0 + b * NT;
         const int je = min(j1, jc + kChunkStages);
-        for (int j = jc; j < je; ++j, ++i) {
-          const int s = static_cast<int>(i % kSmemStages);
-          const int as = static_cast<int>(i % kAStages);
-          if (!warp_wait(full(s), static_cast<uint32_t>((i / kSmemStages) & 1)) ||
-              !warp_wait(a_full(as), static_cast<uint32_t>((i / kAStages) & 1))) {
+        for (int j = jc; j < je; ++j, sm.advance(), ar.advance()) {
+          if (!warp_wait(full(sm.slot), sm.phase) || !warp_wait(a_full(ar.slot), ar.phase)) {
             fail();
             ok = false;
             break;
           }
           if (lane == 0) {
             ptx::tc_fence_after();
-            const uint32_t a_cols = tmem_base + as * kACols;
-            const uint64_t bdesc0 = ptx::sw128_kmajor_desc(slot_addr(s) + kCodeBytes);
+            const uint32_t a_cols = tmem_base + ar.slot * kACols;
+            const uint64_t bdesc0 = ptx::sw128_kmajor_desc(slot_addr(sm.slot) + kCodeBytes);
 #pragma unroll
             for (int sub = 0; sub < kSubs; ++sub) {
 #pragma unroll
@@ -263,8 +276,8 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
                 ptx::mma_f16_ts(d_tmem, a, bd, idesc, (j == jc && sub == 0 && k == 0) ? 0u : 1u);
               }
             }
-            ptx::mma_commit(empty(s));
-            ptx::mma_commit(a_empty(as));
+            ptx::mma_commit(empty(sm.slot));
+            ptx::mma_commit(a_empty(ar.slot));
             if (j == je - 1) ptx::mma_commit(acc_full(b));
           }
           __syncwarp();
@@ -282,18 +295,23 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
     const int r = q * 32 + lane;            // tile row = TMEM lane
     const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
     const bool drainer = p == 0;
+    const uint32_t row_off = r * 128u;
+    const uint32_t sw = static_cast<uint32_t>(r & 7);
+    const uint32_t c0_off = row_off + ((2u * p) ^ sw) * 16u;
+    const uint32_t c1_off = row_off + ((2u * p + 1u) ^ sw) * 16u;
+    const uint32_t s_off = kCodeBytes + kSubs * act_sub_bytes(NT) + r * 16u + 4u * p;
     float run[NT];
 #pragma unroll
     for (int n = 0; n < NT; ++n) run[n] = 0.0f;
 
     // drain cursor: walks the same pieces and chunks as the MMA issuer
     Pieces dpc{u0, u1, Ks};
-    int dt = 0, dj0 = 0, dj1 = 0, djc = 0;
+    int dt = 0, dj0 = 0, dj1 = 0;
     bool dvalid = dpc.next(dt, dj0, dj1);
-    djc = dj0;
-    int64_t drained = 0;
+    int djc = dj0;
+    int drained = 0;
     auto drain_one = [&]() -> bool {
-      const int b = static_cast<int>(drained & 1);
+      const int b = drained & 1;
       if (!warp_wait(acc_full(b), static_cast<uint32_t>((drained >> 1) & 1))) return false;
       ptx::tc_fence_after();
       uint32_t v[NT];
@@ -334,35 +352,47 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
 
     Pieces pc{u0, u1, Ks};
     int t, j0, j1;
-    int64_t i = 0, ch = 0;
+    Ring sm{kSmemStages}, ar{kAStages};
+    int ch = 0;
+    int prev_slot = -1;                      // A stage stored but not yet announced
     bool ok = true;
+    // The store of a stage is waited for (and the stage announced to the MMA
+    // issuer) only after the next stage is decoded, so the tensor-memory
+    // store latency overlaps the decode instead of stalling the warp.
+    auto announce_prev = [&]() {
+      if (prev_slot >= 0) {
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(a_full(prev_slot));
+        prev_slot = -1;
+      }
+    };
     while (ok && pc.next(t, j0, j1)) {
-      for (int j = j0; j < j1; ++j, ++i) {
-        const bool chunk_start = ((j - j0) % kChunkStages) == 0;
-        if (chunk_start) {
+      int in_chunk = 0;
+      for (int j = j0; j < j1; ++j, sm.advance(), ar.advance()) {
+        if (in_chunk == 0) {
           // before the chunk that reuses a buffer, drain the chunk that used it
-          if (drainer && ch >= 2 && !drain_one()) {
-            fail();
-            ok = false;
-            break;
+          if (drainer && ch >= 2) {
+            announce_prev();
+            if (!drain_one()) {
+              fail();
+              ok = false;
+              break;
+            }
           }
           ++ch;
         }
-        const int s = static_cast<int>(i % kSmemStages);
-        const int as = static_cast<int>(i % kAStages);
-        if (!warp_wait(full(s), static_cast<uint32_t>((i / kSmemStages) & 1)) ||
-            !warp_wait(a_empty(as), static_cast<uint32_t>(((i / kAStages) & 1) ^ 1))) {
+        in_chunk = in_chunk + 1 == kChunkStages ? 0 : in_chunk + 1;
+        if (!warp_wait(full(sm.slot), sm.phase)) {
           fail();
           ok = false;
           break;
         }
-        ptx::tc_fence_after();
-        const uint32_t slot = slot_addr(s);
-        const uint32_t line = slot + r * 128u;
-        const uint32_t sw = static_cast<uint32_t>(r & 7);
-        const uint4 c0 = lds128(line + ((2u * p) ^ sw) * 16u);
-        const uint4 c1 = lds128(line + ((2u * p + 1u) ^ sw) * 16u);
-        const uint32_t sc = lds32(slot + kCodeBytes + kSubs * act_sub_bytes(NT) + r * 16u + 4u * p);
+        const uint32_t slot = slot_addr(sm.slot);
+        const uint4 c0 = lds128(slot + c0_off);
+        const uint4 c1 = lds128(slot + c1_off);
+        const uint32_t sc = lds32(slot + s_off);
         const __half2 sp01 = dev::ue4m3x2_to_half2(sc & 0xFFFFu);
         const __half2 sp23 = dev::ue4m3x2_to_half2(sc >> 16);
         const __half2 s0 = __low2half2(sp01), s1 = __high2half2(sp01);
@@ -375,13 +405,18 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
                                 e2.x, e2.y, e2.z, e2.w, e3.x, e3.y, e3.z, e3.w,
                                 e4.x, e4.y, e4.z, e4.w, e5.x, e5.y, e5.z, e5.w,
                                 e6.x, e6.y, e6.z, e6.w, e7.x, e7.y, e7.z, e7.w};
-        ptx::tmem_st_32cols(tmem_base + tlane + as * kACols + p * 32u, v);
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(a_full(as));
+        announce_prev();
+        if (!warp_wait(a_empty(ar.slot), ar.phase ^ 1u)) {
+          fail();
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        ptx::tmem_st_32cols(tmem_base + tlane + ar.slot * kACols + p * 32u, v);
+        prev_slot = ar.slot;
       }
     }
+    if (ok) announce_prev();
     // the chunks not drained yet
     while (ok && drainer && dvalid) {
       if (!drain_one()) {
