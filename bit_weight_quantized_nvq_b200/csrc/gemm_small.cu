@@ -130,7 +130,7 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 }
 
 template <int NT>   // MMA N = 2 * padded tokens (16 or 32)
-__global__ void __maxnreg__(112)   // 18 warps x 112 registers fill the register file
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
                   const __grid_constant__ CUtensorMap scale_map,
                   const __grid_constant__ CUtensorMap act_map, int N, int K, int M,
