@@ -163,6 +163,7 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
   const int64_t u0 = unit_begin(c, W, G), u1 = unit_begin(c + 1, W, G);
   const int t_first = static_cast<int>(u0 / Ks);
 
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSmemStages; ++s) {
       ptx::mbar_init(full(s), 1);
@@ -205,6 +206,40 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
 
   if (warp == 0) {
     // ------------------------------ TMA producer -------------------------------
+    // The weights are never written by the kernels before this one, so the
+    // codes and scales of the first ring slots are requested before waiting
+    // for the previous kernel (the activation expansion); the activations of
+    // those slots follow the wait.
+    auto load_weights = [&](uint32_t dst, uint32_t bar, int t, int j) {
+      ptx::tma_load_2d(dst, &code_map, j * (kStageK / 2), t * kRows, bar);
+      ptx::tma_load_2d(dst + kCodeBytes + kSubs * act_sub_bytes(NT), &scale_map,
+                       j * (kStageK / 16), t * kRows, bar);
+    };
+    auto load_acts = [&](uint32_t dst, uint32_t bar, int j) {
+#pragma unroll
+      for (int sub = 0; sub < kSubs; ++sub)
+        ptx::tma_load_2d(dst + kCodeBytes + sub * act_sub_bytes(NT), &act_map,
+                         j * kStageK + sub * kSubK, 0, bar);
+    };
+    int early_j[kSmemStages];
+    int early = 0;
+    {
+      Pieces pc{u0, u1, Ks};
+      int t, j0, j1;
+      while (early < kSmemStages && pc.next(t, j0, j1)) {
+        for (int j = j0; j < j1 && early < kSmemStages; ++j, ++early) {
+          if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(full(early), slot_bytes(NT));
+            load_weights(slot_addr(early), full(early), t, j);
+          }
+          early_j[early] = j;
+        }
+      }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (lane == 0)
+      for (int e = 0; e < early; ++e) load_acts(slot_addr(e), full(e), early_j[e]);
+    __syncwarp();
     Pieces pc{u0, u1, Ks};
     int t, j0, j1;
     Ring sm{kSmemStages};
@@ -212,6 +247,10 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
     bool ok = true;
     while (ok && pc.next(t, j0, j1)) {
       for (int j = j0; j < j1; ++j, sm.advance()) {
+        if (issued < early) {   // requested above
+          ++issued;
+          continue;
+        }
         if (!warp_wait(empty(sm.slot), sm.phase ^ 1u)) {
           fail();
           ok = false;
@@ -221,13 +260,8 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
           const uint32_t dst = slot_addr(sm.slot);
           const uint32_t bar = full(sm.slot);
           ptx::mbar_arrive_expect_tx(bar, slot_bytes(NT));
-          ptx::tma_load_2d(dst, &code_map, j * (kStageK / 2), t * kRows, bar);
-#pragma unroll
-          for (int sub = 0; sub < kSubs; ++sub)
-            ptx::tma_load_2d(dst + kCodeBytes + sub * act_sub_bytes(NT), &act_map,
-                             j * kStageK + sub * kSubK, 0, bar);
-          ptx::tma_load_2d(dst + kCodeBytes + kSubs * act_sub_bytes(NT), &scale_map,
-                           j * (kStageK / 16), t * kRows, bar);
+          load_weights(dst, bar, t, j);
+          load_acts(dst, bar, j);
         }
         __syncwarp();
         ++issued;
@@ -295,6 +329,9 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
     const int r = q * 32 + lane;            // tile row = TMEM lane
     const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
     const bool drainer = p == 0;
+    // y, the partial sums and tok_scale are touched only after the previous
+    // kernels are complete
+    if (drainer) asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t row_off = r * 128u;
     const uint32_t sw = static_cast<uint32_t>(r & 7);
     const uint32_t c0_off = row_off + ((2u * p) ^ sw) * 16u;
@@ -538,11 +575,22 @@ cudaError_t launch_small(const uint8_t* codes, const uint8_t* scales, float g, i
                                         static_cast<int64_t>(kMaxCtas)});
   const float* tok = reinterpret_cast<const float*>(ws + L.tok);
   float* partial = reinterpret_cast<float*>(ws + L.partial);
-  gemm_small_kernel<NT><<<static_cast<unsigned>(G), kThreads, smem_bytes(NT), stream>>>(
-      code_map, scale_map, act_map, static_cast<int>(N), static_cast<int>(K),
-      static_cast<int>(M), g, tok, y, partial);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(G));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes(NT);
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemm_small_kernel<NT>, code_map, scale_map, act_map,
+                           static_cast<int>(N), static_cast<int>(K), static_cast<int>(M), g, tok,
+                           y, partial);
+    if (e != cudaSuccess) return e;
+  }
   // a tile is split between CTAs when a CTA's range starts inside it
   const int64_t Ks = K / kStageK;
   bool split = false;
@@ -552,9 +600,6 @@ cudaError_t launch_small(const uint8_t* codes, const uint8_t* scales, float g, i
   cfg.gridDim = dim3(static_cast<unsigned>(T));
   cfg.blockDim = dim3(kRows);
   cfg.stream = stream;
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, gemm_small_reduce_kernel<NT / 2>,

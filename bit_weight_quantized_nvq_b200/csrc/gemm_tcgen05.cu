@@ -119,6 +119,10 @@ using dev::ue4m3x2_to_half2;
 __global__ void __launch_bounds__(256)
 expand_act_kernel(const int8_t* __restrict__ q, const __half* __restrict__ d, int M, int K,
                   int M_pad, __half* __restrict__ act, float* __restrict__ tok_scale) {
+  // programmatic dependent launch: the next kernel may start its prologue
+  // (and its weight copies); q and d are read once the previous kernel is done
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x;
   uint4* hi = reinterpret_cast<uint4*>(act + static_cast<size_t>(row) * K);
   uint4* lo = reinterpret_cast<uint4*>(act + static_cast<size_t>(M_pad + row) * K);
@@ -603,10 +607,18 @@ cudaError_t gemm_error_flags(bool clear, unsigned int* flags) {
 
 cudaError_t expand_activations(const int8_t* q, const uint16_t* d, int64_t M, int64_t M_pad,
                                int64_t K, void* act, float* tok_scale, cudaStream_t stream) {
-  expand_act_kernel<<<static_cast<unsigned>(M_pad), 256, 0, stream>>>(
-      q, reinterpret_cast<const __half*>(d), static_cast<int>(M), static_cast<int>(K),
-      static_cast<int>(M_pad), static_cast<__half*>(act), tok_scale);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(M_pad));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, expand_act_kernel, q, reinterpret_cast<const __half*>(d),
+                            static_cast<int>(M), static_cast<int>(K), static_cast<int>(M_pad),
+                            static_cast<__half*>(act), tok_scale);
 }
 
 cudaError_t gemm_expand(const int8_t* q, const uint16_t* d, int64_t M, int64_t K,
