@@ -538,6 +538,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 int64_t padded_tokens(int64_t M) { return (M + kBT - 1) / kBT * kBT; }
 
+// token counts that nvq_gemm hands to the decode GEMV
+constexpr int64_t kGemvTokensMax = 4;
+
 // The scratch array's device address in the current context.  Host code may
 // not use the array's name as an address (it names a host-side shadow), so
 // the address is looked up with cudaGetSymbolAddress, with the device
@@ -677,6 +680,10 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
 cudaError_t launch_gemm(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
                         int64_t K, const int8_t* q, const uint16_t* d, int64_t M, float* y,
                         void* workspace, cudaStream_t stream) {
+  // up to four tokens the CUDA-core decode GEMV streams the weights faster
+  // (its integer dot costs little per token); beyond, the tensor-core
+  // small-token schedule, whose per-weight cost does not grow with M
+  if (M <= kGemvTokensMax) return launch_gemv(codes, scales, g, N, K, q, d, M, y, stream);
   if (gemm_small_supported(M, K))
     return launch_gemm_small(codes, scales, g, N, K, q, d, M, y, workspace, stream);
   cudaError_t e = gemm_expand(q, d, M, K, workspace, stream);

@@ -193,18 +193,30 @@ nvq_status nvq_gemv_grouped(const nvq_linear* linears, int64_t count, const int8
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
- * nvq_gemm - y[M, N] = A[M, K] . W[N, K]^T for any M >= 1 on the tcgen05
- * tensor cores: the prefill GEMM, and for M <= 16 with K % 256 == 0 a
- * small-token schedule (the small-batch decode of several sequences).
+ * nvq_gemm - y[M, N] = A[M, K] . W[N, K]^T for any M >= 1: the prefill GEMM
+ * on the tcgen05 tensor cores, and the small-batch decode of several
+ * sequences.  Three schedules, chosen by the call:
  *
- * The activations are expanded once into `workspace` as fp16 pairs
- * hi = fp16(d*q), lo = fp16(d*q - hi), exact (hi + lo == d*q).  Weight tiles
- * are expanded in tensor memory to fp16 w' = E2M1*s_w (exact) and every
- * 64-wide K slice is multiplied by tcgen05.mma (kind::f16, CTA pairs)
- * against hi and against lo, both accumulating in fp32 into one tensor-
- * memory accumulator per 512-wide K chunk whose partial sums are added in
- * fp32 registers; y = g * sum.  Every product is exact; only the fp32
- * accumulation rounds.
+ *  - M <= 4: the decode GEMV (nvq_gemv), which streams the weights faster
+ *    there (its integer dot costs little per token); the workspace is unused.
+ *  - 5 <= M <= 16 and K % 256 == 0: the small-token tensor-core schedule.
+ *    One CTA per SM; the (128-row tile, 256-wide K stage) units are split
+ *    into equal contiguous ranges (a tile two CTAs share is added from fp32
+ *    partials in the workspace, in a fixed order, by a second launch); 16
+ *    warps expand the weights into tensor memory; tcgen05.mma with N = 2 x
+ *    (tokens padded to 8 or 16) takes the exact hi/lo activations (below)
+ *    from shared memory; accumulators are promoted to fp32 registers every
+ *    1024 K.  Results are deterministic.
+ *  - otherwise: the prefill schedule on CTA pairs: weight tiles expanded in
+ *    tensor memory, every 64-wide K slice multiplied by tcgen05.mma
+ *    (kind::f16, cta_group::2) against hi and against lo into one fp32
+ *    tensor-memory accumulator per 512-wide K chunk, whose partial sums are
+ *    added in fp32 registers.
+ *
+ * The tensor-core schedules expand the activations once into `workspace` as
+ * fp16 pairs hi = fp16(d*q), lo = fp16(d*q - hi), exact (hi + lo == d*q),
+ * and the weights to fp16 w' = E2M1*s_w (exact); every product is exact
+ * and only the fp32 accumulation rounds; y = g * sum.
  * workspace: device, caller-owned, >= nvq_gemm_workspace_size(M, N, K)
  * bytes, 16-byte aligned; its contents are scratch.
  * Errors: as nvq_gemv (M >= 1), plus NVQ_ERR_WORKSPACE.
