@@ -1,6 +1,6 @@
-"""GPU parity of nvq_gemm at M = 1..16 (M <= 4 runs the decode GEMV, 5..16 the
-small-token tensor-core schedule; for the latter K % 256 == 0 is required,
-K % 256 == 0): weights expanded into tensor memory, the exact fp16 hi/lo
+"""GPU parity of nvq_gemm at M = 1..16: M <= 4 runs the decode GEMV, 5..16
+(K % 256 == 0) the small-token tensor-core schedule: weights expanded into
+tensor memory, the exact fp16 hi/lo
 activations by TMA, tcgen05.mma with fp32 accumulation promoted every
 1024 K, and the work split in equal ranges of (row tile, K stage) units over
 the SMs (stream-K), with split tiles added in a fixed order.
