@@ -30,6 +30,10 @@ What it computes, and the passages it follows
 [ROOF]     "Roofline-First Decoding: results": a fused 4-bit dequantise-plus-
            GEMV for batch-1 decoding on fp16 activations (W4A16); here the
            4-bit weights are NVFP4 and the activations binary16 values.
+[MOE]      [HANDOFF] section 7 "Open items / next steps", item 1: the NVFP4
+           row dot inside a mixture-of-experts product (mul_mat_id: K = 2048,
+           256 experts, 6 active per token), each token multiplied by the
+           weight matrices of the experts its routing selects.
 [OCP-MX]   OCP Microscaling Formats (MX) v1.0: the E2M1 element type (1 sign,
            2 exponent bits with bias 1, 1 mantissa bit; max 6) and the E4M3
            type (4 exponent bits with bias 7, 3 mantissa bits, max 448, S.1111.111
@@ -68,7 +72,7 @@ __all__ = [
     "unpack_codes", "dequantize_weights", "dequantize_activations",
     "dot_fp64", "subblock_sums", "subblock_sums_biased", "bsum16",
     "y_from_subblock_sums", "sum_abs_terms", "tolerance",
-    "dot_fp64_f16", "sum_abs_terms_f16",
+    "dot_fp64_f16", "sum_abs_terms_f16", "moe_dot_fp64",
     "ACC_REL_TOL", "ACC_ABS_TOL",
 ]
 
@@ -439,3 +443,33 @@ def sum_abs_terms_f16(codes, scales, g, x_bits, row_chunk: int = 1024) -> np.nda
                          a.reshape(M, K // 16, 16))
         out[:, n0:n1] = np.abs(part).sum(axis=2)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Mixture-of-experts product (mul_mat_id) [MOE]
+# ---------------------------------------------------------------------------
+
+def moe_dot_fp64(codes, scales, g, ids, q, d) -> np.ndarray:
+    """y[t, j, n] = sum_k w_{ids[t, j]}[n, k] * a[t, k] in fp64,
+    fp64 [T, top_k, N].
+
+    codes [E, N, K/2], scales [E, N, K/16], g [E] (one per-tensor scale per
+    expert), ids int [T, top_k] (expert of each slot, every id in 0..E-1),
+    q [T, K], d [T, K/32]: each token is multiplied by the matrices of its
+    selected experts with the plain dot_fp64.
+    Pinned by tests/test_oracle_moe.py.
+    """
+    codes = np.asarray(codes)
+    scales = np.asarray(scales)
+    g = np.asarray(g, dtype=np.float32)
+    ids = np.asarray(ids)
+    T, top_k = ids.shape
+    E, N = codes.shape[0], codes.shape[1]
+    if np.any(ids < 0) or np.any(ids >= E):
+        raise ValueError("expert id out of range")
+    y = np.empty((T, top_k, N), dtype=np.float64)
+    for t in range(T):
+        for j in range(top_k):
+            e = int(ids[t, j])
+            y[t, j] = dot_fp64(codes[e], scales[e], g[e], q[t:t + 1], d[t:t + 1])[0]
+    return y
