@@ -24,6 +24,10 @@ workload under ``"workloads"``, each measured the same way):
                           of NVFP4 weights resident), one token.  Metric:
                           tokens/s of the linear layers.
   stack_prefill           the same stack for 2048 tokens.
+  moe_decode              mixture-of-experts decode (mul_mat_id): 16 tokens,
+                          each times 6 of 256 experts (K = 2048, N = 1536),
+                          a different seeded routing every step.  Metric:
+                          weight GB/s of the selected experts' rows.
 
 Timing: W untimed eager warm-up steps; the K timed steps are captured once
 into a CUDA graph (the public entry points only enqueue work) and replayed
@@ -84,7 +88,7 @@ WEIGHT_BYTES_PER_ELEMENT = 0.5625       # 4-bit code + one UE4M3 byte per 16
 L2_BYTES = 126e6
 SUB_WORKLOADS = ["gemv_4096", "small_batch_m2", "small_batch_m4", "small_batch_m8",
                  "small_batch_m16", "prefill_m256", "prefill_m2048", "stack_decode",
-                 "stack_prefill"]
+                 "stack_prefill", "moe_decode"]
 
 
 # ---------------------------------------------------------------------------
@@ -648,6 +652,116 @@ class StackWorkload:
                 "activations), scaled to the 64-layer pass by the fraction of weights processed")
 
 
+class MoeWorkload:
+    """Mixture-of-experts decode: Q8_0 of 16 tokens and nvq_moe_gemv."""
+
+    kernel = "moe_gemv"
+    sources = ("gemv.cu", "nvq_device.cuh", "tcgen05.cuh")
+    bound = "hbm"
+    metric = "nvfp4_q8_0_moe_gemv_weight_GBps"
+    unit = "GB/s"
+    ROUTINGS = 8
+
+    def __init__(self, name):
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        self.name = name
+        self.E, self.N, self.K = wl.MOE_EXPERTS, wl.MOE_N, wl.MOE_K
+        self.top_k, self.T = wl.MOE_TOP_K, wl.MOE_TOKENS
+
+    def setup(self, device):
+        import torch
+        from bit_weight_quantized_nvq_b200 import capi, workloads as wl
+        self.capi = capi
+        E, N, K = self.E, self.N, self.K
+        self.codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.empty((E, N, K // 16), dtype=torch.uint8, device=device)
+        g = np.empty(E, np.float32)
+        for e in range(E):
+            c, sc, g[e] = capi.pack_nvfp4(wl.moe_expert_weights(e))
+            self.codes[e].copy_(torch.from_numpy(c))
+            self.scales[e].copy_(torch.from_numpy(sc))
+        self.g = torch.from_numpy(g).to(device)
+        self.ids = [torch.from_numpy(wl.moe_routing(self.T, step=s)).to(device)
+                    for s in range(self.ROUTINGS)]
+        x = wl.moe_tokens(self.T)
+        self.x = torch.from_numpy(x).to(device)
+        self.x_host = torch.from_numpy(x).pin_memory()
+        self.q = torch.empty((self.T, K), dtype=torch.int8, device=device)
+        self.d = torch.empty((self.T, K // 32), dtype=torch.float16, device=device)
+        self.y = torch.empty((self.T, self.top_k, N), dtype=torch.float32, device=device)
+        self.y_host = torch.empty(tuple(self.y.shape), dtype=torch.float32).pin_memory()
+        self.i = 0
+
+    def config(self):
+        return {"workload": self.name, "tokens": self.T, "experts": self.E,
+                "top_k": self.top_k, "expert_KN": [self.K, self.N],
+                "weights": "NVFP4 experts, N(0,0.02^2); routing uniform without replacement, "
+                           f"{self.ROUTINGS} seeded routings used in turn",
+                "activations": "fp32 N(0,1) -> Q8_0 on the GPU every step",
+                "l2": "inputs larger than L2 (%.0f MB of expert rows per step, 453 MB of "
+                      "experts)" % (self.weight_bytes() / 1e6),
+                "parallelism": "replicas"}
+
+    def weight_bytes(self):
+        return self.T * self.top_k * self.N * self.K * WEIGHT_BYTES_PER_ELEMENT
+
+    def units_per_step(self):
+        return self.weight_bytes() / 1e9
+
+    def kernel_amount(self):
+        return (self.weight_bytes() + self.T * self.K * (1 + 2 / 32)
+                + 4 * self.T * self.top_k * self.N + 4 * self.T * self.top_k)
+
+    def launches_per_step(self):
+        return 2
+
+    def dominant(self, ids, stream):
+        self.capi.moe_gemv(self.codes, self.scales, self.g, ids, self.q, self.d, self.y,
+                           stream=stream)
+
+    def step(self, stream, e2e=False):
+        ids = self.ids[self.i % self.ROUTINGS]
+        self.i += 1
+        if e2e:
+            self.x.copy_(self.x_host, non_blocking=True)
+        self.capi.quantize_act_q8_0(self.x, self.q, self.d, stream=stream)
+        self.dominant(ids, stream)
+        if e2e:
+            self.y_host.copy_(self.y, non_blocking=True)
+
+    def e2e_bytes(self):
+        return self.x.numel() * 4, self.y.numel() * 4
+
+    def shape_timings(self, stream, reps):
+        import torch
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            s = torch.cuda.current_stream()
+            for i in range(reps):
+                self.dominant(self.ids[i % self.ROUTINGS], s)
+        graph.replay()
+        ms = replay_ms(graph, stream)
+        del graph
+        return [{"K": self.K, "N": self.N * self.top_k * self.T, "us_per_launch": ms * 1e3 / reps,
+                 "amount": self.kernel_amount(), "weight_copies": self.ROUTINGS}]
+
+    def oracle_tasks(self, rows):
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        ids = wl.moe_routing(self.T, step=0)
+        x = wl.moe_tokens(self.T)[:1]
+        tasks = []
+        for e in ids[0]:
+            base = oracle_base(("moe", int(e)), lambda e=e: (
+                wl.weight_rows("moe", f"expert{int(e)}", self.N, self.K, ORACLE_BASE_ROWS), x))
+            tasks.append(sample_task(base, rows, self.K * WEIGHT_BYTES_PER_ELEMENT / 1e9))
+        return tasks
+
+    def oracle_sample_desc(self, rows):
+        return (f"one token x {rows} weight rows of each of its {self.top_k} experts (the first "
+                f"{ORACLE_BASE_ROWS} rows, oracle-packed, run repeatedly): oracle Q8_0 + fp64 "
+                "dequantise-then-dot")
+
+
 def make_workload(name: str):
     from bit_weight_quantized_nvq_b200 import workloads as wl
     if name == "decode_sweep":
@@ -670,6 +784,8 @@ def make_workload(name: str):
         return StackWorkload(name, 1)
     if name == "stack_prefill":
         return StackWorkload(name, 2048)
+    if name == "moe_decode":
+        return MoeWorkload(name)
     raise SystemExit(f"unknown workload {name!r}")
 
 

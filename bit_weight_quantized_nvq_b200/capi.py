@@ -48,6 +48,8 @@ SIGNATURES = {
                                         _vp, _vp, _vp, _vp]),
     "nvq_gemv_grouped": (ctypes.c_int, [ctypes.POINTER(Linear), _c_i64, _vp, _vp, _c_i64,
                                         ctypes.POINTER(_vp), _vp]),
+    "nvq_moe_gemv": (ctypes.c_int, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _vp, _c_i64, _c_i64,
+                                    _vp, _vp, _vp, _vp]),
     "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
@@ -198,6 +200,23 @@ def gemv_grouped(mats, q: torch.Tensor, d: torch.Tensor, ys=None, stream=None):
     return ys
 
 
+def moe_gemv(codes: torch.Tensor, scales: torch.Tensor, g: torch.Tensor, ids: torch.Tensor,
+             q: torch.Tensor, d: torch.Tensor, y: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """Mixture-of-experts decode GEMV (nvq_moe_gemv): codes [E, N, K/2],
+    scales [E, N, K/16], g float32 [E], ids int32 [T, top_k] (all on the
+    device); returns y fp32 [T, top_k, N]."""
+    E, N = codes.shape[0], codes.shape[1]
+    T, K = q.shape
+    top_k = ids.shape[1]
+    if y is None:
+        y = torch.empty((T, top_k, N), dtype=torch.float32, device=q.device)
+    _check("nvq_moe_gemv", _lib.nvq_moe_gemv(
+        _ptr(codes), _ptr(scales), _ptr(g), E, N, K, _ptr(ids), T, top_k, _ptr(q), _ptr(d),
+        _ptr(y), _stream(stream)))
+    return y
+
+
 def gemm_workspace_size(M: int, N: int, K: int) -> int:
     return int(_lib.nvq_gemm_workspace_size(M, N, K))
 
@@ -253,6 +272,7 @@ def debug_subblock_sums(codes: torch.Tensor, scales: torch.Tensor, g: float, q: 
 
 FLAG_GEMV_TIMEOUT = 1
 FLAG_GEMM_TIMEOUT = 2
+FLAG_BAD_INDEX = 4
 
 
 def error_flags(clear: bool = False) -> int:

@@ -319,7 +319,7 @@ gemv_m1_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
 // never written by the kernels before it) overlap the previous kernel's tail
 // without changing results.
 constexpr uint32_t kRegStageMax = 46080;
-constexpr int kMaxGroup = 3;       // matrices per register-schedule launch
+constexpr int kMaxGroup = 8;       // matrices per register-schedule launch
 
 __host__ __device__ constexpr int reg_rows(int K, int wpr) {
   int r = kM1Consumers / wpr;
@@ -360,6 +360,23 @@ struct RegGroup {
   int count;
   int rows;          // concatenated rows
 };
+
+// A mixture-of-experts launch: grid row t handles token t, whose group is
+// the experts ids[t, 0..top_k) of a stacked expert tensor, built on the
+// device once the routing ids are visible (ids == nullptr: not a MoE launch).
+struct MoeArgs {
+  const int32_t* ids;     // [T, top_k]
+  const uint8_t* codes;   // [E, N, K/2]
+  const uint8_t* scales;  // [E, N, K/16]
+  const float* g;         // [E]
+  float* y;               // [T, top_k, N]
+  int E;
+  int N;
+  int top_k;
+};
+
+// bit 1 of the GEMV error flags: a routing id outside 0..E-1 (its slot is skipped)
+__device__ __forceinline__ void raise_bad_index() { atomicOr(&g_gemv_error_flags, 2u); }
 
 // Q8_0 of the 32 outputs of block b, one lane per output: the same IEEE
 // operations as the activation quantiser (amax, d32 = amax/127, q =
@@ -426,9 +443,14 @@ __device__ __forceinline__ void next_stage(const RegGroup& grp, int& gr, int r_e
 
 template <int NPL, int WPR, bool ISUM>
 __global__ void __launch_bounds__(kM1Threads, 1)
-gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __restrict__ q,
-                   const __half* __restrict__ d, int32_t* __restrict__ isum) {
+gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_constant__ MoeArgs moe,
+                   int K, const int8_t* __restrict__ q_all, const __half* __restrict__ d_all,
+                   int32_t* __restrict__ isum) {
   extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ RegGroup grp;
+  // token of this grid row (several only for mixture-of-experts launches)
+  const int8_t* __restrict__ q = q_all + static_cast<size_t>(blockIdx.y) * K;
+  const __half* __restrict__ d = d_all + static_cast<size_t>(blockIdx.y) * (K / 32);
   const int R = reg_rows(K, WPR);
   const int active = R * WPR;                      // consumer warps in use
   const uint32_t row_code = K / 2, row_scale = K / 16;
@@ -443,11 +465,38 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x;
-  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * grp.rows / G);
-  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * grp.rows / G);
 
   grid_dependents_launch();
-  for (int i = threadIdx.x; i < reg_block_slots(grp.rows, G); i += blockDim.x) scnt[i] = 0;
+  const bool is_moe = moe.ids != nullptr;
+  if (is_moe) {
+    // the routing ids come from the previous kernel
+    grid_dependency_wait();
+    if (threadIdx.x == 0) {
+      const int t = blockIdx.y;
+      int rows = 0, cnt = 0;
+      for (int j = 0; j < moe.top_k; ++j) {
+        const int e = moe.ids[t * moe.top_k + j];
+        if (e < 0 || e >= moe.E) {
+          raise_bad_index();
+          continue;
+        }
+        RegMat m = {};
+        m.codes = moe.codes + static_cast<size_t>(e) * moe.N * (K / 2);
+        m.scales = moe.scales + static_cast<size_t>(e) * moe.N * (K / 16);
+        m.y = moe.y + (static_cast<size_t>(t) * moe.top_k + j) * moe.N;
+        m.half_g = 0.5f * moe.g[e];
+        m.N = moe.N;
+        m.row_off = rows;
+        rows += moe.N;
+        grp.m[cnt++] = m;
+      }
+      grp.count = cnt;
+      grp.rows = rows;
+    }
+  } else {
+    if (threadIdx.x == 0) grp = grp_param;
+    for (int i = threadIdx.x; i < reg_block_slots(grp_param.rows, G); i += blockDim.x) scnt[i] = 0;
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kM1Stages; ++i) {
       ptx::mbar_init(ptx::smem_addr(full + i), 1);
@@ -457,6 +506,8 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp, int K, const int8_t* __
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * grp.rows / G);
+  const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * grp.rows / G);
 
   if (warp == kM1Consumers) {
     // ------------- producer: bulk copies, and the sum of row partials --------
@@ -872,8 +923,35 @@ cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, grp, static_cast<int>(K), q,
+  const MoeArgs no_moe = {};
+  return cudaLaunchKernelEx(&cfg, kernel, grp, no_moe, static_cast<int>(K), q,
                             reinterpret_cast<const __half*>(d), isum);
+}
+
+template <int NPL, int WPR>
+cudaError_t launch_moe_reg(const MoeArgs& moe, int64_t T, int64_t K, const int8_t* q,
+                           const uint16_t* d, cudaStream_t stream) {
+  auto kernel = gemv_m1_reg_kernel<NPL, WPR, false>;
+  static SmemAttrOnce attr;
+  cudaError_t e = attr.ensure(kernel, static_cast<int>(kSmemPerCtaMax));
+  if (e != cudaSuccess) return e;
+  // the SMs split evenly over the tokens; each token's rows over its CTAs
+  const int64_t per_token = std::max<int64_t>(1, device_sm_count() / T);
+  const int64_t rows = static_cast<int64_t>(moe.top_k) * moe.N;
+  const int64_t ctas = std::min<int64_t>(per_token, rows);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), static_cast<unsigned>(T));
+  cfg.blockDim = dim3(kM1Threads);
+  cfg.dynamicSmemBytes = reg_smem_bytes(static_cast<int>(K), WPR);
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  const RegGroup none = {};
+  return cudaLaunchKernelEx(&cfg, kernel, none, moe, static_cast<int>(K), q,
+                            reinterpret_cast<const __half*>(d), static_cast<int32_t*>(nullptr));
 }
 
 // The register schedule covers K = 1024 * NPL * WPR for the (NPL, WPR) pairs
@@ -881,7 +959,8 @@ cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const
 bool reg_supported(int64_t K) {
   if (K % 1024 != 0) return false;
   switch (K / 1024) {
-    case 4: case 5: case 6: case 8: case 10: case 12: case 15: case 16: case 20: case 25:
+    case 2: case 3: case 4: case 5: case 6: case 8: case 10: case 12: case 15: case 16:
+    case 20: case 25:
       return true;
     default:
       return false;
@@ -894,6 +973,8 @@ cudaError_t launch_m1_reg_group(const RegGroup& grp, int64_t K, const int8_t* q,
   if (!reg_supported(K)) return cudaErrorNotSupported;
 #define NVQ_REG(npl, wpr) return launch_m1_reg<npl, wpr, ISUM>(grp, K, q, d, isum, stream)
   switch (K / 1024) {
+    case 2: NVQ_REG(2, 1);
+    case 3: NVQ_REG(3, 1);
     case 4: NVQ_REG(4, 1);
     case 5: NVQ_REG(5, 1);
     case 6: NVQ_REG(6, 1);
@@ -1037,6 +1118,42 @@ cudaError_t launch_gemv_group(const GemvTarget* t, int n, int64_t K, const int8_
     ++done;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_moe_gemv(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t E,
+                            int64_t N, int64_t K, const int32_t* ids, int64_t T, int64_t top_k,
+                            const int8_t* q, const uint16_t* d, float* y, cudaStream_t stream) {
+  if (!reg_supported(K) || top_k < 1 || top_k > kMaxGroup) return cudaErrorNotSupported;
+  MoeArgs moe = {};
+  moe.ids = ids;
+  moe.codes = codes;
+  moe.scales = scales;
+  moe.g = g;
+  moe.y = y;
+  moe.E = static_cast<int>(E);
+  moe.N = static_cast<int>(N);
+  moe.top_k = static_cast<int>(top_k);
+#define NVQ_MOE(npl, wpr) return launch_moe_reg<npl, wpr>(moe, T, K, q, d, stream)
+  switch (K / 1024) {
+    case 2: NVQ_MOE(2, 1);
+    case 3: NVQ_MOE(3, 1);
+    case 4: NVQ_MOE(4, 1);
+    case 5: NVQ_MOE(5, 1);
+    case 6: NVQ_MOE(6, 1);
+    case 8: NVQ_MOE(4, 2);
+    case 10: NVQ_MOE(5, 2);
+    case 12: NVQ_MOE(6, 2);
+    case 15: NVQ_MOE(5, 3);
+    case 16: NVQ_MOE(4, 4);
+    case 20: NVQ_MOE(5, 4);
+    case 25: NVQ_MOE(5, 5);
+    default: return cudaErrorNotSupported;
+  }
+#undef NVQ_MOE
+}
+
+bool moe_supported(int64_t K, int64_t top_k) {
+  return reg_supported(K) && top_k >= 1 && top_k <= kMaxGroup;
 }
 
 cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream) {

@@ -196,6 +196,25 @@ nvq_status nvq_gemv_grouped(const nvq_linear* linears, int64_t count, const int8
   return NVQ_OK;
 }
 
+nvq_status nvq_moe_gemv(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t E,
+                        int64_t N, int64_t K, const int32_t* ids, int64_t T, int64_t top_k,
+                        const int8_t* q, const uint16_t* d, float* y, void* stream) {
+  if (E < 0 || N < 0 || K < 0 || T < 0 || top_k < 0) return NVQ_ERR_INVALID_ARG;
+  if (K == 0 || K % 64 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (T == 0 || top_k == 0 || N == 0) return NVQ_OK;
+  if (E == 0) return NVQ_ERR_INVALID_ARG;
+  if (!nvq::moe_supported(K, top_k)) return NVQ_ERR_BAD_SHAPE;
+  if (T > 65535 || N > (int64_t{1} << 24) || E * N > (int64_t{1} << 32)) return NVQ_ERR_BAD_SHAPE;
+  if (!codes || !scales || !g || !ids || !q || !d || !y) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(q) || !aligned16(d) ||
+      !aligned16(y) || !aligned16(ids) || !aligned16(g))
+    return NVQ_ERR_MISALIGNED;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_moe_gemv(codes, scales, g, E, N, K, ids, T, top_k, q, d, y,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || K <= 0 || N < 0) return 0;
   return nvq::gemm_workspace_size(M, N, K);
@@ -268,7 +287,8 @@ nvq_status nvq_error_flags(unsigned int* flags, int clear) {
     cudaGetLastError();
     return cuda_status(e);
   }
-  *flags = (gemv ? NVQ_FLAG_GEMV_TIMEOUT : 0u) | (gemm ? NVQ_FLAG_GEMM_TIMEOUT : 0u);
+  *flags = ((gemv & 1u) ? NVQ_FLAG_GEMV_TIMEOUT : 0u) | (gemm ? NVQ_FLAG_GEMM_TIMEOUT : 0u) |
+           ((gemv & 2u) ? NVQ_FLAG_BAD_INDEX : 0u);
   return NVQ_OK;
 }
 

@@ -45,6 +45,15 @@ struct GemvTarget {
 cudaError_t launch_gemv_group(const GemvTarget* targets, int n, int64_t K, const int8_t* q,
                               const uint16_t* d, cudaStream_t stream);
 
+// Mixture-of-experts decode GEMV: token t times the experts ids[t, j] of a
+// stacked expert tensor, y [T, top_k, N]; supported for the K of the
+// register schedule and top_k <= 8.  A routing id outside 0..E-1 raises
+// error bit 1 and its slot is left unwritten.
+bool moe_supported(int64_t K, int64_t top_k);
+cudaError_t launch_moe_gemv(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t E,
+                            int64_t N, int64_t K, const int32_t* ids, int64_t T, int64_t top_k,
+                            const int8_t* q, const uint16_t* d, float* y, cudaStream_t stream);
+
 // Test-only: a pipeline wait that can never complete, bounded by limit_ns;
 // result[0] = 1 if the wait completed (never), result[1] = microseconds waited.
 cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream);

@@ -17,6 +17,12 @@ Workloads (shapes are (K, N) of a weight W[N, K]; M is the token count):
 * ``prefill``       M in {256, 2048} over (5120, 5120), (5120, 25600) and
                     (25600, 5120); W ~ N(0, 0.02^2); x ~ N(0, 1) with 0.1 % of
                     the hidden channels scaled x50 in every token row.
+* ``moe``           a mixture-of-experts layer at decode: 256 experts with
+                    K = 2048 (hidden) and N = 1536 (the stacked gate and up
+                    projections of a 768-wide expert), 6 experts per token,
+                    16 tokens per step; W ~ N(0, 0.02^2) per expert, x ~
+                    N(0, 1); each token's experts drawn uniformly without
+                    replacement, seeded per step.
 * ``stack``         the seven linears of one layer of a 64-layer dense
                     transformer (hidden 5120, gated MLP 25600): q, k, v, o
                     (5120, 5120), up and gate (5120, 25600), down (25600, 5120);
@@ -45,6 +51,11 @@ SMALL_BATCH_MS = [2, 4, 8, 16]
 SMALL_BATCH_SHAPES = [(5120, 25600), (25600, 5120)]
 PREFILL_MS = [256, 2048]
 PREFILL_SHAPES = [(5120, 5120), (5120, 25600), (25600, 5120)]
+MOE_EXPERTS = 256
+MOE_TOP_K = 6
+MOE_K = 2048
+MOE_N = 1536
+MOE_TOKENS = 16
 STACK_LAYERS = 64
 STACK_HIDDEN = 5120
 STACK_MLP = 25600
@@ -179,3 +190,20 @@ def stack_layer_weights():
 def stack_input(M: int):
     """fp32 layer input x[M, 5120] ~ N(0, 1)."""
     return activations("stack", "x", M, STACK_HIDDEN, "normal")
+
+
+def moe_expert_weights(e: int, N: int = MOE_N, K: int = MOE_K, workload: str = "moe") -> np.ndarray:
+    """fp32 W_e[N, K] of expert e ~ N(0, 0.02^2)."""
+    return weights(workload, f"expert{e}", N, K)
+
+
+def moe_routing(T: int, top_k: int = MOE_TOP_K, E: int = MOE_EXPERTS, step: int = 0,
+                workload: str = "moe") -> np.ndarray:
+    """int32 ids[T, top_k]: each token's experts, distinct, uniform."""
+    rng = np.random.Generator(np.random.PCG64(seed_sequence(workload, "routing", T, top_k, E, step)))
+    return np.stack([rng.choice(E, size=top_k, replace=False) for _ in range(T)]).astype(np.int32)
+
+
+def moe_tokens(T: int = MOE_TOKENS, K: int = MOE_K, workload: str = "moe") -> np.ndarray:
+    """fp32 x[T, K] ~ N(0, 1)."""
+    return activations(workload, "x", T, K, "normal")

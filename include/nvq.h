@@ -186,6 +186,34 @@ nvq_status nvq_gemv_grouped(const nvq_linear* linears, int64_t count, const int8
                             const uint16_t* d, int64_t M, float* const* ys, void* stream);
 
 /*
+ * nvq_moe_gemv - the mixture-of-experts product of decode (mul_mat_id):
+ * every token times the weight matrices of the experts its routing selects,
+ * y[t, j, :] = A[t, :] . W_{ids[t, j]}^T.  ("HANDOFF: flint CPU optimization
+ * (Q4_1 + NVFP4)", section 7 "Open items / next steps", item 1: the NVFP4 x
+ * Q8_0 row dot on a mixture-of-experts shape, K = 2048, 256 experts, 6
+ * active per token.)
+ *
+ * codes   device uint8 [E, N, K/2], scales device uint8 [E, N, K/16]: the E
+ *         experts' NVFP4 matrices W_e[N, K], stacked.
+ * g       device float [E]: per-expert tensor scales.
+ * ids     device int32 [T, top_k]: the experts of each token (read on the
+ *         device, so the routing may come from a previous kernel).
+ * q, d    device Q8_0 activations [T, K], [T, K/32].
+ * y       device float [T, top_k, N].
+ * Each token's CTAs stream its selected experts' rows (concatenated, split
+ * evenly) with the register schedule of nvq_gemv, so the result of every
+ * slot is that of nvq_gemv on its expert.  Requires K = 1024 * T' with T' in
+ * {2,3,4,5,6,8,10,12,15,16,20,25} and 1 <= top_k <= 8 (NVQ_ERR_BAD_SHAPE
+ * otherwise), T <= 65535.  An id outside 0..E-1 is skipped (its slot of y is
+ * left as it was) and raises NVQ_FLAG_BAD_INDEX (nvq_error_flags).
+ * Errors: NVQ_ERR_INVALID_ARG, NVQ_ERR_BAD_SHAPE, NVQ_ERR_MISALIGNED,
+ * NVQ_ERR_UNSUPPORTED_DEVICE, NVQ_ERR_CUDA.
+ */
+nvq_status nvq_moe_gemv(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t E,
+                        int64_t N, int64_t K, const int32_t* ids, int64_t T, int64_t top_k,
+                        const int8_t* q, const uint16_t* d, float* y, void* stream);
+
+/*
  * nvq_gemm_workspace_size - bytes of device workspace nvq_gemm needs for
  * M tokens of K features (0 when M == 0).  It holds the activations
  * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q.
@@ -285,6 +313,7 @@ nvq_status nvq_debug_subblock_sums(const uint8_t* codes, const uint8_t* scales, 
 /* Bits of nvq_error_flags. */
 #define NVQ_FLAG_GEMV_TIMEOUT 1u  /* a GEMV pipeline wait gave up (4 s)  */
 #define NVQ_FLAG_GEMM_TIMEOUT 2u  /* a GEMM pipeline wait gave up (4 s)  */
+#define NVQ_FLAG_BAD_INDEX    4u  /* nvq_moe_gemv met a routing id outside 0..E-1 */
 
 /*
  * nvq_error_flags - device-side error flags of the current device.

@@ -62,15 +62,15 @@ def test_small_shapes_all_rows(M, N, K):
 
 
 # K -> the M = 1 kernel nvq_gemv dispatches to:
-#   K = 1024*T, T in {4,5,6,8,10,12,15,16,20,25}: register schedule
-#     <chunks per lane, warps per row> = <4,1> <5,1> <6,1> <4,2> <5,2> <6,2>
+#   K = 1024*T, T in {2,3,4,5,6,8,10,12,15,16,20,25}: register schedule
+#     <chunks per lane, warps per row> = <2,1> <3,1> <4,1> <5,1> <6,1> <4,2> <5,2> <6,2>
 #     <5,3> <4,4> <5,4> <5,5>;
 #   30720: shared-memory schedule, 5120-element segments (<5>);
 #   28672: shared-memory schedule, 4096-element segments (<4>);
 #   1280, 12800: shared-memory schedule, other segments (<0>);
 #   35840: its shared memory does not fit, the TMA schedule <1>;
 #   1088: K % 256 != 0, the one-warp-per-row kernel <1>.
-M1_DISPATCH_KS = [4096, 5120, 6144, 8192, 10240, 12288, 15360, 16384, 20480, 25600,
+M1_DISPATCH_KS = [2048, 3072, 4096, 5120, 6144, 8192, 10240, 12288, 15360, 16384, 20480, 25600,
                   30720, 28672, 1280, 12800, 35840, 1088]
 
 
