@@ -361,6 +361,11 @@ struct RegGroup {
   int rows;          // concatenated rows
 };
 
+// dynamic shared memory the register schedule may request: the opt-in
+// maximum less room for its static shared memory (the group of matrices)
+constexpr uint32_t kRegDynSmemMax = kSmemPerCtaMax - 2048;
+static_assert(sizeof(RegGroup) <= 2048, "static shared memory of the register schedule");
+
 // A mixture-of-experts launch: grid row t handles token t, whose group is
 // the experts ids[t, 0..top_k) of a stacked expert tensor, built on the
 // device once the routing ids are visible (ids == nullptr: not a MoE launch).
@@ -907,12 +912,12 @@ cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const
                           int32_t* isum, cudaStream_t stream) {
   auto kernel = gemv_m1_reg_kernel<NPL, WPR, ISUM>;
   static SmemAttrOnce attr;
-  cudaError_t e = attr.ensure(kernel, static_cast<int>(kSmemPerCtaMax));
+  cudaError_t e = attr.ensure(kernel, static_cast<int>(kRegDynSmemMax));
   if (e != cudaSuccess) return e;
   const int64_t ctas = std::min<int64_t>(device_sm_count(), grp.rows);
   const uint32_t smem = reg_smem_bytes(static_cast<int>(K), WPR) +
                         4u * reg_block_slots(grp.rows, static_cast<int>(ctas));
-  if (smem > kSmemPerCtaMax) return cudaErrorInvalidValue;
+  if (smem > kRegDynSmemMax) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas));
   cfg.blockDim = dim3(kM1Threads);
@@ -933,7 +938,7 @@ cudaError_t launch_moe_reg(const MoeArgs& moe, int64_t T, int64_t K, const int8_
                            const uint16_t* d, cudaStream_t stream) {
   auto kernel = gemv_m1_reg_kernel<NPL, WPR, false>;
   static SmemAttrOnce attr;
-  cudaError_t e = attr.ensure(kernel, static_cast<int>(kSmemPerCtaMax));
+  cudaError_t e = attr.ensure(kernel, static_cast<int>(kRegDynSmemMax));
   if (e != cudaSuccess) return e;
   // the SMs split evenly over the tokens; each token's rows over its CTAs
   const int64_t per_token = std::max<int64_t>(1, device_sm_count() / T);
