@@ -24,6 +24,8 @@ workload under ``"workloads"``, each measured the same way):
                           of NVFP4 weights resident), one token.  Metric:
                           tokens/s of the linear layers.
   stack_prefill           the same stack for 2048 tokens.
+  w4a16_decode            the decode-sweep shapes at one token with fp16
+                          activations (nvq_gemm_w4a16).  Metric: weight GB/s.
   moe_decode              mixture-of-experts decode (mul_mat_id): 16 tokens,
                           each times 6 of 256 experts (K = 2048, N = 1536),
                           a different seeded routing every step.  Metric:
@@ -88,7 +90,7 @@ WEIGHT_BYTES_PER_ELEMENT = 0.5625       # 4-bit code + one UE4M3 byte per 16
 L2_BYTES = 126e6
 SUB_WORKLOADS = ["gemv_4096", "small_batch_m2", "small_batch_m4", "small_batch_m8",
                  "small_batch_m16", "prefill_m256", "prefill_m2048", "stack_decode",
-                 "stack_prefill", "moe_decode"]
+                 "stack_prefill", "moe_decode", "w4a16_decode"]
 
 
 # ---------------------------------------------------------------------------
@@ -259,9 +261,14 @@ def l2_copies(nbytes: float) -> int:
 def oracle_task(task):
     """Run one oracle task, (codes, scales, g, x, reps, units) -> units: the
     oracle's Q8_0 quantisation of x, then its fp64 dequantise-then-dot of the
-    weight block, `reps` times."""
+    weight block, `reps` times (x given as fp16 bit patterns, uint16: the
+    fp16-activation dot instead)."""
     import oracle as o
     codes, scales, g, x, reps, units = task
+    if x.dtype == np.uint16:
+        for _ in range(reps):
+            o.dot_fp64_f16(codes, scales, g, x)
+        return units
     q, d = o.quantize_q8_0(x)
     for _ in range(reps):
         o.dot_fp64(codes, scales, g, q, d)
@@ -652,6 +659,67 @@ class StackWorkload:
                 "activations), scaled to the 64-layer pass by the fraction of weights processed")
 
 
+class W4A16Workload(GemvWorkload):
+    """fp16-activation decode (W4A16): nvq_gemm_w4a16 over the decode-sweep
+    shapes, one token; the activations are given in fp16 (no quantiser)."""
+
+    kernel = "gemm_w4a16"
+    sources = ("gemm_small.cu", "gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+    metric = "nvfp4_f16_w4a16_weight_GBps"
+
+    def setup(self, device):
+        import torch
+        super().setup(device)
+        for c in self.cases:
+            c["x"] = c["x"].half()
+            c["x_host"] = c["x_host"].half().pin_memory()
+            c["ws"] = torch.empty(
+                int(self.capi.lib().nvq_gemm_w4a16_workspace_size(self.M, c["N"], c["K"])),
+                dtype=torch.uint8, device=device)
+
+    def config(self):
+        cfg = super().config()
+        cfg["activations"] = "fp16 N(0,1) (no quantisation)"
+        cfg["path"] = "nvq_gemm_w4a16 (small-token tcgen05 schedule on fp16 activations)"
+        return cfg
+
+    def kernel_amount(self, K, N):
+        return N * K * WEIGHT_BYTES_PER_ELEMENT + 2 * self.M * K + 4 * self.M * N
+
+    def launches_per_step(self):
+        return 3 * len(self.cases)       # fp16 operand layout, tcgen05 kernel, split-tile sum
+
+    def dominant(self, c, codes, scales, stream):
+        self.capi.gemm_w4a16(codes, scales, c["g"], c["x"], c["y"], c["ws"], stream=stream)
+
+    def step(self, stream, e2e=False):
+        for c in self.cases:
+            if e2e:
+                c["x"].copy_(c["x_host"], non_blocking=True)
+            self.dominant(c, c["codes"], c["scales"], stream)
+            if e2e:
+                c["y_host"].copy_(c["y"], non_blocking=True)
+
+    def e2e_bytes(self):
+        return (sum(c["x"].numel() * 2 for c in self.cases),
+                sum(c["y"].numel() * 4 for c in self.cases))
+
+    def oracle_tasks(self, rows):
+        tasks = []
+        for K, N in self.shapes:
+            def make(K=K, N=N):
+                W, x = self.oracle_rows(K, N, ORACLE_BASE_ROWS)
+                return W, x.astype(np.float16).view(np.uint16)
+            base = oracle_base(("w4a16", self.name, K, N), make)
+            tasks.append(sample_task(base, rows, K * WEIGHT_BYTES_PER_ELEMENT / 1e9))
+        return tasks
+
+    def oracle_sample_desc(self, rows):
+        return (f"{rows} weight rows of each of the {len(self.shapes)} shapes (the first "
+                f"{ORACLE_BASE_ROWS} rows, oracle-packed, run repeatedly), one fp16 token: "
+                "oracle fp64 dequantise-then-dot")
+
+
 class MoeWorkload:
     """Mixture-of-experts decode: Q8_0 of 16 tokens and nvq_moe_gemv."""
 
@@ -786,6 +854,10 @@ def make_workload(name: str):
         return StackWorkload(name, 2048)
     if name == "moe_decode":
         return MoeWorkload(name)
+    if name == "w4a16_decode":
+        return W4A16Workload(name, wl.DECODE_SHAPES, 1, lambda K, N: wl.decode_case(K, N),
+                             lambda K, N, r: (wl.weight_rows("decode_sweep", "W", N, K, r, True),
+                                              wl.activations("decode_sweep", "x", 1, K)))
     raise SystemExit(f"unknown workload {name!r}")
 
 

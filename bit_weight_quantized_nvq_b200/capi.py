@@ -51,6 +51,9 @@ SIGNATURES = {
     "nvq_moe_gemv": (ctypes.c_int, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _vp, _c_i64, _c_i64,
                                     _vp, _vp, _vp, _vp]),
     "nvq_gemm_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
+    "nvq_gemm_w4a16_workspace_size": (ctypes.c_size_t, [_c_i64, _c_i64, _c_i64]),
+    "nvq_gemm_w4a16": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _c_i64, _vp,
+                                      _vp, ctypes.c_size_t, _vp]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
     "nvq_gemm_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
@@ -214,6 +217,24 @@ def moe_gemv(codes: torch.Tensor, scales: torch.Tensor, g: torch.Tensor, ids: to
     _check("nvq_moe_gemv", _lib.nvq_moe_gemv(
         _ptr(codes), _ptr(scales), _ptr(g), E, N, K, _ptr(ids), T, top_k, _ptr(q), _ptr(d),
         _ptr(y), _stream(stream)))
+    return y
+
+
+def gemm_w4a16(codes: torch.Tensor, scales: torch.Tensor, g: float, x: torch.Tensor,
+               y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """NVFP4 weights x fp16 activations (nvq_gemm_w4a16): x float16 [M, K]
+    on the device, M = 1..16; returns y fp32 [M, N]."""
+    N = codes.shape[0]
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    nbytes = int(_lib.nvq_gemm_w4a16_workspace_size(M, N, K))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=x.device)
+    _check("nvq_gemm_w4a16", _lib.nvq_gemm_w4a16(
+        _ptr(codes), _ptr(scales), float(g), N, K, _ptr(x), M, _ptr(y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return y
 
 

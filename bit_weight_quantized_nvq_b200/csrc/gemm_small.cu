@@ -509,6 +509,25 @@ gemm_small_reduce_kernel(const float* __restrict__ partial, int N, int K, int M,
     if (m < M) y[static_cast<size_t>(m) * N + row] = acc[m] * (g * tok_scale[m]);
 }
 
+// fp16 activations (W4A16) into the operand layout of the small-token
+// schedule: hi rows = x (exact), lo rows = 0, rows >= M zero, token scales 1.
+__global__ void __launch_bounds__(256)
+expand_f16_kernel(const uint4* __restrict__ x, int M, int K, int MP, uint4* __restrict__ act,
+                  float* __restrict__ tok_scale) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = blockIdx.x;
+  const int K8 = K / 8;
+  uint4* hi = act + static_cast<size_t>(row) * K8;
+  uint4* lo = act + static_cast<size_t>(MP + row) * K8;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = threadIdx.x; i < K8; i += blockDim.x) {
+    hi[i] = row < M ? x[static_cast<size_t>(row) * K8 + i] : z;
+    lo[i] = z;
+  }
+  if (threadIdx.x == 0) tok_scale[row] = 1.0f;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -623,6 +642,29 @@ cudaError_t launch_gemm_small(const uint8_t* codes, const uint8_t* scales, float
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   cudaError_t e = expand_activations(q, d, M, L.mp, K, ws + L.act,
                                      reinterpret_cast<float*>(ws + L.tok), stream);
+  if (e != cudaSuccess) return e;
+  if (L.mp == 8) return launch_small<16>(codes, scales, g, N, K, M, y, L, ws, stream);
+  return launch_small<32>(codes, scales, g, N, K, M, y, L, ws, stream);
+}
+
+cudaError_t launch_gemm_small_f16(const uint8_t* codes, const uint8_t* scales, float g,
+                                  int64_t N, int64_t K, const uint16_t* x, int64_t M, float* y,
+                                  void* workspace, cudaStream_t stream) {
+  const SmallLayout L = small_layout(M, K);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(L.mp));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, expand_f16_kernel, reinterpret_cast<const uint4*>(x),
+                                     static_cast<int>(M), static_cast<int>(K),
+                                     static_cast<int>(L.mp), reinterpret_cast<uint4*>(ws + L.act),
+                                     reinterpret_cast<float*>(ws + L.tok));
   if (e != cudaSuccess) return e;
   if (L.mp == 8) return launch_small<16>(codes, scales, g, N, K, M, y, L, ws, stream);
   return launch_small<32>(codes, scales, g, N, K, M, y, L, ws, stream);

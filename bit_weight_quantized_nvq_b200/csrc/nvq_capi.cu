@@ -259,6 +259,29 @@ nvq_status nvq_gemm_noalloc(const uint8_t* codes, const uint8_t* scales, float g
                                       static_cast<cudaStream_t>(stream)));
 }
 
+size_t nvq_gemm_w4a16_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || M > 16 || K <= 0 || K % 256 != 0 || N < 0) return 0;
+  return nvq::gemm_small_workspace_size(M, K);
+}
+
+nvq_status nvq_gemm_w4a16(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                          int64_t K, const uint16_t* x, int64_t M, float* y, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  // x plays the part of q for the pointer checks; there is no d
+  nvq_status st = check_dot_args(codes, scales, N, K, x, x, M, y, 1, 16, true);
+  if (st != NVQ_OK) return st;
+  if (!(g == g)) return NVQ_ERR_INVALID_ARG;
+  if (K % 256 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (N == 0 || M == 0) return NVQ_OK;
+  if (!workspace || workspace_bytes < nvq::gemm_small_workspace_size(M, K))
+    return NVQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return NVQ_ERR_MISALIGNED;
+  st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_gemm_small_f16(codes, scales, g, N, K, x, M, y, workspace,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 nvq_status nvq_debug_subblock_sums(const uint8_t* codes, const uint8_t* scales, float g,
                                    int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
                                    int64_t M, float* y, int32_t* isum, void* stream) {

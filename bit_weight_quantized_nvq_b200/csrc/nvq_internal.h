@@ -81,6 +81,11 @@ cudaError_t launch_gemm_small(const uint8_t* codes, const uint8_t* scales, float
                               int64_t K, const int8_t* q, const uint16_t* d, int64_t M, float* y,
                               void* workspace, cudaStream_t stream);
 cudaError_t gemm_small_error_flags(bool clear, unsigned int* flags);
+// The same schedule on fp16 activations x [M, K] (W4A16), workspace of
+// gemm_small_workspace_size(M, K) bytes.
+cudaError_t launch_gemm_small_f16(const uint8_t* codes, const uint8_t* scales, float g,
+                                  int64_t N, int64_t K, const uint16_t* x, int64_t M, float* y,
+                                  void* workspace, cudaStream_t stream);
 // The two halves of launch_gemm for the large-token schedule: expand Q8_0 activations into the
 // workspace, then run the tensor-core GEMM on an expanded workspace (which
 // several weight matrices with the same K may share).

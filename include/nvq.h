@@ -255,6 +255,28 @@ nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
                     size_t workspace_bytes, void* stream);
 
 /*
+ * nvq_gemm_w4a16 - NVFP4 weights times fp16 activations (W4A16), the fused
+ * 4-bit dequantise-plus-GEMV of batch-1 decoding in "Roofline-First
+ * Decoding: results", for M = 1..16 tokens:
+ * y[m, n] = sum_k w[n, k] * x[m, k].
+ *
+ * x          device uint16 [M, K]: IEEE binary16 bit patterns (finite).
+ * workspace  device, >= nvq_gemm_w4a16_workspace_size(M, N, K) bytes,
+ *            16-byte aligned, scratch.
+ * Runs the small-token tensor-core schedule of nvq_gemm with the
+ * activations taken as they are (an fp16 value is already an exact operand;
+ * the second operand row of each token is zero): w' = E2M1*s_w in fp16,
+ * every product exact, fp32 accumulation promoted every 1024 K, y = g*sum.
+ * Accuracy: |y - exact| <= 1e-5 * sum over 16-subblocks |sum w*x| + 1e-6.
+ * Requires K % 256 == 0 and 1 <= M <= 16 (NVQ_ERR_BAD_SHAPE).
+ * Errors: as nvq_gemm.
+ */
+size_t nvq_gemm_w4a16_workspace_size(int64_t M, int64_t N, int64_t K);
+nvq_status nvq_gemm_w4a16(const uint8_t* codes, const uint8_t* scales, float g, int64_t N,
+                          int64_t K, const uint16_t* x, int64_t M, float* y, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
  * nvq_gemm_noalloc - nvq_gemm for callers that cannot allocate device memory
  * and cannot hand the library a workspace.  (An addition of this library;
  * the web pages describing the method have no counterpart.)
