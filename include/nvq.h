@@ -267,7 +267,8 @@ nvq_status nvq_gemm(const uint8_t* codes, const uint8_t* scales, float g,
  * activations taken as they are (an fp16 value is already an exact operand;
  * the second operand row of each token is zero): w' = E2M1*s_w in fp16,
  * every product exact, fp32 accumulation promoted every 1024 K, y = g*sum.
- * Accuracy: |y - exact| <= 1e-5 * sum over 16-subblocks |sum w*x| + 1e-6.
+ * Accuracy: |y - exact| <= 1e-5 * sum_k |w*x| + 1e-6 per element (the
+ * products are the terms: there are no integer subblock sums here).
  * Requires K % 256 == 0 and 1 <= M <= 16 (NVQ_ERR_BAD_SHAPE).
  * Errors: as nvq_gemm.
  */

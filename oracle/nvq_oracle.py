@@ -428,48 +428,16 @@ def dot_fp64_f16(codes, scales, g, x_bits, row_chunk: int = 4096) -> np.ndarray:
 
 
 def sum_abs_terms_f16(codes, scales, g, x_bits, row_chunk: int = 1024) -> np.ndarray:
-    """sum|terms|[m, n] = sum over 16-element subblocks sb of
-    |sum_{k in sb} w[n, k] * x[m, k]|, fp64 [M, N]: the per-element scale of
-    the accuracy bound for fp16 activations (the subblock partial sums play
-    the part of the Q8_0 path's per-subblock terms)."""
-    a = fp16_values()[np.asarray(x_bits, dtype=np.uint16)]
-    M, K = a.shape
+    """sum|terms|[m, n] = sum_k |w[n, k] * x[m, k]|, fp64 [M, N]: the
+    per-element scale of the accuracy bound for fp16 activations.  The
+    product has no integer subblock sums, so its terms are the individual
+    products w*x (fp32 accumulation of large products that cancel rounds at
+    their scale, not at that of their sum)."""
+    a = np.abs(fp16_values()[np.asarray(x_bits, dtype=np.uint16)])
     N = np.asarray(codes).shape[0]
-    out = np.empty((M, N), dtype=np.float64)
+    out = np.empty((a.shape[0], N), dtype=np.float64)
     for n0 in range(0, N, row_chunk):
         n1 = min(N, n0 + row_chunk)
-        w = dequantize_weights(codes[n0:n1], scales[n0:n1], g)
-        part = np.einsum("nsj,msj->mns", w.reshape(n1 - n0, K // 16, 16),
-                         a.reshape(M, K // 16, 16))
-        out[:, n0:n1] = np.abs(part).sum(axis=2)
+        w = np.abs(dequantize_weights(codes[n0:n1], scales[n0:n1], g))
+        out[:, n0:n1] = a @ w.T
     return out
-
-
-# ---------------------------------------------------------------------------
-# Mixture-of-experts product (mul_mat_id) [MOE]
-# ---------------------------------------------------------------------------
-
-def moe_dot_fp64(codes, scales, g, ids, q, d) -> np.ndarray:
-    """y[t, j, n] = sum_k w_{ids[t, j]}[n, k] * a[t, k] in fp64,
-    fp64 [T, top_k, N].
-
-    codes [E, N, K/2], scales [E, N, K/16], g [E] (one per-tensor scale per
-    expert), ids int [T, top_k] (expert of each slot, every id in 0..E-1),
-    q [T, K], d [T, K/32]: each token is multiplied by the matrices of its
-    selected experts with the plain dot_fp64.
-    Pinned by tests/test_oracle_moe.py.
-    """
-    codes = np.asarray(codes)
-    scales = np.asarray(scales)
-    g = np.asarray(g, dtype=np.float32)
-    ids = np.asarray(ids)
-    T, top_k = ids.shape
-    E, N = codes.shape[0], codes.shape[1]
-    if np.any(ids < 0) or np.any(ids >= E):
-        raise ValueError("expert id out of range")
-    y = np.empty((T, top_k, N), dtype=np.float64)
-    for t in range(T):
-        for j in range(top_k):
-            e = int(ids[t, j])
-            y[t, j] = dot_fp64(codes[e], scales[e], g[e], q[t:t + 1], d[t:t + 1])[0]
-    return y

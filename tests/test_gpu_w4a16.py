@@ -7,7 +7,7 @@ weights), against the oracle's dot_fp64_f16:
   1.5B-class decoder (hidden 1536, 256-wide key/value, MLP 8960);
 * a decode-sweep shape at full size, sampled rows;
 * activations near the fp16 maximum, fp16 subnormals and zero tokens;
-* fp32 outputs: |y - y_ref| <= 1e-5 * sum over subblocks |sum w*x| + 1e-6.
+* fp32 outputs: |y - y_ref| <= 1e-5 * sum_k |w*x| + 1e-6 per element.
 """
 import numpy as np
 import pytest
