@@ -441,3 +441,33 @@ def sum_abs_terms_f16(codes, scales, g, x_bits, row_chunk: int = 1024) -> np.nda
         w = np.abs(dequantize_weights(codes[n0:n1], scales[n0:n1], g))
         out[:, n0:n1] = a @ w.T
     return out
+
+
+# ---------------------------------------------------------------------------
+# Mixture-of-experts product (mul_mat_id) [MOE]
+# ---------------------------------------------------------------------------
+
+def moe_dot_fp64(codes, scales, g, ids, q, d) -> np.ndarray:
+    """y[t, j, n] = sum_k w_{ids[t, j]}[n, k] * a[t, k] in fp64,
+    fp64 [T, top_k, N].
+
+    codes [E, N, K/2], scales [E, N, K/16], g [E] (one per-tensor scale per
+    expert), ids int [T, top_k] (expert of each slot, every id in 0..E-1),
+    q [T, K], d [T, K/32]: each token is multiplied by the matrices of its
+    selected experts with the plain dot_fp64.
+    Pinned by tests/test_oracle_moe.py.
+    """
+    codes = np.asarray(codes)
+    scales = np.asarray(scales)
+    g = np.asarray(g, dtype=np.float32)
+    ids = np.asarray(ids)
+    T, top_k = ids.shape
+    E, N = codes.shape[0], codes.shape[1]
+    if np.any(ids < 0) or np.any(ids >= E):
+        raise ValueError("expert id out of range")
+    y = np.empty((T, top_k, N), dtype=np.float64)
+    for t in range(T):
+        for j in range(top_k):
+            e = int(ids[t, j])
+            y[t, j] = dot_fp64(codes[e], scales[e], g[e], q[t:t + 1], d[t:t + 1])[0]
+    return y
