@@ -34,6 +34,12 @@ What it computes, and the passages it follows
            row dot inside a mixture-of-experts product (mul_mat_id: K = 2048,
            256 experts, 6 active per token), each token multiplied by the
            weight matrices of the experts its routing selects.
+[NVF4]     NVFP4 on both operands (the Blackwell NVFP4 tensor-core engines
+           of "TKintegers K5 ..." and the NVFP4 serving rows of the
+           protolabsai lab-benchmarks card): the activations in the weights'
+           format, E2M1 codes with one UE4M3 scale per 16, and (reading: the
+           pages define NVFP4 only for weights) one fp32 scale per token
+           instead of per tensor.
 [OCP-MX]   OCP Microscaling Formats (MX) v1.0: the E2M1 element type (1 sign,
            2 exponent bits with bias 1, 1 mantissa bit; max 6) and the E4M3
            type (4 exponent bits with bias 7, 3 mantissa bits, max 448, S.1111.111
@@ -73,6 +79,7 @@ __all__ = [
     "dot_fp64", "subblock_sums", "subblock_sums_biased", "bsum16",
     "y_from_subblock_sums", "sum_abs_terms", "tolerance",
     "dot_fp64_f16", "sum_abs_terms_f16", "moe_dot_fp64",
+    "quantize_act_nvfp4", "dot_fp64_nvf4", "sum_abs_terms_nvf4",
     "ACC_REL_TOL", "ACC_ABS_TOL",
 ]
 
@@ -471,3 +478,45 @@ def moe_dot_fp64(codes, scales, g, ids, q, d) -> np.ndarray:
             e = int(ids[t, j])
             y[t, j] = dot_fp64(codes[e], scales[e], g[e], q[t:t + 1], d[t:t + 1])[0]
     return y
+
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 activations, NVFP4 x NVFP4 product [NVF4]
+# ---------------------------------------------------------------------------
+
+def quantize_act_nvfp4(x):
+    """NVFP4 activations: each token row packed with the weight recipe
+    (pack_nvfp4) and its own fp32 scale g[m] = amax(|x[m]|) / (6*448).
+    Returns codes uint8 [M, K/2], scales uint8 [M, K/16], g float32 [M].
+    Pinned by tests/test_oracle_nvf4.py (and pack_nvfp4's own pins)."""
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 16), np.uint8)
+    g = np.empty(M, np.float32)
+    for m in range(M):
+        codes[m], scales[m], g[m] = pack_nvfp4(x[m:m + 1])
+    return codes, scales, g
+
+
+def dot_fp64_nvf4(w_codes, w_scales, w_g, a_codes, a_scales, a_g) -> np.ndarray:
+    """y[m, n] = sum_k w[n, k] * a[m, k] in fp64, fp64 [M, N], with both
+    operands NVFP4: w = w_g * UE4M3 * E2M1 (one tensor scale), a[m] = a_g[m] *
+    UE4M3 * E2M1 (one scale per token).  Every dequantised value is exact in
+    fp64; the matrix product is a library primitive.
+    Pinned by tests/test_oracle_nvf4.py."""
+    a = np.stack([dequantize_weights(a_codes[m:m + 1], a_scales[m:m + 1], a_g[m])[0]
+                  for m in range(np.asarray(a_codes).shape[0])])
+    w = dequantize_weights(w_codes, w_scales, w_g)
+    return a @ w.T
+
+
+def sum_abs_terms_nvf4(w_codes, w_scales, w_g, a_codes, a_scales, a_g) -> np.ndarray:
+    """sum|terms|[m, n] = sum_k |w[n, k] * a[m, k]|, fp64 [M, N]: the scale
+    of the accuracy bound of the NVFP4 x NVFP4 product (its terms are the
+    products; there are no integer sums)."""
+    a = np.stack([dequantize_weights(a_codes[m:m + 1], a_scales[m:m + 1], a_g[m])[0]
+                  for m in range(np.asarray(a_codes).shape[0])])
+    w = dequantize_weights(w_codes, w_scales, w_g)
+    return np.abs(a) @ np.abs(w).T
