@@ -446,13 +446,16 @@ __device__ __forceinline__ void next_stage(const RegGroup& grp, int& gr, int r_e
   gr += nrows;
 }
 
-template <int NPL, int WPR, bool ISUM>
+template <int NPL, int WPR, bool ISUM, bool MOE>
 __global__ void __launch_bounds__(kM1Threads, 1)
 gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_constant__ MoeArgs moe,
                    int K, const int8_t* __restrict__ q_all, const __half* __restrict__ d_all,
                    int32_t* __restrict__ isum) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ RegGroup grp;
+  // the matrices: from the launch parameters, or (mixture of experts) built
+  // in shared memory from the routing ids
+  __shared__ RegGroup moe_grp;
+  const RegGroup& grp = MOE ? moe_grp : grp_param;
   // token of this grid row (several only for mixture-of-experts launches)
   const int8_t* __restrict__ q = q_all + static_cast<size_t>(blockIdx.y) * K;
   const __half* __restrict__ d = d_all + static_cast<size_t>(blockIdx.y) * (K / 32);
@@ -472,8 +475,7 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
   const int G = gridDim.x;
 
   grid_dependents_launch();
-  const bool is_moe = moe.ids != nullptr;
-  if (is_moe) {
+  if constexpr (MOE) {
     // the routing ids come from the previous kernel
     grid_dependency_wait();
     if (threadIdx.x == 0) {
@@ -493,13 +495,12 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
         m.N = moe.N;
         m.row_off = rows;
         rows += moe.N;
-        grp.m[cnt++] = m;
+        moe_grp.m[cnt++] = m;
       }
-      grp.count = cnt;
-      grp.rows = rows;
+      moe_grp.count = cnt;
+      moe_grp.rows = rows;
     }
   } else {
-    if (threadIdx.x == 0) grp = grp_param;
     for (int i = threadIdx.x; i < reg_block_slots(grp_param.rows, G); i += blockDim.x) scnt[i] = 0;
   }
   if (threadIdx.x == 0) {
@@ -910,7 +911,7 @@ cudaError_t launch_m1(const uint8_t* codes, const uint8_t* scales, float g, int6
 template <int NPL, int WPR, bool ISUM>
 cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const uint16_t* d,
                           int32_t* isum, cudaStream_t stream) {
-  auto kernel = gemv_m1_reg_kernel<NPL, WPR, ISUM>;
+  auto kernel = gemv_m1_reg_kernel<NPL, WPR, ISUM, false>;
   static SmemAttrOnce attr;
   cudaError_t e = attr.ensure(kernel, static_cast<int>(kRegDynSmemMax));
   if (e != cudaSuccess) return e;
@@ -936,7 +937,7 @@ cudaError_t launch_m1_reg(const RegGroup& grp, int64_t K, const int8_t* q, const
 template <int NPL, int WPR>
 cudaError_t launch_moe_reg(const MoeArgs& moe, int64_t T, int64_t K, const int8_t* q,
                            const uint16_t* d, cudaStream_t stream) {
-  auto kernel = gemv_m1_reg_kernel<NPL, WPR, false>;
+  auto kernel = gemv_m1_reg_kernel<NPL, WPR, false, true>;
   static SmemAttrOnce attr;
   cudaError_t e = attr.ensure(kernel, static_cast<int>(kRegDynSmemMax));
   if (e != cudaSuccess) return e;
