@@ -56,6 +56,9 @@ SIGNATURES = {
                                       _vp, ctypes.c_size_t, _vp]),
     "nvq_gemm": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                 _c_i64, _vp, _vp, ctypes.c_size_t, _vp]),
+    "nvq_quantize_act_nvfp4": (ctypes.c_int, [_vp, _c_i64, _c_i64, _vp, _vp, _vp, _vp]),
+    "nvq_gemm_nvf4": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp, _vp,
+                                     _c_i64, _vp, _vp]),
     "nvq_gemm_noalloc": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp, _vp,
                                         _c_i64, _vp, _vp]),
     "nvq_debug_subblock_sums": (ctypes.c_int, [_vp, _vp, ctypes.c_float, _c_i64, _c_i64, _vp,
@@ -235,6 +238,33 @@ def gemm_w4a16(codes: torch.Tensor, scales: torch.Tensor, g: float, x: torch.Ten
     _check("nvq_gemm_w4a16", _lib.nvq_gemm_w4a16(
         _ptr(codes), _ptr(scales), float(g), N, K, _ptr(x), M, _ptr(y), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y
+
+
+def quantize_act_nvfp4(x: torch.Tensor, stream=None):
+    """NVFP4 activations (nvq_quantize_act_nvfp4): x float32 [M, K] on the
+    device; returns (codes uint8 [M, K/2], scales uint8 [M, K/16], g float32 [M])."""
+    M, K = x.shape
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // 16), dtype=torch.uint8, device=x.device)
+    g = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check("nvq_quantize_act_nvfp4", _lib.nvq_quantize_act_nvfp4(
+        _ptr(x), M, K, _ptr(codes), _ptr(scales), _ptr(g), _stream(stream)))
+    return codes, scales, g
+
+
+def gemm_nvf4(w_codes: torch.Tensor, w_scales: torch.Tensor, g_w: float, a_codes: torch.Tensor,
+              a_scales: torch.Tensor, a_g: torch.Tensor, y: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """NVFP4 weights x NVFP4 activations (nvq_gemm_nvf4) on the block-scaled
+    FP4 tensor-core path; returns y fp32 [M, N]."""
+    N = w_codes.shape[0]
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=a_codes.device)
+    _check("nvq_gemm_nvf4", _lib.nvq_gemm_nvf4(
+        _ptr(w_codes), _ptr(w_scales), float(g_w), N, K, _ptr(a_codes), _ptr(a_scales),
+        _ptr(a_g), M, _ptr(y), _stream(stream)))
     return y
 
 

@@ -1,0 +1,526 @@
+// NVFP4 x NVFP4: NVFP4 activations and the product on the tensor core's
+// native block-scaled FP4 path (tcgen05.mma.kind::mxf4nvf4.block_scale with
+// one UE4M3 scale per 16 elements on both operands).
+//
+// The NVFP4 serving engines that "TKintegers K5: 3.21x prefill and 3.10x
+// decode throughput vs TorchAO FP8 on NVIDIA L4" links to, and the NVFP4
+// rows of the protolabsai lab-benchmarks card, run both operands in the
+// weights' 4-bit format.  Here the activations take the weight recipe with
+// one fp32 scale per token: g[m] = amax(|x[m]|)/(6*448); per 16 elements
+// s = UE4M3(amax_blk/(6*g)); code = E2M1(x/(g*s)), round to nearest, ties
+// to even, saturating, a zero magnitude stored as +0.
+//
+// The product needs no decode: the packed codes go from HBM to shared
+// memory by TMA exactly as stored (two E2M1 per byte, element 2i in the low
+// nibble), the tensor core reads them there, and the per-16 scales, copied
+// into tensor memory (lane = row, one 32-bit column per 64-wide K step,
+// byte j for K block j), are applied inside the MMA.  Every product of two
+// E2M1 values and two UE4M3 scales is exact in fp32; the accumulation is
+// fp32, promoted to registers every 1024 K; y = g_w * g_a[m] * sum.
+//
+// gemm_nvf4_kernel: one CTA per (128 weight rows, 128 tokens) tile.
+//   warp 0     TMA: per 256-wide K stage the 128 x 128-byte code tiles of
+//              weights and tokens (128-byte swizzle) and their 128 x 16-byte
+//              scale tiles, into a 4-deep ring;
+//   warp 1     allocates tensor memory; issues 4 block-scaled MMAs per stage
+//              (M = 128 weight rows, N = 128 tokens, K = 64);
+//   warps 2-5  (one per tensor-memory lane quarter) copy each stage's scales
+//              to tensor memory with tcgen05.st;
+//   warps 2-9  drain finished 1024-wide K chunks into fp32 registers (two
+//              warps per lane quarter, 64 token columns each) and store y.
+// Every wait is bounded (4 s): a timeout raises the GEMM error flag and the
+// CTA drains what it issued before freeing tensor memory.
+#include <algorithm>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+
+#include "nvq_device.cuh"
+#include "nvq_internal.h"
+#include "tcgen05.cuh"
+
+namespace nvq {
+namespace {
+
+// ---------------------------------------------------------------------------
+// NVFP4 activation quantiser (one CTA per token row)
+// ---------------------------------------------------------------------------
+constexpr int kQThreads = 256;
+
+// UE4M3 byte nearest to r >= 0 (ties to the even code), saturating at
+// 0x7E = 448.  Bytes 0..7 are m * 2^-9 and byte 8e + m (e >= 1) is
+// (8 + m) * 2^(e-10): inside exponent e the code is (e-1)*8 + rint(r*2^(10-e)).
+__device__ __forceinline__ uint32_t ue4m3_encode(float r) {
+  if (!(r > 0.0f)) return 0;
+  if (r >= 448.0f) return 0x7E;
+  int ex = 0;
+  frexpf(r, &ex);                 // r = f * 2^ex, f in [0.5, 1)
+  int e = ex + 6;
+  if (e < 1) e = 1;
+  const int n = __float2int_rn(ldexpf(r, 10 - e));   // exact scaling, rint half-even
+  const int code = (e - 1) * 8 + n;
+  return static_cast<uint32_t>(code > 0x7E ? 0x7E : code);
+}
+__device__ __forceinline__ float ue4m3_value(uint32_t b) {
+  const int e = (b >> 3) & 0xF;
+  const int m = b & 0x7;
+  return e == 0 ? ldexpf(static_cast<float>(m), -9) : ldexpf(static_cast<float>(8 + m), e - 10);
+}
+// E2M1 code nearest to x (ties to the even code), saturating at 6; the
+// magnitudes 0, .5, 1, 1.5 | 2, 3 | 4, 6 have spacings 0.5, 1 and 2, so the
+// codes are rint(2|x|), rint(|x|) + 2 and rint(|x|/2) + 4 there.
+__device__ __forceinline__ uint32_t e2m1_encode(float x) {
+  const float a = fabsf(x);
+  int code;
+  if (a >= 6.0f)
+    code = 7;
+  else if (a < 2.0f)
+    code = __float2int_rn(a * 2.0f);
+  else if (a < 4.0f)
+    code = __float2int_rn(a) + 2;
+  else
+    code = __float2int_rn(a * 0.5f) + 4;
+  if (code != 0 && x < 0.0f) code |= 0x8;
+  return static_cast<uint32_t>(code);
+}
+
+__global__ void __launch_bounds__(kQThreads)
+quantize_nvfp4_kernel(const float* __restrict__ x, int K, uint8_t* __restrict__ codes,
+                      uint8_t* __restrict__ scales, float* __restrict__ g_out) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = blockIdx.x;
+  const float* xr = x + static_cast<size_t>(row) * K;
+  __shared__ float red[kQThreads / 32];
+  float a = 0.0f;
+  for (int i = threadIdx.x; i < K / 4; i += kQThreads) {
+    const float4 v = reinterpret_cast<const float4*>(xr)[i];
+    a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  float amax = red[0];
+#pragma unroll
+  for (int i = 1; i < kQThreads / 32; ++i) amax = fmaxf(amax, red[i]);
+  const float g = __fdiv_rn(amax, 2688.0f);
+  const float six_g = __fmul_rn(6.0f, g);
+  if (threadIdx.x == 0) g_out[row] = g;
+  // one thread per 16-element subblock
+  for (int b = threadIdx.x; b < K / 16; b += kQThreads) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 t = reinterpret_cast<const float4*>(xr + 16 * b)[i];
+      v[4 * i] = t.x;
+      v[4 * i + 1] = t.y;
+      v[4 * i + 2] = t.z;
+      v[4 * i + 3] = t.w;
+    }
+    float ab = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(v[i]));
+    const float r = six_g > 0.0f ? __fdiv_rn(ab, six_g) : 0.0f;
+    const uint32_t s = ue4m3_encode(r);
+    const float gs = __fmul_rn(g, ue4m3_value(s));
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t c = gs > 0.0f ? e2m1_encode(__fdiv_rn(v[i], gs)) : 0u;
+      if (i < 8)
+        w0 |= c << (4 * i);
+      else
+        w1 |= c << (4 * (i - 8));
+    }
+    reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2))[b] = make_uint2(w0, w1);
+    scales[static_cast<size_t>(row) * (K / 16) + b] = static_cast<uint8_t>(s);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 x NVFP4 GEMM
+// ---------------------------------------------------------------------------
+constexpr int kTile = 128;                 // weight rows (MMA M) and tokens (MMA N) per CTA
+constexpr int kStageK = 256;               // K per stage: 128 code bytes per row
+constexpr int kMmaK = 64;                  // K per block-scaled MMA
+constexpr int kStages = 4;
+constexpr int kChunkStages = 4;            // stages per accumulator chunk (1024 K)
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr uint32_t kCodeTile = kTile * kStageK / 2;       // 16 KB
+constexpr uint32_t kScaleTile = kTile * kStageK / 16;     // 2 KB
+constexpr uint32_t kSlot = 2 * kCodeTile + 2 * kScaleTile;   // weights | tokens | w scales | t scales
+constexpr uint32_t kAccCols = kTile;                      // one accumulator: 128 fp32 columns
+constexpr uint32_t kSfCol0 = 2 * kAccCols;                // scale factors after the accumulators
+constexpr uint32_t kSfColsPerMma = kTile / 32;                 // 4 columns per operand
+constexpr uint32_t kSfColsPerOperand = (kStageK / kMmaK) * kSfColsPerMma;   // 16 per stage
+constexpr uint32_t kSfColsPerStage = 2 * kSfColsPerOperand;    // weights | tokens
+constexpr uint32_t kTmemCols = 512;
+static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory");
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// barriers: full[4] sf_full[4] empty[4] acc_full[2] acc_empty[2] mma_done
+constexpr int kNumBars = 3 * kStages + 5;
+constexpr uint32_t kSmemBytes = kStages * kSlot + kNumBars * 8 + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+// bit 0: a pipeline wait timed out
+__device__ unsigned int g_nvf4_error_flags = 0;
+
+// Instruction descriptor of kind::mxf4nvf4 with block scaling: A and B E2M1
+// (format 1), K-major, scale format E4M3 (bit 23 = 0), N >> 3 at bits
+// 17-22, M >> 4 at bits 24-28, scale-factor byte ids 0 (bits 4-5, 29-30),
+// dense K = 64 (bit 31 = 0).
+__host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+      "[%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
+                 const __grid_constant__ CUtensorMap wscale_map,
+                 const __grid_constant__ CUtensorMap acode_map,
+                 const __grid_constant__ CUtensorMap ascale_map, int N, int K, int M,
+                 float g_w, const float* __restrict__ g_a, float* __restrict__ y) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_addr(smem_raw);
+  const uint32_t sbase = raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* smem = smem_raw + (sbase - raw);
+  const uint32_t bars = sbase + kStages * kSlot;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto sf_full = [&](int s) { return bars + 8u * (kStages + s); };
+  auto empty = [&](int s) { return bars + 8u * (2 * kStages + s); };
+  auto acc_full = [&](int b) { return bars + 8u * (3 * kStages + b); };
+  auto acc_empty = [&](int b) { return bars + 8u * (3 * kStages + 2 + b); };
+  const uint32_t mma_done = bars + 8u * (kNumBars - 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kStages * kSlot + kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  auto slot = [&](int s) { return sbase + s * kSlot; };
+
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTile;          // weight rows
+  const int m0 = blockIdx.y * kTile;          // tokens
+  const int num_k = K / kStageK;
+  const int num_chunks = (num_k + kChunkStages - 1) / kChunkStages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(sf_full(s), 4);
+      ptx::mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(acc_full(b), 1);
+      ptx::mbar_init(acc_empty(b), kEpiWarps);
+    }
+    ptx::mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tensormap(&wcode_map);
+    ptx::prefetch_tensormap(&wscale_map);
+    ptx::prefetch_tensormap(&acode_map);
+    ptx::prefetch_tensormap(&ascale_map);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicOr(&g_nvf4_error_flags, 1u);
+  };
+  auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (__all_sync(0xffffffffu, ptx::mbar_try_wait(bar, parity))) return true;
+    const bool got = ptx::mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
+    return __all_sync(0xffffffffu, got);
+  };
+
+  if (warp == 0) {
+    // ------------------------------- TMA producer ------------------------------
+    // the weights are never written by the kernels before this one: the first
+    // slots' weight tiles are requested before waiting for the token tiles
+    const int early = min(num_k, kStages);
+    if (lane == 0) {
+      for (int k = 0; k < early; ++k) {
+        ptx::mbar_arrive_expect_tx(full(k), kSlot);
+        ptx::tma_load_2d(slot(k), &wcode_map, k * (kStageK / 2), n0, full(k));
+        ptx::tma_load_2d(slot(k) + 2 * kCodeTile, &wscale_map, k * (kStageK / 16), n0, full(k));
+      }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (lane == 0) {
+      for (int k = 0; k < early; ++k) {
+        ptx::tma_load_2d(slot(k) + kCodeTile, &acode_map, k * (kStageK / 2), m0, full(k));
+        ptx::tma_load_2d(slot(k) + 2 * kCodeTile + kScaleTile, &ascale_map, k * (kStageK / 16),
+                         m0, full(k));
+      }
+    }
+    __syncwarp();
+    int issued = early;
+    for (int k = early; k < num_k; ++k) {
+      const int s = k % kStages;
+      if (!warp_wait(empty(s), ((k / kStages) & 1) ^ 1)) {
+        fail();
+        break;
+      }
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(full(s), kSlot);
+        ptx::tma_load_2d(slot(s), &wcode_map, k * (kStageK / 2), n0, full(s));
+        ptx::tma_load_2d(slot(s) + kCodeTile, &acode_map, k * (kStageK / 2), m0, full(s));
+        ptx::tma_load_2d(slot(s) + 2 * kCodeTile, &wscale_map, k * (kStageK / 16), n0, full(s));
+        ptx::tma_load_2d(slot(s) + 2 * kCodeTile + kScaleTile, &ascale_map, k * (kStageK / 16), m0,
+                         full(s));
+      }
+      __syncwarp();
+      ++issued;
+    }
+    if (*abort_flag) {
+      for (int k = max(0, issued - kStages); k < issued; ++k)
+        ptx::mbar_wait_bounded(full(k % kStages), (k / kStages) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // -------------------------------- MMA issuer -------------------------------
+    constexpr uint32_t idesc = idesc_nvf4(kTile, kTile);
+    bool ok = true;
+    for (int c = 0; c < num_chunks && ok; ++c) {
+      const int b = c & 1;
+      if (c >= 2 && !warp_wait(acc_empty(b), ((c >> 1) - 1) & 1)) {
+        fail();
+        break;
+      }
+      const uint32_t d_tmem = tmem_base + b * kAccCols;
+      const int k_end = min(num_k, (c + 1) * kChunkStages);
+      for (int k = c * kChunkStages; k < k_end; ++k) {
+        const int s = k % kStages;
+        if (!warp_wait(sf_full(s), (k / kStages) & 1)) {
+          fail();
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          ptx::tc_fence_after();
+          const uint64_t adesc0 = ptx::sw128_kmajor_desc(slot(s));
+          const uint64_t bdesc0 = ptx::sw128_kmajor_desc(slot(s) + kCodeTile);
+          const uint32_t sf = tmem_base + kSfCol0 + s * kSfColsPerStage;
+#pragma unroll
+          for (int j = 0; j < kStageK / kMmaK; ++j) {
+            // 64 E2M1 = 32 bytes per K step inside the 128-byte swizzled rows
+            mma_nvf4(d_tmem, adesc0 + 2u * j, bdesc0 + 2u * j, idesc, sf + kSfColsPerMma * j,
+                     sf + kSfColsPerOperand + kSfColsPerMma * j,
+                     (k == c * kChunkStages && j == 0) ? 0u : 1u);
+          }
+          ptx::mma_commit(empty(s));
+          if (k == k_end - 1) ptx::mma_commit(acc_full(b));
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) ptx::mma_commit(mma_done);
+    __syncwarp();
+    ptx::mbar_wait_bounded(mma_done, 0, nullptr, kWaitLimitNs);
+  } else {
+    // ------------- scale factors to tensor memory; then the epilogue -----------
+    const int q = warp & 3;                   // lane quarter
+    const int half = (warp - 2) >> 2;         // token columns [64*half, 64*half + 64)
+    const int r = q * 32 + lane;              // weight row of the accumulator lane
+    const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
+    const bool mover = half == 0;
+    float run[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) run[i] = 0.0f;
+    int drained = 0;
+    auto drain = [&]() -> bool {
+      const int b = drained & 1;
+      if (!warp_wait(acc_full(b), (drained >> 1) & 1)) return false;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t v[32];
+        ptx::tmem_ld_32cols(tmem_base + tlane + b * kAccCols + 64 * half + 32 * cc, v);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) run[32 * cc + i] += __uint_as_float(v[i]);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(acc_empty(b));
+      ++drained;
+      return true;
+    };
+    bool ok = true;
+    for (int k = 0; k < num_k && ok; ++k) {
+      if (k % kChunkStages == 0 && k / kChunkStages >= 2) {
+        if (!drain()) {
+          fail();
+          ok = false;
+          break;
+        }
+      }
+      if (!mover) continue;
+      const int s = k % kStages;
+      if (!warp_wait(full(s), (k / kStages) & 1)) {
+        fail();
+        ok = false;
+        break;
+      }
+      // this lane's column j of K step t: word t of the 16 scale bytes of
+      // row 32*j + lane (the same in every lane quarter)
+      uint32_t va[16], vb[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 a4 = lds128(slot(s) + 2 * kCodeTile + 16u * (32 * j + lane));
+        const uint4 b4 = lds128(slot(s) + 2 * kCodeTile + kScaleTile + 16u * (32 * j + lane));
+        va[j] = a4.x, va[4 + j] = a4.y, va[8 + j] = a4.z, va[12 + j] = a4.w;
+        vb[j] = b4.x, vb[4 + j] = b4.y, vb[8 + j] = b4.z, vb[12 + j] = b4.w;
+      }
+      ptx::tc_fence_after();
+      const uint32_t sf = tmem_base + tlane + kSfCol0 + s * kSfColsPerStage;
+      ptx::tmem_st_16cols(sf, va);
+      ptx::tmem_st_16cols(sf + kSfColsPerOperand, vb);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(sf_full(s));
+    }
+    while (ok && drained < num_chunks) {
+      if (!drain()) {
+        fail();
+        ok = false;
+      }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (ok) {
+      const int n = n0 + r;
+      if (n < N) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int m = m0 + 64 * half + i;
+          if (m < M) y[static_cast<size_t>(m) * N + n] = run[i] * (g_w * g_a[m]);
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_bytes_2d(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t rows,
+                     uint32_t box_bytes, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = encoder();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+cudaLaunchAttribute pdl_attr() {
+  cudaLaunchAttribute a = {};
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_nvfp4(const float* x, int64_t M, int64_t K, uint8_t* codes,
+                                  uint8_t* scales, float* g, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(M));
+  cfg.blockDim = dim3(kQThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_nvfp4_kernel, x, static_cast<int>(K), codes, scales, g);
+}
+
+cudaError_t launch_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w,
+                             int64_t N, int64_t K, const uint8_t* a_codes,
+                             const uint8_t* a_scales, const float* g_a, int64_t M, float* y,
+                             cudaStream_t stream) {
+  CUtensorMap wc, ws, ac, as;
+  if (!encode_bytes_2d(&wc, w_codes, K / 2, N, 128, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bytes_2d(&ws, w_scales, K / 16, N, 16, kTile, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_bytes_2d(&ac, a_codes, K / 2, M, 128, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bytes_2d(&as, a_scales, K / 16, M, 16, kTile, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  static SmemAttrOnce attr;
+  cudaError_t e = attr.ensure(gemm_nvf4_kernel, static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((N + kTile - 1) / kTile),
+                     static_cast<unsigned>((M + kTile - 1) / kTile));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute a[1] = {pdl_attr()};
+  cfg.attrs = a;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_nvf4_kernel, wc, ws, ac, as, static_cast<int>(N),
+                            static_cast<int>(K), static_cast<int>(M), g_w, g_a, y);
+}
+
+cudaError_t nvf4_error_flags(bool clear, unsigned int* flags) {
+  cudaError_t e = cudaMemcpyFromSymbol(flags, g_nvf4_error_flags, sizeof(unsigned int));
+  if (e == cudaSuccess && clear) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_nvf4_error_flags, &zero, sizeof(zero));
+  }
+  return e;
+}
+
+}  // namespace nvq

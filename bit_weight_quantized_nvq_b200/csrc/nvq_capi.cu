@@ -282,6 +282,40 @@ nvq_status nvq_gemm_w4a16(const uint8_t* codes, const uint8_t* scales, float g, 
                                                 static_cast<cudaStream_t>(stream)));
 }
 
+nvq_status nvq_quantize_act_nvfp4(const float* x, int64_t M, int64_t K, uint8_t* codes,
+                                  uint8_t* scales, float* g, void* stream) {
+  if (M < 0 || K < 0) return NVQ_ERR_INVALID_ARG;
+  if (K % 16 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (M == 0 || K == 0) return NVQ_OK;
+  if (M > INT32_MAX || K > (int64_t{1} << 30)) return NVQ_ERR_BAD_SHAPE;
+  if (!x || !codes || !scales || !g) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(g))
+    return NVQ_ERR_MISALIGNED;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_quantize_nvfp4(x, M, K, codes, scales, g,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+nvq_status nvq_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w, int64_t N,
+                         int64_t K, const uint8_t* a_codes, const uint8_t* a_scales,
+                         const float* a_g, int64_t M, float* y, void* stream) {
+  if (N < 0 || K < 0 || M < 0) return NVQ_ERR_INVALID_ARG;
+  if (K == 0 || K % 256 != 0) return NVQ_ERR_BAD_SHAPE;
+  if (K > (int64_t{1} << 30) || N > INT32_MAX || M > int64_t{65535} * 128)
+    return NVQ_ERR_BAD_SHAPE;
+  if (!(g_w == g_w)) return NVQ_ERR_INVALID_ARG;
+  if (N == 0 || M == 0) return NVQ_OK;
+  if (!w_codes || !w_scales || !a_codes || !a_scales || !a_g || !y) return NVQ_ERR_INVALID_ARG;
+  if (!aligned16(w_codes) || !aligned16(w_scales) || !aligned16(a_codes) ||
+      !aligned16(a_scales) || !aligned16(a_g) || !aligned16(y))
+    return NVQ_ERR_MISALIGNED;
+  nvq_status st = check_device();
+  if (st != NVQ_OK) return st;
+  return cuda_status(nvq::launch_gemm_nvf4(w_codes, w_scales, g_w, N, K, a_codes, a_scales, a_g,
+                                           M, y, static_cast<cudaStream_t>(stream)));
+}
+
 nvq_status nvq_debug_subblock_sums(const uint8_t* codes, const uint8_t* scales, float g,
                                    int64_t N, int64_t K, const int8_t* q, const uint16_t* d,
                                    int64_t M, float* y, int32_t* isum, void* stream) {
@@ -301,11 +335,12 @@ nvq_status nvq_error_flags(unsigned int* flags, int clear) {
   if (!flags) return NVQ_ERR_INVALID_ARG;
   nvq_status st = check_device();
   if (st != NVQ_OK) return st;
-  unsigned int gemv = 0, gemm = 0, gemm_small = 0;
+  unsigned int gemv = 0, gemm = 0, gemm_small = 0, nvf4 = 0;
   cudaError_t e = nvq::gemv_error_flags(clear != 0, &gemv);
   if (e == cudaSuccess) e = nvq::gemm_error_flags(clear != 0, &gemm);
   if (e == cudaSuccess) e = nvq::gemm_small_error_flags(clear != 0, &gemm_small);
-  gemm |= gemm_small;
+  if (e == cudaSuccess) e = nvq::nvf4_error_flags(clear != 0, &nvf4);
+  gemm |= gemm_small | nvf4;
   if (e != cudaSuccess) {
     cudaGetLastError();
     return cuda_status(e);

@@ -86,6 +86,17 @@ cudaError_t gemm_small_error_flags(bool clear, unsigned int* flags);
 cudaError_t launch_gemm_small_f16(const uint8_t* codes, const uint8_t* scales, float g,
                                   int64_t N, int64_t K, const uint16_t* x, int64_t M, float* y,
                                   void* workspace, cudaStream_t stream);
+// NVFP4 activations: per token row g[m] = amax/2688 and the weight recipe
+// (codes [M, K/2], scales [M, K/16]), K % 16 == 0.
+cudaError_t launch_quantize_nvfp4(const float* x, int64_t M, int64_t K, uint8_t* codes,
+                                  uint8_t* scales, float* g, cudaStream_t stream);
+// NVFP4 weights x NVFP4 activations on the block-scaled FP4 tensor-core path,
+// y [M, N] fp32, K % 256 == 0.
+cudaError_t launch_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w,
+                             int64_t N, int64_t K, const uint8_t* a_codes,
+                             const uint8_t* a_scales, const float* g_a, int64_t M, float* y,
+                             cudaStream_t stream);
+cudaError_t nvf4_error_flags(bool clear, unsigned int* flags);
 // The two halves of launch_gemm for the large-token schedule: expand Q8_0 activations into the
 // workspace, then run the tensor-core GEMM on an expanded workspace (which
 // several weight matrices with the same K may share).

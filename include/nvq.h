@@ -278,6 +278,52 @@ nvq_status nvq_gemm_w4a16(const uint8_t* codes, const uint8_t* scales, float g, 
                           size_t workspace_bytes, void* stream);
 
 /*
+ * nvq_quantize_act_nvfp4 - fp32 activations to NVFP4, one fp32 scale per
+ * token: the operand of nvq_gemm_nvf4.  The NVFP4 x NVFP4 engines that
+ * "TKintegers K5: 3.21x prefill and 3.10x decode throughput vs TorchAO FP8
+ * on NVIDIA L4" points to (and the NVFP4 rows of the lab-benchmarks card)
+ * quantise activations to the weights' 4-bit format; this library takes the
+ * weight recipe of nvq_pack_nvfp4 row by row:
+ *   g[m] = amax(|x[m, :]|) / 2688;  per 16 elements s = UE4M3(amax_blk/(6 g[m]));
+ *   code = E2M1(x / (g[m] * s)),
+ * fp32 with one IEEE rounding per operation, round to nearest with ties to
+ * the even code, saturating; a zero magnitude is stored as +0 and a
+ * subblock whose 6*g or g*s is 0 stores codes 0.
+ * x       device fp32 [M, K] row-major, finite.
+ * codes   device uint8 [M, K/2] out: element 2i in the low nibble of byte i.
+ * scales  device uint8 [M, K/16] out; g device fp32 [M] out.
+ * Requires K % 16 == 0 (NVQ_ERR_BAD_SHAPE).  Results are bit-identical to
+ * nvq_pack_nvfp4 applied to each row on its own.
+ * Errors: NVQ_ERR_INVALID_ARG, NVQ_ERR_BAD_SHAPE, NVQ_ERR_MISALIGNED,
+ * NVQ_ERR_UNSUPPORTED_DEVICE, NVQ_ERR_CUDA.
+ */
+nvq_status nvq_quantize_act_nvfp4(const float* x, int64_t M, int64_t K, uint8_t* codes,
+                                  uint8_t* scales, float* g, void* stream);
+
+/*
+ * nvq_gemm_nvf4 - NVFP4 weights times NVFP4 activations on the tensor
+ * core's block-scaled FP4 path (tcgen05.mma kind::mxf4nvf4, one UE4M3 scale
+ * per 16 elements on both operands):
+ *   y[m, n] = g_w * a_g[m] * sum_k (s_w E2M1_w)[n, k] * (s_a E2M1_a)[m, k].
+ * w_codes/w_scales/g_w  weights as nvq_pack_nvfp4 writes them ([N, K/2],
+ *                       [N, K/16], tensor scale).
+ * a_codes/a_scales/a_g  activations as nvq_quantize_act_nvfp4 writes them
+ *                       ([M, K/2], [M, K/16], fp32 [M]).
+ * y                     device fp32 [M, N] out.
+ * Every product of two E2M1 values and two UE4M3 scales is exact in fp32;
+ * the sums accumulate in fp32 in tensor memory and are promoted to fp32
+ * registers every 1024 K.  Accuracy: |y - exact| <= 1e-5 * sum_k |w*a| +
+ * 1e-6 per element, exact being the fp64 product of the dequantised
+ * operands.
+ * Requires K % 256 == 0, 1 <= M <= 65535*128 (NVQ_ERR_BAD_SHAPE); any N.
+ * No workspace.  Errors: as nvq_gemm; a pipeline wait that gives up raises
+ * NVQ_FLAG_GEMM_TIMEOUT.
+ */
+nvq_status nvq_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w, int64_t N,
+                         int64_t K, const uint8_t* a_codes, const uint8_t* a_scales,
+                         const float* a_g, int64_t M, float* y, void* stream);
+
+/*
  * nvq_gemm_noalloc - nvq_gemm for callers that cannot allocate device memory
  * and cannot hand the library a workspace.  (An addition of this library;
  * the web pages describing the method have no counterpart.)
