@@ -26,6 +26,11 @@ workload under ``"workloads"``, each measured the same way):
   stack_prefill           the same stack for 2048 tokens.
   w4a16_decode            the decode-sweep shapes at one token with fp16
                           activations (nvq_gemm_w4a16).  Metric: weight GB/s.
+  nvf4_prefill_m{256,2048} NVFP4 activations (nvq_quantize_act_nvfp4) and the
+                          block-scaled FP4 tensor-core GEMM (nvq_gemm_nvf4)
+                          over the prefill shapes.  Metric: TFLOP/s 2*M*N*K,
+                          against the FP4 dense peak (measured bf16 x 4, the
+                          nominal FP4/bf16 ratio).
   moe_decode              mixture-of-experts decode (mul_mat_id): 16 tokens,
                           each times 6 of 256 experts (K = 2048, N = 1536),
                           a different seeded routing every step.  Metric:
@@ -90,7 +95,7 @@ WEIGHT_BYTES_PER_ELEMENT = 0.5625       # 4-bit code + one UE4M3 byte per 16
 L2_BYTES = 126e6
 SUB_WORKLOADS = ["gemv_4096", "small_batch_m2", "small_batch_m4", "small_batch_m8",
                  "small_batch_m16", "prefill_m256", "prefill_m2048", "stack_decode",
-                 "stack_prefill", "moe_decode", "w4a16_decode"]
+                 "stack_prefill", "moe_decode", "w4a16_decode", "nvf4_prefill_m2048"]
 
 
 # ---------------------------------------------------------------------------
@@ -262,9 +267,15 @@ def oracle_task(task):
     """Run one oracle task, (codes, scales, g, x, reps, units) -> units: the
     oracle's Q8_0 quantisation of x, then its fp64 dequantise-then-dot of the
     weight block, `reps` times (x given as fp16 bit patterns, uint16: the
-    fp16-activation dot instead)."""
+    fp16-activation dot instead; x = ("nvf4", fp32 x): the oracle's NVFP4
+    activation quantiser and the NVFP4 x NVFP4 dot)."""
     import oracle as o
     codes, scales, g, x, reps, units = task
+    if isinstance(x, tuple):              # ("nvf4", fp32 x): NVFP4 activations
+        ac, as_, ag = o.quantize_act_nvfp4(x[1])
+        for _ in range(reps):
+            o.dot_fp64_nvf4(codes, scales, g, ac, as_, ag)
+        return units
     if x.dtype == np.uint16:
         for _ in range(reps):
             o.dot_fp64_f16(codes, scales, g, x)
@@ -567,6 +578,79 @@ class GemmWorkload(GemvWorkload):
                 "fp64 dequantise-then-dot")
 
 
+class Nvf4GemmWorkload(GemmWorkload):
+    """Prefill on the block-scaled FP4 path: NVFP4 quantisation of M tokens
+    (nvq_quantize_act_nvfp4) and nvq_gemm_nvf4 for each shape."""
+
+    kernel = "gemm_nvf4"
+    sources = ("nvf4.cu", "tcgen05.cuh")
+    metric = "nvfp4_nvfp4_prefill_gemm_TFLOPs"
+    peak_scale = 4.0
+    peak_note = "bf16_tflops (burst) x 4, the nominal dense FP4/bf16 ratio (9 / 2.25 PFLOP/s)"
+
+    def setup(self, device):
+        import torch
+        GemvWorkload.setup(self, device)
+        for c in self.cases:
+            M, K = self.M, c["K"]
+            c["ac"] = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+            c["as"] = torch.empty((M, K // 16), dtype=torch.uint8, device=device)
+            c["ag"] = torch.empty((M,), dtype=torch.float32, device=device)
+            del c["q"], c["d"]
+            self.capi.quantize_act_nvfp4(c["x"])      # library warm (tensor maps, attributes)
+
+    def config(self):
+        cfg = super().config()
+        cfg["activations"] = ("fp32 N(0,1), 0.1% channels x50 -> NVFP4 (per-token fp32 scale) "
+                              "on the GPU every step")
+        cfg["path"] = "nvq_quantize_act_nvfp4 + nvq_gemm_nvf4 (tcgen05.mma kind::mxf4nvf4)"
+        return cfg
+
+    def launches_per_step(self):
+        return 2 * len(self.cases)       # quantise, block-scaled GEMM
+
+    def quantize(self, c, stream):
+        lib = self.capi.lib()
+        st = lib.nvq_quantize_act_nvfp4(c["x"].data_ptr(), self.M, c["K"], c["ac"].data_ptr(),
+                                        c["as"].data_ptr(), c["ag"].data_ptr(), stream.cuda_stream)
+        if st != 0:
+            raise self.capi.NVQError("nvq_quantize_act_nvfp4", st)
+
+    def dominant(self, c, codes, scales, stream):
+        self.capi.gemm_nvf4(codes, scales, c["g"], c["ac"], c["as"], c["ag"], c["y"],
+                            stream=stream)
+
+    def step(self, stream, e2e=False):
+        for c in self.cases:
+            if e2e:
+                c["x"].copy_(c["x_host"], non_blocking=True)
+            self.quantize(c, stream)
+            self.dominant(c, c["codes"], c["scales"], stream)
+            if e2e:
+                c["y_host"].copy_(c["y"], non_blocking=True)
+
+    def oracle_tasks(self, rows):
+        from bit_weight_quantized_nvq_b200 import workloads as wl
+        toks = max(1, min(self.M, 16))
+        tasks = []
+        for K, N in self.shapes:
+            base = oracle_base(
+                ("gemm", self.name, K, N),
+                lambda K=K, N=N: (wl.weight_rows("prefill", "W", N, K, ORACLE_BASE_ROWS),
+                                  wl.activations("prefill", "x", self.M, K, "normal",
+                                                 outliers=True)[:toks]))
+            codes, scales, g, x = base
+            tasks.append(sample_task((codes, scales, g, ("nvf4", x)), rows,
+                                     2.0 * toks * K / 1e12))
+        return tasks
+
+    def oracle_sample_desc(self, rows):
+        toks = max(1, min(self.M, 16))
+        return (f"{toks} tokens x {rows} weight rows of each of the {len(self.shapes)} shapes "
+                f"(the first {ORACLE_BASE_ROWS} rows, oracle-packed, run repeatedly): oracle "
+                "NVFP4 activation quantisation + fp64 dequantise-then-dot")
+
+
 class StackWorkload:
     """Every linear of a 64-layer dense decoder through nvq_decoder_stack."""
 
@@ -846,6 +930,8 @@ def make_workload(name: str):
             name, wl.SMALL_BATCH_SHAPES, M, lambda K, N: wl.small_batch_case(M, K, N),
             lambda K, N, r: (wl.weight_rows("small_batch", "W", N, K, r, True),
                              wl.activations("small_batch", "x", M, K, "student_t4")))
+    if name.startswith("nvf4_prefill_m"):
+        return Nvf4GemmWorkload(name, wl.PREFILL_SHAPES, int(name[len("nvf4_prefill_m"):]))
     if name.startswith("prefill_m"):
         return GemmWorkload(name, wl.PREFILL_SHAPES, int(name[len("prefill_m"):]))
     if name == "stack_decode":
@@ -869,6 +955,9 @@ def roofline_entry(wk, shapes, ms_per_step, peaks):
     """The dominant kernel's achieved rate against the measured peak."""
     if wk.bound == "hbm":
         scale, peak, unit, src = 1e9, peaks["hbm_gbs"], "GB/s", "hbm_gbs (copy)"
+    elif getattr(wk, "peak_scale", None):
+        scale, peak, unit, src = 1e12, peaks["bf16_tflops"] * wk.peak_scale, "TFLOP/s", \
+            wk.peak_note
     else:
         scale, peak, unit, src = 1e12, peaks["bf16_tflops"], "TFLOP/s", \
             "bf16_tflops (burst; fp16 runs at the bf16 rate)"

@@ -118,7 +118,9 @@ def test_traffic_is_used_only_for_the_measured_sources(tmp_path, monkeypatch):
 def test_workload_table():
     for name, bound in (("decode_sweep", "hbm"), ("gemv_4096", "hbm"), ("small_batch_m8", "hbm"),
                         ("prefill_m256", "tensor"), ("prefill_m2048", "tensor"),
-                        ("stack_decode", "hbm"), ("stack_prefill", "tensor")):
+                        ("stack_decode", "hbm"), ("stack_prefill", "tensor"),
+                        ("moe_decode", "hbm"), ("w4a16_decode", "hbm"),
+                        ("nvf4_prefill_m2048", "tensor")):
         wk = bench.make_workload(name)
         assert wk.bound == bound, name
         assert wk.config()["workload"] == name
@@ -138,6 +140,25 @@ def test_oracle_tasks_split_over_workers_keep_their_units():
     assert sum(p[4] for p in parts) == reps
     assert abs(sum(p[5] for p in parts) - units) < 1e-12
     assert abs(bench.run_tasks_serial(parts) - bench.run_tasks_serial(tasks)) < 1e-15
+
+
+def test_nvf4_oracle_task_runs_the_nvf4_oracle():
+    """The NVFP4 x NVFP4 sample runs the oracle's NVFP4 activation quantiser
+    and its NVFP4 dot (not the Q8_0 path), and its units are FLOPs."""
+    wk = bench.make_workload("nvf4_prefill_m256")
+    assert wk.peak_scale == 4.0
+    tasks = wk.oracle_tasks(64)
+    assert len(tasks) == len(wk.shapes)
+    codes, scales, g, x, reps, units = tasks[0]
+    assert isinstance(x, tuple) and x[0] == "nvf4" and x[1].shape[0] == 16
+    K = wk.shapes[0][0]
+    assert abs(units - 2.0 * 16 * K * 64 / 1e12) < 1e-15
+    assert bench.oracle_task((codes, scales, g, x, 1, units)) == units
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "source": "test"}
+    shapes = [{"K": K, "N": 64, "us_per_launch": 10.0, "amount": 1e9, "weight_copies": 2}]
+    r = bench.roofline_entry(wk, shapes, 0.02, peaks)
+    assert r["peak"] == 6000.0 and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - 100.0) < 1e-9
 
 
 def test_cpu_baseline_reports_one_core_and_all_cores():
