@@ -381,6 +381,7 @@ class GemvWorkload:
     kernel = "gemv"
     sources = ("gemv.cu", "nvq_device.cuh", "tcgen05.cuh")
     bound = "hbm"
+    dtype = "nvfp4 x q8_0 (int32 subblock sums, fp32 accumulate)"
     metric = "nvfp4_q8_0_gemv_weight_GBps"
     unit = "GB/s"
 
@@ -497,6 +498,7 @@ class SmallGemmWorkload(GemvWorkload):
 
     kernel = "gemm_small"
     sources = ("gemm_small.cu", "gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+    dtype = "nvfp4 x q8_0 (exact fp16 operands, fp32 accumulate)"
 
     def setup(self, device):
         import torch
@@ -524,6 +526,7 @@ class GemmWorkload(GemvWorkload):
     kernel = "gemm"
     sources = ("gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
     bound = "tensor"
+    dtype = "nvfp4 x q8_0 (exact fp16 operands, fp32 accumulate)"
     metric = "nvfp4_q8_0_prefill_gemm_TFLOPs"
     unit = "TFLOP/s"
 
@@ -584,6 +587,7 @@ class Nvf4GemmWorkload(GemmWorkload):
 
     kernel = "gemm_nvf4"
     sources = ("nvf4.cu", "tcgen05.cuh")
+    dtype = "nvfp4 x nvfp4 (block-scaled e2m1 tensor-core products, fp32 accumulate)"
     metric = "nvfp4_nvfp4_prefill_gemm_TFLOPs"
     peak_scale = 4.0
     peak_note = "bf16_tflops (burst) x 4, the nominal dense FP4/bf16 ratio (9 / 2.25 PFLOP/s)"
@@ -655,6 +659,7 @@ class StackWorkload:
     """Every linear of a 64-layer dense decoder through nvq_decoder_stack."""
 
     kernel = "stack_pass"
+    dtype = "nvfp4 x q8_0 (int32 subblock sums / exact fp16 operands, fp32 accumulate)"
     sources = ("nvq_stack.cpp", "gemv.cu", "gemm_tcgen05.cu", "quantize_q8_0.cu")
     unit = "tokens/s"
 
@@ -749,6 +754,7 @@ class W4A16Workload(GemvWorkload):
 
     kernel = "gemm_w4a16"
     sources = ("gemm_small.cu", "gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+    dtype = "nvfp4 x f16 (exact fp16 operands, fp32 accumulate)"
     metric = "nvfp4_f16_w4a16_weight_GBps"
 
     def setup(self, device):
@@ -808,6 +814,7 @@ class MoeWorkload:
     """Mixture-of-experts decode: Q8_0 of 16 tokens and nvq_moe_gemv."""
 
     kernel = "moe_gemv"
+    dtype = "nvfp4 x q8_0 (int32 subblock sums, fp32 accumulate)"
     sources = ("gemv.cu", "nvq_device.cuh", "tcgen05.cuh")
     bound = "hbm"
     metric = "nvfp4_q8_0_moe_gemv_weight_GBps"
@@ -1045,7 +1052,7 @@ def measure(wk, args, dist: Dist, peaks, device, sampler):
     h2d, d2h = wk.e2e_bytes()
     return {
         "metric": wk.metric, "value": round(units / (ms_max / 1e3), 3), "unit": wk.unit,
-        "ms_per_step": round(ms_per_step, 5),
+        "ms_per_step": round(ms_per_step, 5), "dtype": wk.dtype,
         "config": wk.config(),
         "e2e": {"value": round(units / (e2e_ms / 1e3), 3), "unit": wk.unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -1133,7 +1140,7 @@ def run_nvq(args, dist: Dist):
         "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": main["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4 x q8_0 (int32 subblock sums / exact fp16 operands, fp32 accumulate)",
+        "dtype": main["dtype"],
         "data": "synthetic (seeded; shapes and distributions of the workload)",
         "config": main["config"],
         "impl": "nvq",
