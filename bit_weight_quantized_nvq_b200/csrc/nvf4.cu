@@ -21,7 +21,7 @@
 // gemm_nvf4_kernel: one CTA per (128 weight rows, 128 tokens) tile.
 //   warp 0     TMA: per 256-wide K stage the 128 x 128-byte code tiles of
 //              weights and tokens (128-byte swizzle) and their 128 x 16-byte
-//              scale tiles, into a 4-deep ring;
+//              scale tiles, into a 6-deep ring (216 KB in flight per SM);
 //   warp 1     allocates tensor memory; issues 4 block-scaled MMAs per stage
 //              (M = 128 weight rows, N = 128 tokens, K = 64);
 //   warps 2-5  (one per tensor-memory lane quarter) copy each stage's scales
@@ -47,96 +47,216 @@ namespace {
 // ---------------------------------------------------------------------------
 // NVFP4 activation quantiser (one CTA per token row)
 // ---------------------------------------------------------------------------
-constexpr int kQThreads = 256;
-
 // UE4M3 byte nearest to r >= 0 (ties to the even code), saturating at
 // 0x7E = 448.  Bytes 0..7 are m * 2^-9 and byte 8e + m (e >= 1) is
-// (8 + m) * 2^(e-10): inside exponent e the code is (e-1)*8 + rint(r*2^(10-e)).
+// (8 + m) * 2^(e-10): inside exponent e the code is (e-1)*8 + rint(r*2^(10-e)),
+// e = (fp32 biased exponent of r) - 120, at least 1 (the subnormal bytes
+// share the spacing of e = 1).  2^(10-e) is built from its exponent bits, so
+// the scaling is exact.
 __device__ __forceinline__ uint32_t ue4m3_encode(float r) {
   if (!(r > 0.0f)) return 0;
   if (r >= 448.0f) return 0x7E;
-  int ex = 0;
-  frexpf(r, &ex);                 // r = f * 2^ex, f in [0.5, 1)
-  int e = ex + 6;
-  if (e < 1) e = 1;
-  const int n = __float2int_rn(ldexpf(r, 10 - e));   // exact scaling, rint half-even
+  const int e = max(1, static_cast<int>(__float_as_uint(r) >> 23) - 120);
+  const int n = __float2int_rn(r * __uint_as_float(static_cast<uint32_t>(137 - e) << 23));
   const int code = (e - 1) * 8 + n;
   return static_cast<uint32_t>(code > 0x7E ? 0x7E : code);
 }
+// Value of a UE4M3 byte (b <= 0x7E): m * 2^-9 for exponent 0, else the fp32
+// with exponent e - 7 and the three mantissa bits on top.
 __device__ __forceinline__ float ue4m3_value(uint32_t b) {
-  const int e = (b >> 3) & 0xF;
-  const int m = b & 0x7;
-  return e == 0 ? ldexpf(static_cast<float>(m), -9) : ldexpf(static_cast<float>(8 + m), e - 10);
+  const uint32_t e = (b >> 3) & 0xF, m = b & 0x7;
+  return e == 0 ? static_cast<float>(m) * 0x1p-9f : __uint_as_float(((e + 120) << 23) | (m << 20));
 }
-// E2M1 code nearest to x (ties to the even code), saturating at 6; the
-// magnitudes 0, .5, 1, 1.5 | 2, 3 | 4, 6 have spacings 0.5, 1 and 2, so the
-// codes are rint(2|x|), rint(|x|) + 2 and rint(|x|/2) + 4 there.
-__device__ __forceinline__ uint32_t e2m1_encode(float x) {
-  const float a = fabsf(x);
+// E2M1 magnitude code nearest to q >= 0 (ties to the even code), saturating
+// at 6; the magnitudes 0, .5, 1, 1.5 | 2, 3 | 4, 6 have spacings 0.5, 1 and
+// 2, so the codes are rint(2q), rint(q) + 2 and rint(q/2) + 4 there.
+__device__ __forceinline__ uint32_t e2m1_mag(float q) {
   int code;
-  if (a >= 6.0f)
+  if (q >= 6.0f)
     code = 7;
-  else if (a < 2.0f)
-    code = __float2int_rn(a * 2.0f);
-  else if (a < 4.0f)
-    code = __float2int_rn(a) + 2;
+  else if (q < 2.0f)
+    code = __float2int_rn(q * 2.0f);
+  else if (q < 4.0f)
+    code = __float2int_rn(q) + 2;
   else
-    code = __float2int_rn(a * 0.5f) + 4;
-  if (code != 0 && x < 0.0f) code |= 0x8;
+    code = __float2int_rn(q * 0.5f) + 4;
   return static_cast<uint32_t>(code);
 }
+// E2M1 code of the correctly rounded fp32 quotient x / gs, by IEEE division
+// and round-to-nearest-even on the E2M1 grid (a zero magnitude stored as +0).
+__device__ __forceinline__ uint32_t e2m1_code_exact(float x, float gs) {
+  uint32_t c = e2m1_mag(__fdiv_rn(fabsf(x), gs));
+  if (c != 0 && x < 0.0f) c |= 0x8;
+  return c;
+}
 
-__global__ void __launch_bounds__(kQThreads)
+// Eight fp32 values to eight E2M1 codes with the hardware conversion
+// (round to nearest, saturating at 6), value i in bits 4i..4i+3; a zero
+// magnitude is stored as +0.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+      : "=r"(w)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  const uint32_t mag = w & 0x77777777u;
+  return mag | (w & ((mag + 0x77777777u) & 0x88888888u));   // sign only where the magnitude is not 0
+}
+
+// The codes and scale of one subblock held by one thread (16 values).
+// Codes: the quotient x/gs is bracketed by x*inv*(1 - 2^-16) and
+// x*inv*(1 + 2^-16) (inv = 1/gs rounded; the correctly rounded quotient lies
+// strictly between them, their error being below 2^-22), and both brackets
+// are converted; rounding is monotone, so where the two codes agree that is
+// the code of the correctly rounded quotient, whatever the tie rule.  Where
+// they differ (the quotient is within 2^-16 of a rounding tie of the grid),
+// and when 1/gs could overflow (gs < 2^-120), the code is computed from the
+// IEEE quotient with ties to the even code.
+__device__ __forceinline__ void quantize_subblock(const float4 (&v)[4], float g, float six_g,
+                                                  uint2* cdst, uint8_t* sdst) {
+  float e[16];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    e[4 * j] = v[j].x;
+    e[4 * j + 1] = v[j].y;
+    e[4 * j + 2] = v[j].z;
+    e[4 * j + 3] = v[j].w;
+  }
+  float ab = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(e[i]));
+  const float r = six_g > 0.0f ? __fdiv_rn(ab, six_g) : 0.0f;
+  const uint32_t sc = ue4m3_encode(r);
+  const float gs = __fmul_rn(g, ue4m3_value(sc));
+  uint32_t w[2] = {0u, 0u};
+  if (gs > 0.0f) {
+    uint32_t diff[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+    if (gs >= 0x1p-120f) {
+      const float inv = __frcp_rn(gs);
+      const float ilo = inv * (1.0f - 0x1p-16f), ihi = inv * (1.0f + 0x1p-16f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float lo[8], hi[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          lo[i] = e[8 * h + i] * ilo;
+          hi[i] = e[8 * h + i] * ihi;
+        }
+        w[h] = cvt_e2m1x8(lo);
+        diff[h] = w[h] ^ cvt_e2m1x8(hi);
+      }
+    }
+    if (__builtin_expect((diff[0] | diff[1]) != 0u, 0)) {
+      for (int i = 0; i < 16; ++i) {
+        const int h = i >> 3, sh = 4 * (i & 7);
+        if ((diff[h] >> sh) & 0xFu)
+          w[h] = (w[h] & ~(0xFu << sh)) | (e2m1_code_exact(e[i], gs) << sh);
+      }
+    }
+  }
+  *cdst = make_uint2(w[0], w[1]);
+  *sdst = static_cast<uint8_t>(sc);
+}
+
+// One cluster of P CTAs per token row (P = gridDim.y <= 8), one thread per
+// 16-element subblock: CTA p takes subblocks [p*T, p*T + T).  Every load is
+// issued before any is used and the subblocks stay in registers between the
+// amax and the codes, so the row is read from memory once.  The row amax is
+// each CTA's block maximum, combined over the cluster through distributed
+// shared memory (the second cluster barrier keeps every CTA's shared memory
+// alive until all have read it).
+__global__ void __launch_bounds__(1024)
 quantize_nvfp4_kernel(const float* __restrict__ x, int K, uint8_t* __restrict__ codes,
                       uint8_t* __restrict__ scales, float* __restrict__ g_out) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int row = blockIdx.x;
-  const float* xr = x + static_cast<size_t>(row) * K;
-  __shared__ float red[kQThreads / 32];
+  const int T = blockDim.x;
+  const int P = gridDim.y;
+  const int nsub = K / 16;
+  const int sb = blockIdx.y * T + threadIdx.x;
+  const bool in = sb < nsub;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * K);
+  float4 v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = in ? __ldcs(xr + 4 * sb + j) : make_float4(0.f, 0.f, 0.f, 0.f);
   float a = 0.0f;
-  for (int i = threadIdx.x; i < K / 4; i += kQThreads) {
-    const float4 v = reinterpret_cast<const float4*>(xr)[i];
-    a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    a = fmaxf(a, fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w))));
+  __shared__ float red[32];
+  __shared__ float cta_max;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int w = 1; w < (T + 31) / 32; ++w) m = fmaxf(m, red[w]);
+    cta_max = m;
   }
+  float amax;
+  if (P == 1) {
+    __syncthreads();
+    amax = cta_max;
+  } else {
+    ptx::cluster_sync();
+    amax = 0.0f;
+    const uint32_t local = ptx::smem_addr(&cta_max);
+    for (int r = 0; r < P; ++r) {
+      float m;
+      asm volatile("ld.shared::cluster.f32 %0, [%1];"
+                   : "=f"(m) : "r"(ptx::mapa_shared(local, r)) : "memory");
+      amax = fmaxf(amax, m);
+    }
+    ptx::cluster_sync();
+  }
+  const float g = __fdiv_rn(amax, 2688.0f);
+  const float six_g = __fmul_rn(6.0f, g);
+  if (blockIdx.y == 0 && threadIdx.x == 0) g_out[row] = g;
+  if (in)
+    quantize_subblock(v, g, six_g,
+                      reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2)) + sb,
+                      scales + static_cast<size_t>(row) * (K / 16) + sb);
+}
+
+// Rows of more than 8 x 256 subblocks (K > 32768): two passes over the row (amax,
+// then the subblocks), the second pass reading it again.
+__global__ void __launch_bounds__(1024)
+quantize_nvfp4_long_kernel(const float* __restrict__ x, int K, uint8_t* __restrict__ codes,
+                           uint8_t* __restrict__ scales, float* __restrict__ g_out) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = blockIdx.x;
+  const int T = blockDim.x;
+  const int n4 = K / 4;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * K);
+  float a = 0.0f;
+  for (int i = threadIdx.x; i < n4; i += T) {
+    const float4 t = xr[i];
+    a = fmaxf(a, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+  }
+  __shared__ float red[32];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
   __syncthreads();
   float amax = red[0];
-#pragma unroll
-  for (int i = 1; i < kQThreads / 32; ++i) amax = fmaxf(amax, red[i]);
+  for (int w = 1; w < T / 32; ++w) amax = fmaxf(amax, red[w]);
   const float g = __fdiv_rn(amax, 2688.0f);
   const float six_g = __fmul_rn(6.0f, g);
   if (threadIdx.x == 0) g_out[row] = g;
-  // one thread per 16-element subblock
-  for (int b = threadIdx.x; b < K / 16; b += kQThreads) {
-    float v[16];
+  uint2* crow = reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2));
+  uint8_t* srow = scales + static_cast<size_t>(row) * (K / 16);
+  for (int sb = threadIdx.x; sb < K / 16; sb += T) {   // one subblock per thread and pass
+    float4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 t = reinterpret_cast<const float4*>(xr + 16 * b)[i];
-      v[4 * i] = t.x;
-      v[4 * i + 1] = t.y;
-      v[4 * i + 2] = t.z;
-      v[4 * i + 3] = t.w;
-    }
-    float ab = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) ab = fmaxf(ab, fabsf(v[i]));
-    const float r = six_g > 0.0f ? __fdiv_rn(ab, six_g) : 0.0f;
-    const uint32_t s = ue4m3_encode(r);
-    const float gs = __fmul_rn(g, ue4m3_value(s));
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t c = gs > 0.0f ? e2m1_encode(__fdiv_rn(v[i], gs)) : 0u;
-      if (i < 8)
-        w0 |= c << (4 * i);
-      else
-        w1 |= c << (4 * (i - 8));
-    }
-    reinterpret_cast<uint2*>(codes + static_cast<size_t>(row) * (K / 2))[b] = make_uint2(w0, w1);
-    scales[static_cast<size_t>(row) * (K / 16) + b] = static_cast<uint8_t>(s);
+    for (int j = 0; j < 4; ++j) v[j] = xr[4 * sb + j];
+    quantize_subblock(v, g, six_g, crow + sb, srow + sb);
   }
 }
 
@@ -146,7 +266,7 @@ quantize_nvfp4_kernel(const float* __restrict__ x, int K, uint8_t* __restrict__ 
 constexpr int kTile = 128;                 // weight rows (MMA M) and tokens (MMA N) per CTA
 constexpr int kStageK = 256;               // K per stage: 128 code bytes per row
 constexpr int kMmaK = 64;                  // K per block-scaled MMA
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kChunkStages = 4;            // stages per accumulator chunk (1024 K)
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
@@ -222,8 +342,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kTile;          // weight rows
-  const int m0 = blockIdx.y * kTile;          // tokens
+  // token tiles vary fastest, so the CTAs of a wave share weight tiles
+  const int m0 = blockIdx.x * kTile;          // tokens
+  const int n0 = blockIdx.y * kTile;          // weight rows
   const int num_k = K / kStageK;
   const int num_chunks = (num_k + kChunkStages - 1) / kChunkStages;
 
@@ -478,14 +599,30 @@ cudaLaunchAttribute pdl_attr() {
 
 cudaError_t launch_quantize_nvfp4(const float* x, int64_t M, int64_t K, uint8_t* codes,
                                   uint8_t* scales, float* g, cudaStream_t stream) {
+  // one thread per subblock, about 256 per CTA, a row split over a cluster
+  // of P <= 8 CTAs; rows of more than 2048 subblocks take the two-pass kernel
+  const int64_t nsub = K / 16;
+  const int64_t P = std::max<int64_t>(1, (nsub + 255) / 256);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(M));
-  cfg.blockDim = dim3(kQThreads);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cudaLaunchAttribute attr[2] = {pdl_attr(), {}};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_nvfp4_kernel, x, static_cast<int>(K), codes, scales, g);
+  const int k = static_cast<int>(K);
+  if (P > 8) {
+    cfg.gridDim = dim3(static_cast<unsigned>(M));
+    cfg.blockDim = dim3(1024);
+    return cudaLaunchKernelEx(&cfg, quantize_nvfp4_long_kernel, x, k, codes, scales, g);
+  }
+  const int64_t T = ((nsub + P - 1) / P + 31) / 32 * 32;
+  cfg.gridDim = dim3(static_cast<unsigned>(M), static_cast<unsigned>(P));
+  cfg.blockDim = dim3(static_cast<unsigned>(T));
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = static_cast<unsigned>(P);
+  attr[1].val.clusterDim.z = 1;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, quantize_nvfp4_kernel, x, k, codes, scales, g);
 }
 
 cudaError_t launch_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w,
@@ -502,8 +639,8 @@ cudaError_t launch_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, fl
   cudaError_t e = attr.ensure(gemm_nvf4_kernel, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((N + kTile - 1) / kTile),
-                     static_cast<unsigned>((M + kTile - 1) / kTile));
+  cfg.gridDim = dim3(static_cast<unsigned>((M + kTile - 1) / kTile),
+                     static_cast<unsigned>((N + kTile - 1) / kTile));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;

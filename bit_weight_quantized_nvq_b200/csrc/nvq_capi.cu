@@ -302,7 +302,7 @@ nvq_status nvq_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float 
                          const float* a_g, int64_t M, float* y, void* stream) {
   if (N < 0 || K < 0 || M < 0) return NVQ_ERR_INVALID_ARG;
   if (K == 0 || K % 256 != 0) return NVQ_ERR_BAD_SHAPE;
-  if (K > (int64_t{1} << 30) || N > INT32_MAX || M > int64_t{65535} * 128)
+  if (K > (int64_t{1} << 30) || N > int64_t{65535} * 128 || M > INT32_MAX)
     return NVQ_ERR_BAD_SHAPE;
   if (!(g_w == g_w)) return NVQ_ERR_INVALID_ARG;
   if (N == 0 || M == 0) return NVQ_OK;

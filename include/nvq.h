@@ -315,7 +315,7 @@ nvq_status nvq_quantize_act_nvfp4(const float* x, int64_t M, int64_t K, uint8_t*
  * registers every 1024 K.  Accuracy: |y - exact| <= 1e-5 * sum_k |w*a| +
  * 1e-6 per element, exact being the fp64 product of the dequantised
  * operands.
- * Requires K % 256 == 0, 1 <= M <= 65535*128 (NVQ_ERR_BAD_SHAPE); any N.
+ * Requires K % 256 == 0 and N <= 65535*128 (NVQ_ERR_BAD_SHAPE).
  * No workspace.  Errors: as nvq_gemm; a pipeline wait that gives up raises
  * NVQ_FLAG_GEMM_TIMEOUT.
  */

@@ -55,7 +55,11 @@ def reference(wref, aref, rows=None, toks=None):
             o.sum_abs_terms_nvf4(wc, ws, wg, ac, as_, ag))
 
 
-@pytest.mark.parametrize("M,K", [(1, 16), (3, 272), (37, 4096), (300, 5120), (5, 25600)])
+# K -> schedule: one CTA per row up to 256 subblocks (16 .. 4096), a cluster
+# of 2..8 CTAs per row up to 2048 (5120, 25600), the two-pass kernel beyond
+# (33024).
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 272), (37, 4096), (300, 5120), (5, 25600),
+                                 (3, 33024)])
 def test_quantiser_bit_exact(M, K):
     x = wl.activations("nvf4_test", "xq", M, K, "student_t4", outliers=K >= 1024)
     if M >= 3:
