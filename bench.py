@@ -1147,8 +1147,9 @@ def run_nvq(args, dist: Dist):
         "timing": ("CUDA graph of the K steps replayed once, events on the launching stream "
                    "before and after; no event nodes inside that replay"),
         "e2e": main["e2e"],
-        "gpu_launches": main["gpu_launches"] + sum(e["gpu_launches"] for e in entries.values()),
-        "gpu_launches_headline": main["gpu_launches"],
+        "gpu_launches": main["gpu_launches"],
+        "gpu_launches_all_workloads": main["gpu_launches"] + sum(e["gpu_launches"]
+                                                                 for e in entries.values()),
         "roofline": main["roofline"],
         "cpu_baseline": main["cpu_baseline"],
         "clocks": main["clocks"],

@@ -17,7 +17,15 @@
  *    table (download step): Q8_0 = 32 int8 values + one fp16 scale, 34 bytes.
  *  - "TKintegers K5: 3.21x prefill and 3.10x decode throughput vs TorchAO
  *    FP8 on NVIDIA L4": compact weight tiles expanded to FP16 tensor-core
- *    operands with FP32 accumulation (the prefill GEMM's design).
+ *    operands with FP32 accumulation (the prefill GEMM's design); and the
+ *    NVFP4 tensor-core engines it links to, which run both operands in
+ *    NVFP4 (nvq_gemm_nvf4).
+ *  - "HANDOFF ...", section 7 "Open items / next steps": item 1, the
+ *    mixture-of-experts product (mul_mat_id; nvq_moe_gemv); item 2, the
+ *    per-32 costs of the accumulation (the fused requantisation of
+ *    nvq_gemv_requant).
+ *  - "Roofline-First Decoding: results": a fused 4-bit dequantise-plus-GEMV
+ *    on fp16 activations for batch-1 decoding (nvq_gemm_w4a16).
  *
  * Data formats (all planar, row-major, owned by the caller):
  *  - NVFP4 weights W[N, K]:
@@ -41,9 +49,10 @@
  *    Accuracy: |y - exact| <= 1e-5 * sum_sb |term_sb| + 1e-6 per element.
  *
  * Conventions shared by every entry point:
- *  - Shapes: K a positive multiple of 64 (the 64-element blocks of the row
- *    dot).  The empty product (N == 0 or M == 0) is accepted and does
- *    nothing.
+ *  - Shapes: the NVFP4 x Q8_0 products take K a positive multiple of 64
+ *    (the 64-element blocks of the row dot); each entry point states its
+ *    own further conditions.  The empty product (N == 0 or M == 0) is
+ *    accepted and does nothing.
  *  - Device pointers must be 16-byte aligned (NVQ_ERR_MISALIGNED).
  *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *    stream.  Device entry points only enqueue work and return at once;
