@@ -126,14 +126,6 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
 }
 
 // ---- fp16 operand expansion (tensor-core paths) ------------------------------
-// fp16 high bytes of the E2M1 values: 0, .5, 1, 1.5, 2, 3, 4, 6 are 0x0000,
-// 0x3800, 0x3C00, 0x3E00, 0x4000, 0x4200, 0x4400, 0x4600 (low bytes zero);
-// codes 8..15 carry the sign bit 0x80.
-constexpr uint32_t kHbPosLo = 0x3E3C3800u;
-constexpr uint32_t kHbPosHi = 0x46444240u;
-constexpr uint32_t kHbNegLo = 0xBEBCB880u;
-constexpr uint32_t kHbNegHi = 0xC6C4C2C0u;
-
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
@@ -143,16 +135,25 @@ __device__ __forceinline__ __half2 bits_h2(uint32_t u) {
 
 // Eight codes (one word, element i in nibble i) -> eight fp16
 // w' = E2M1 * s as four half2 words (element 2i in the low half of word i).
-// E2M1 * s has at most 6 significant bits and lies in 2^-10 .. 2688, so the
-// fp16 product is exact.
+// The hardware E2M1 -> f16x2 conversion takes one byte (two codes, the low
+// nibble to the low half) and is exact: every E2M1 value is an fp16 value
+// (code 8 gives -0, as a signed zero should).  E2M1 * s has at most 6
+// significant bits and lies in 2^-10 .. 2688, so the fp16 product is exact.
 __device__ __forceinline__ uint4 expand8(uint32_t w, __half2 s2) {
-  uint32_t lo, hi;
-  lut16_x8<kHbPosLo, kHbPosHi, kHbNegLo, kHbNegHi>(w, lo, hi);
+  uint32_t e0, e1, e2, e3;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(e0), "=r"(e1), "=r"(e2), "=r"(e3)
+      : "r"(w));
   uint4 r;
-  r.x = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x1404)), s2));
-  r.y = h2_bits(__hmul2(bits_h2(__byte_perm(lo, 0u, 0x3424)), s2));
-  r.z = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x1404)), s2));
-  r.w = h2_bits(__hmul2(bits_h2(__byte_perm(hi, 0u, 0x3424)), s2));
+  r.x = h2_bits(__hmul2(bits_h2(e0), s2));
+  r.y = h2_bits(__hmul2(bits_h2(e1), s2));
+  r.z = h2_bits(__hmul2(bits_h2(e2), s2));
+  r.w = h2_bits(__hmul2(bits_h2(e3), s2));
   return r;
 }
 
