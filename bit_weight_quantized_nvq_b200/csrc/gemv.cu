@@ -678,6 +678,391 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
+// The linears of a decoder stack at one token in one persistent launch
+// ---------------------------------------------------------------------------
+// Matrices of a layer: q, k, v (input Q8_0(x)), o (input Q8_0(y_v)), up,
+// gate (input Q8_0(y_o)), down (input Q8_0(y_up)); v, o and up also emit the
+// Q8_0 of their output.  Every CTA takes an even slice of the rows of every
+// matrix, always in the same order of units (matrix, layer):
+//   v0 q0 k0 o0 | v1 q1 k1 up0 gate0 down0 o1 | v2 q2 k2 up1 gate1 down1 o2 | ...
+// so each unit that needs another unit's output finds it finished long
+// before: v before q and k (o waits for v), the next layer's v, q, k between
+// o and up (up and gate wait for o), up before gate (down waits for up).  A
+// finished unit raises a grid counter (its warps count in shared memory and
+// the last one adds 1 per CTA); a waiting warp reads the counter with
+// acquire semantics, so usually it is already complete.  The weights do not
+// depend on any activation, so the producer streams stage after stage across
+// units and layers.  The requantised activations alternate between two
+// buffers by layer parity, so no unit overwrites an input that a slower CTA
+// may still read.  The launch is cooperative (all CTAs resident); every wait
+// is bounded (4 s) and a timeout raises the GEMV error flag and stops the CTA.
+constexpr int kStackMaxLayers = 64;
+constexpr int kStackLin = 7;
+constexpr int kStackScnt = 16;     // block counters per requantised matrix and CTA
+constexpr int kStackArr = 8;       // ring of per-CTA arrival counters
+enum : int { kSq = 0, kSk, kSv, kSo, kSup, kSgate, kSdown };
+
+struct StackArgs {
+  const uint8_t* codes[kStackMaxLayers * kStackLin];
+  const uint8_t* scales[kStackMaxLayers * kStackLin];
+  float half_g[kStackMaxLayers * kStackLin];
+  float* outs[kStackLin];
+  const int8_t* x_q;              // Q8_0(x)
+  const __half* x_d;
+  int8_t* b_q[3][2];              // Q8_0 of y_v, y_o, y_up, by layer parity
+  __half* b_d[3][2];
+  int* rq_cnt[3];                 // global block counters of v, o, up
+  unsigned int* bar;              // [layer][3] CTAs done with v, o, up
+  int n_layers;
+  int N[kStackLin];
+  int K0;                         // K of q, k, v, o, up, gate
+  int Kd;                         // K of down (= N of up)
+};
+
+// Unit u of the schedule -> (layer, matrix).  7 units per layer: the first
+// four are v0 q0 k0 o0, then per layer l a block v(l+1) q(l+1) k(l+1) up(l)
+// gate(l) down(l) o(l+1), the last layer's block only up, gate, down.
+__device__ __forceinline__ void stack_unit(int u, int L, int& l, int& m) {
+  if (u < 4) {
+    l = 0;
+    m = u == 3 ? kSo : (u == 0 ? kSv : u - 1);
+    return;
+  }
+  u -= 4;
+  l = u / 7;
+  int r = u % 7;
+  if (l >= L - 1) {
+    l = L - 1;
+    r = u - 7 * (L - 1) + 3;
+  }
+  if (r < 3) {
+    m = r == 0 ? kSv : r - 1;
+    ++l;
+  } else if (r < 6) {
+    m = kSup + (r - 3);
+  } else {
+    m = kSo;
+    ++l;
+  }
+}
+// requantised-matrix index (v, o, up) or -1; its counter instance k = 3l + index
+__device__ __forceinline__ int stack_rq(int m) {
+  return m == kSv ? 0 : m == kSo ? 1 : m == kSup ? 2 : -1;
+}
+// the unit a matrix waits for: o waits for v, up for o, down for up
+__device__ __forceinline__ int stack_dep(int m) {
+  return m == kSo ? 0 : m == kSup ? 1 : m == kSdown ? 2 : -1;
+}
+
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Waits until *ctr >= target (bounded; false on timeout or abort).
+__device__ __forceinline__ bool wait_counter(const unsigned int* ctr, unsigned int target,
+                                             volatile int* abort_flag) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (ld_acquire_u32(ctr) < target) {
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(256);
+  }
+  return true;
+}
+
+struct StackCta {                 // what a consumer warp needs of its CTA
+  uint8_t* smem;
+  float* part;
+  uint64_t* full;
+  uint64_t* empty;
+  int* arrived;                   // [kStackArr] warps done, per counter instance
+  int* scnt;                      // [3][kStackScnt] rows per 32-row block
+  volatile int* abort_flag;
+  int warp, lane, G;
+};
+
+// A warp waits until every CTA has finished a unit (lane 0 polls).
+__device__ __forceinline__ bool stack_wait(const unsigned int* ctr, const StackCta& c) {
+  int ok = 1;
+  if (c.lane == 0) ok = wait_counter(ctr, static_cast<unsigned int>(c.G), c.abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// A run of units with the same input for one consumer warp: the activations
+// once into registers, then for each unit its wait (if any), its stages and
+// its arrival (if it is v, o or up).  Returns false on a timeout or abort.
+template <int NPL, int WPR>
+__device__ __forceinline__ bool stack_consume(const StackArgs& a, const StackCta& c, int u0,
+                                              int u1, const int8_t* q, const __half* d, int K,
+                                              int& it) {
+  const int warp = c.warp, lane = c.lane;
+  const int R = reg_rows(K, WPR);
+  const int active = R * WPR;
+  const uint32_t row_code = K / 2, row_scale = K / 16;
+  const uint32_t codes_bytes = static_cast<uint32_t>(R) * row_code;
+  const int rl = warp / WPR;
+  const int pt = warp % WPR;
+  // the first unit's wait comes before its input is read
+  {
+    int l, m;
+    stack_unit(u0, a.n_layers, l, m);
+    const int dep = stack_dep(m);
+    if (dep >= 0 && !stack_wait(a.bar + 3 * l + dep, c)) return false;
+  }
+  uint4 qa[NPL], qb[NPL];
+  float dd[NPL];
+  int c0[NPL], c1[NPL];
+  // written during this launch by other CTAs: read through L2
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int ch = pt * (NPL * 32) + lane + 32 * i;
+    const uint4* src = reinterpret_cast<const uint4*>(q) + 2 * ch;
+    qa[i] = __ldcg(src);
+    qb[i] = __ldcg(src + 1);
+    dd[i] = __half2float(__ushort_as_half(__ldcg(reinterpret_cast<const unsigned short*>(d) + ch)));
+    const int s0 = dev::dp4a(qa[i].x, 0x01010101u, dev::dp4a(qa[i].y, 0x01010101u,
+                   dev::dp4a(qa[i].z, 0x01010101u, dev::dp4a(qa[i].w, 0x01010101u, 0))));
+    const int s1 = dev::dp4a(qb[i].x, 0x01010101u, dev::dp4a(qb[i].y, 0x01010101u,
+                   dev::dp4a(qb[i].z, 0x01010101u, dev::dp4a(qb[i].w, 0x01010101u, 0))));
+    c0[i] = -12 * s0;
+    c1[i] = -12 * s1;
+  }
+  for (int u = u0; u < u1; ++u) {
+    int l, m;
+    stack_unit(u, a.n_layers, l, m);
+    const int dep = stack_dep(m);
+    if (u > u0 && dep >= 0 && !stack_wait(a.bar + 3 * l + dep, c)) return false;
+    const int N = a.N[m];
+    const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / c.G);
+    const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / c.G);
+    const int li = l * kStackLin + m;
+    const int rq = stack_rq(m);
+    float* y = a.outs[m];
+    for (int row0 = r_begin; row0 < r_end; row0 += R, ++it) {
+      const int nrows = min(R, r_end - row0);
+      const int s = it % kM1Stages;
+      const uint32_t ph = (it / kM1Stages) & 1;
+      if (!ptx::mbar_wait_bounded(ptx::smem_addr(c.full + s), ph, c.abort_flag, kWaitLimitNs))
+        return false;
+      if (warp < active && rl < nrows) {
+        const uint8_t* st = c.smem + s * kRegStageMax;
+        const uint4* cw = reinterpret_cast<const uint4*>(st + rl * row_code) + pt * (NPL * 32);
+        const uint16_t* sw =
+            reinterpret_cast<const uint16_t*>(st + codes_bytes + rl * row_scale) + pt * (NPL * 32);
+        uint4 w[NPL];
+        uint32_t s2[NPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          w[i] = cw[lane + 32 * i];
+          s2[i] = sw[lane + 32 * i];
+        }
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+          const int i0 = dev::dot16_biased(w[i].x, w[i].y, qa[i], c0[i]);
+          const int i1 = dev::dot16_biased(w[i].z, w[i].w, qb[i], c1[i]);
+          const float2 sf = dev::ue4m3x2_to_float2(s2[i]);
+          acc = fmaf(dd[i], fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
+        }
+        acc = dev::warp_sum(acc);
+        if (WPR == 1) {
+          const int row = row0 + rl;
+          int how = 0;
+          if (lane == 0) {
+            y[row] = acc * a.half_g[li];
+            if (rq >= 0) {
+              // rows of this CTA per 32-row block counted in shared memory
+              // (reset by the row that completes the CTA's share), the share
+              // of a block that straddles two CTAs through the global counter
+              const int bstart = row & ~31;
+              const int mine = min(r_end, bstart + 32) - max(r_begin, bstart);
+              int* sc = c.scnt + rq * kStackScnt + ((row >> 5) - (r_begin >> 5));
+              __threadfence_block();
+              if (atomicAdd(sc, 1) + 1 == mine) {
+                atomicExch(sc, 0);
+                if (mine == 32) {
+                  how = 1;
+                } else {
+                  __threadfence();
+                  if (atomicAdd(a.rq_cnt[rq] + (row >> 5), mine) + mine == 32) how = 2;
+                }
+              }
+            }
+          }
+          if (rq >= 0) {
+            how = __shfl_sync(0xffffffffu, how, 0);
+            if (how != 0) {
+              if (how == 1) __threadfence_block(); else __threadfence();
+              RegMat rm = {};
+              rm.y = y;
+              rm.rq_q = a.b_q[rq][l & 1];
+              rm.rq_d = a.b_d[rq][l & 1];
+              requant_block_warp(rm, row >> 5, lane);
+              if (how == 2 && lane == 0) atomicExch(a.rq_cnt[rq] + (row >> 5), 0);
+            }
+          }
+        } else if (lane == 0) {
+          c.part[s * kM1Consumers + warp] = acc;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(c.empty + s));
+    }
+    if (rq >= 0) {
+      // this warp's rows and requantisations of the unit are written: count
+      // it; the CTA's last warp raises the grid counter once
+      const int k = 3 * l + rq;
+      __threadfence();
+      __syncwarp();
+      if (lane == 0 && atomicAdd(c.arrived + k % kStackArr, 1) == kM1Consumers - 1) {
+        c.arrived[k % kStackArr] = 0;
+        __threadfence();
+        atomicAdd(a.bar + k, 1u);
+      }
+      __syncwarp();
+    }
+  }
+  return true;
+}
+
+template <int NPL0, int NPL3, int WPR3>
+__global__ void __launch_bounds__(kM1Threads, 1)
+stack_m1_kernel(const __grid_constant__ StackArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  float* part = reinterpret_cast<float*>(smem + kM1Stages * kRegStageMax);   // [stage][warp]
+  uint64_t* full = reinterpret_cast<uint64_t*>(part + kM1Stages * kM1Consumers);
+  uint64_t* empty = full + kM1Stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kM1Stages);
+  int* arrived = reinterpret_cast<int*>(empty + kM1Stages + 1);   // [kStackArr]
+  int* scnt = arrived + kStackArr;                                 // [3][kStackScnt]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const int L = a.n_layers;
+  const int units = kStackLin * L;
+
+  grid_dependents_launch();
+  for (int i = threadIdx.x; i < kStackArr + 3 * kStackScnt; i += blockDim.x) arrived[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kM1Stages; ++i) {
+      ptx::mbar_init(ptx::smem_addr(full + i), 1);
+      ptx::mbar_init(ptx::smem_addr(empty + i), kM1Consumers);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kM1Consumers) {
+    // ---------------- producer: the weight stages of every unit --------------
+    if (lane != 0) return;
+    bool waited = false;
+    int sli[kM1Stages] = {}, srow[kM1Stages] = {}, snr[kM1Stages] = {};
+    bool sfin[kM1Stages] = {};
+    auto finalize = [&](int it) {   // rows of a down stage: sum of the WPR3 partials
+      const int s = it % kM1Stages;
+      if (!sfin[s]) return;
+      float* y = a.outs[kSdown];
+      const float hg = a.half_g[sli[s]];
+      for (int r = 0; r < snr[s]; ++r) {
+        float v = 0.0f;
+#pragma unroll
+        for (int pp = 0; pp < WPR3; ++pp) v += part[s * kM1Consumers + r * WPR3 + pp];
+        y[srow[s] + r] = v * hg;
+      }
+    };
+    int it = 0;
+    bool ok = true;
+    for (int u = 0; u < units && ok; ++u) {
+      int l, m;
+      stack_unit(u, L, l, m);
+      const int K = m == kSdown ? a.Kd : a.K0;
+      const int R = m == kSdown ? reg_rows(K, WPR3) : reg_rows(K, 1);
+      const uint32_t row_code = K / 2, row_scale = K / 16;
+      const uint32_t codes_bytes = static_cast<uint32_t>(R) * row_code;
+      const int N = a.N[m];
+      const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
+      const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
+      const int li = l * kStackLin + m;
+      for (int row0 = r_begin; row0 < r_end; row0 += R) {
+        const int nrows = min(R, r_end - row0);
+        const int s = it % kM1Stages;
+        const uint32_t ph = (it / kM1Stages) & 1;
+        if (it == kM1Stages) {
+          grid_dependency_wait();
+          waited = true;
+        }
+        if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + s), ph ^ 1, abort_flag, kWaitLimitNs)) {
+          *abort_flag = 1;
+          raise_timeout();
+          ok = false;
+          break;
+        }
+        if (it >= kM1Stages) finalize(it - kM1Stages);
+        sli[s] = li;
+        srow[s] = row0;
+        snr[s] = nrows;
+        sfin[s] = m == kSdown && WPR3 > 1;
+        const uint32_t bar = ptx::smem_addr(full + s);
+        uint8_t* st = smem + s * kRegStageMax;
+        ptx::mbar_arrive_expect_tx(bar, nrows * (row_code + row_scale));
+        ptx::bulk_load(ptx::smem_addr(st), a.codes[li] + static_cast<size_t>(row0) * row_code,
+                       nrows * row_code, bar);
+        ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
+                       a.scales[li] + static_cast<size_t>(row0) * row_scale, nrows * row_scale,
+                       bar);
+        ++it;
+      }
+    }
+    if (!waited) grid_dependency_wait();
+    if (ok) {
+      for (int i = max(0, it - kM1Stages); i < it; ++i) {
+        if (!ptx::mbar_wait_bounded(ptx::smem_addr(empty + i % kM1Stages), (i / kM1Stages) & 1,
+                                    abort_flag, kWaitLimitNs)) {
+          *abort_flag = 1;
+          raise_timeout();
+          break;
+        }
+        finalize(i);
+      }
+    } else {
+      for (int i = max(0, it - kM1Stages); i < it; ++i)
+        ptx::mbar_wait_bounded(ptx::smem_addr(full + i % kM1Stages), (i / kM1Stages) & 1, nullptr,
+                               kWaitLimitNs);
+    }
+    return;
+  }
+
+  // ---------------- consumers: runs of units with the same input ----------------
+  grid_dependency_wait();   // Q8_0(x) from the quantiser before this kernel
+  const StackCta c = {smem, part, full, empty, arrived, scnt, abort_flag, warp, lane, G};
+  int it = 0;
+  int u = 0;
+  while (u < units) {
+    int l, m;
+    stack_unit(u, L, l, m);
+    // the run: v q k (Q8_0(x)), o, up gate, down
+    const int len = (m == kSv || m == kSup) ? (m == kSv ? 3 : 2) : 1;
+    bool ok;
+    if (m == kSdown) {
+      ok = stack_consume<NPL3, WPR3>(a, c, u, u + len, a.b_q[2][l & 1], a.b_d[2][l & 1], a.Kd, it);
+    } else {
+      const int8_t* q = m == kSv ? a.x_q : m == kSo ? a.b_q[0][l & 1] : a.b_q[1][l & 1];
+      const __half* d = m == kSv ? a.x_d : m == kSo ? a.b_d[0][l & 1] : a.b_d[1][l & 1];
+      ok = stack_consume<NPL0, 1>(a, c, u, u + len, q, d, a.K0, it);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      raise_timeout();
+      return;
+    }
+    u += len;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // M = 2..16 (and fallback M = 1) schedule: persistent CTAs, TMA ring
 // ---------------------------------------------------------------------------
 template <int MT, bool ISUM>
@@ -1067,7 +1452,98 @@ cudaError_t launch_gemv_any(const uint8_t* codes, const uint8_t* scales, float g
   }
 }
 
+// ---- the persistent stack launch ----
+constexpr uint32_t kStackSmem = kM1Stages * kRegStageMax + kM1Stages * kM1Consumers * 4 +
+                                2 * kM1Stages * 8 + 8 + (kStackArr + 3 * kStackScnt) * 4;
+static_assert(kStackSmem <= kSmemPerCtaMax, "shared memory of the stack kernel");
+
+template <int NPL0, int NPL3, int WPR3>
+cudaError_t launch_stack_t(const StackM1& s, cudaStream_t stream) {
+  auto kernel = stack_m1_kernel<NPL0, NPL3, WPR3>;
+  static SmemAttrOnce attr;
+  cudaError_t e = attr.ensure(kernel, static_cast<int>(kStackSmem));
+  if (e != cudaSuccess) return e;
+  const int G = device_sm_count();
+  StackArgs a = {};
+  for (int i = 0; i < kStackLin; ++i) {
+    a.outs[i] = s.outs[i];
+    a.N[i] = static_cast<int>(s.N[i]);
+  }
+  a.x_q = s.x_q;
+  a.x_d = reinterpret_cast<const __half*>(s.x_d);
+  for (int i = 0; i < 3; ++i) {
+    for (int par = 0; par < 2; ++par) {
+      a.b_q[i][par] = s.b_q[i][par];
+      a.b_d[i][par] = reinterpret_cast<__half*>(s.b_d[i][par]);
+    }
+    a.rq_cnt[i] = s.cnt[i];
+  }
+  a.bar = s.bar;
+  a.K0 = static_cast<int>(s.K0);
+  a.Kd = static_cast<int>(s.Kd);
+  for (int64_t l0 = 0; l0 < s.n_layers; l0 += kStackMaxLayers) {
+    const int nl = static_cast<int>(std::min<int64_t>(kStackMaxLayers, s.n_layers - l0));
+    a.n_layers = nl;
+    for (int l = 0; l < nl; ++l)
+      for (int i = 0; i < kStackLin; ++i) {
+        const StackLinear& w = s.lin[(l0 + l) * kStackLin + i];
+        a.codes[l * kStackLin + i] = w.codes;
+        a.scales[l * kStackLin + i] = w.scales;
+        a.half_g[l * kStackLin + i] = 0.5f * w.g;
+      }
+    // the unit counters start at zero in every launch
+    e = cudaMemsetAsync(s.bar, 0, 3 * kStackMaxLayers * sizeof(unsigned int), stream);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(G));
+    cfg.blockDim = dim3(kM1Threads);
+    cfg.dynamicSmemBytes = kStackSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeCooperative;
+    attrs[0].val.cooperative = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kernel, a);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
+
+bool stack_m1_supported(int64_t K0, int64_t Kd, const int64_t* N) {
+  if (K0 != 4096 && K0 != 5120) return false;
+  switch (Kd) {
+    case 8192: case 10240: case 12288: case 16384: case 20480: case 25600: break;
+    default: return false;
+  }
+  // requantised matrices (v, o, up) in whole 32-row blocks; a CTA's slice of
+  // one spans at most kStackScnt - 2 blocks
+  const int64_t G = device_sm_count();
+  for (int i : {2, 3, 4}) {
+    if (N[i] % 32 != 0) return false;
+    if ((N[i] + G - 1) / G / 32 + 2 > kStackScnt) return false;
+  }
+  for (int i = 0; i < 7; ++i)
+    if (N[i] >= (int64_t{1} << 30)) return false;
+  return true;
+}
+
+cudaError_t launch_stack_m1(const StackM1& s, cudaStream_t stream) {
+#define NVQ_STACK(n0, n3, w3) return launch_stack_t<n0, n3, w3>(s, stream)
+  const bool k4 = s.K0 == 4096;
+  switch (s.Kd) {
+    case 8192: if (k4) NVQ_STACK(4, 4, 2); NVQ_STACK(5, 4, 2);
+    case 10240: if (k4) NVQ_STACK(4, 5, 2); NVQ_STACK(5, 5, 2);
+    case 12288: if (k4) NVQ_STACK(4, 6, 2); NVQ_STACK(5, 6, 2);
+    case 16384: if (k4) NVQ_STACK(4, 4, 4); NVQ_STACK(5, 4, 4);
+    case 20480: if (k4) NVQ_STACK(4, 5, 4); NVQ_STACK(5, 5, 4);
+    case 25600: if (k4) NVQ_STACK(4, 5, 5); NVQ_STACK(5, 5, 5);
+    default: return cudaErrorNotSupported;
+  }
+#undef NVQ_STACK
+}
 
 cudaError_t launch_gemv(const uint8_t* codes, const uint8_t* scales, float g,
                         int64_t N, int64_t K, const int8_t* q, const uint16_t* d,

@@ -54,6 +54,30 @@ cudaError_t launch_moe_gemv(const uint8_t* codes, const uint8_t* scales, const f
                             int64_t N, int64_t K, const int32_t* ids, int64_t T, int64_t top_k,
                             const int8_t* q, const uint16_t* d, float* y, cudaStream_t stream);
 
+// The linears of a decoder stack at one token in one persistent (cooperative)
+// launch per 64 layers; see nvq_decoder_stack for the dataflow.  Supported
+// for K0 (hidden) 4096 or 5120 and the down K of stack_m1_supported.
+struct StackLinear {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  float g;
+};
+struct StackM1 {
+  const StackLinear* lin;        // host [n_layers * 7]: q, k, v, o, up, gate, down
+  int64_t n_layers;
+  int64_t N[7];
+  int64_t K0, Kd;
+  float* outs[7];
+  const int8_t* x_q;             // Q8_0(x), written before the launch
+  const uint16_t* x_d;
+  int8_t* b_q[3][2];             // Q8_0 of y_v, y_o, y_up, two buffers each
+  uint16_t* b_d[3][2];
+  int* cnt[3];                   // block counters of v, o, up: zero, left zero
+  unsigned int* bar;             // 3 * 64 unit counters (zeroed by the launcher)
+};
+bool stack_m1_supported(int64_t K0, int64_t Kd, const int64_t* N);
+cudaError_t launch_stack_m1(const StackM1& s, cudaStream_t stream);
+
 // Test-only: a pipeline wait that can never complete, bounded by limit_ns;
 // result[0] = 1 if the wait completed (never), result[1] = microseconds waited.
 cudaError_t launch_stalled_wait(uint64_t limit_ns, int* result, cudaStream_t stream);

@@ -3,16 +3,20 @@
 // 64-layer token pass issues its launches without crossing back into
 // Python.  The dataflow of a layer is documented in include/nvq.h.
 //
-// One token (M = 1) takes five launches per layer: the quantiser of x; one
-// GEMV over q, k and v together (they read the same activations) that also
-// emits Q8_0(y_v); the o GEMV that emits Q8_0(y_o); one GEMV over up and gate
-// that emits Q8_0(y_up); the down GEMV.  The requantisations write the other
-// of two activation buffers than the one the launch reads.  Other token
-// counts run the quantiser and the products separately (GEMV for M <= 16,
-// the tensor-core GEMM above, whose fp16 expansion of the activations is
-// shared by the products that read it).
+// One token (M = 1), for the common shapes (hidden 4096 or 5120, v and o
+// as wide as the hidden size): Q8_0(x) once (every layer reads the same x),
+// then one persistent launch per 64 layers that runs all their products,
+// layer after layer pipelined, with the requantisations of y_v, y_o and
+// y_up fused into the products (launch_stack_m1).  Other one-token shapes take five launches per
+// layer: the quantiser of x; one GEMV over q, k and v together (they read
+// the same activations) that also emits Q8_0(y_v); the o GEMV that emits
+// Q8_0(y_o); one GEMV over up and gate that emits Q8_0(y_up); the down GEMV.
+// Other token counts run the quantiser and the products separately (GEMV for
+// M <= 16, the tensor-core GEMM above, whose fp16 expansion of the
+// activations is shared by the products that read it).
 #include <algorithm>
 #include <cstdint>
+#include <vector>
 
 #include <cuda_runtime.h>
 
@@ -43,24 +47,31 @@ bool layer_shapes_ok(const nvq_linear* L) {
          L[kUp].K == L[kO].N && L[kGate].K == L[kO].N && L[kDown].K == L[kUp].N;
 }
 
-// Workspace: two Q8_0 activation buffers (codes, scales), the requantisation
-// block counters of v, o and up (one token), and the GEMM's expansion.
+// Workspace: Q8_0 activation buffers (codes, scales; two, or seven for one
+// token: x and two each for y_v, y_o, y_up), the requantisation block
+// counters of v, o and up and the unit counters of the persistent launch
+// (one token), and the GEMM's expansion.
+constexpr int kBuffers = 7;
+constexpr size_t kBarBytes = 3 * 64 * sizeof(unsigned int);
+
 struct Layout {
-  size_t q_off[2], d_off[2], cnt_off, cnt_bytes, gemm_off, total;
+  size_t q_off[kBuffers], d_off[kBuffers], cnt_off, cnt_bytes, bar_off, gemm_off, total;
 };
 
 Layout workspace_layout(const nvq_linear* L, int64_t M) {
   const int64_t km = max_k(L);
   const size_t qb = round256(static_cast<size_t>(M * km));
   const size_t db = round256(static_cast<size_t>(M * (km / 32) * 2));
-  Layout w;
-  w.q_off[0] = 0;
-  w.d_off[0] = qb;
-  w.q_off[1] = qb + db;
-  w.d_off[1] = 2 * qb + db;
-  w.cnt_off = 2 * (qb + db);
+  const int nb = M == 1 ? kBuffers : 2;
+  Layout w = {};
+  for (int i = 0; i < nb; ++i) {
+    w.q_off[i] = i * (qb + db);
+    w.d_off[i] = i * (qb + db) + qb;
+  }
+  w.cnt_off = nb * (qb + db);
   w.cnt_bytes = M == 1 ? round256(static_cast<size_t>((L[kV].N + L[kO].N + L[kUp].N) / 32) * 4) : 0;
-  w.gemm_off = w.cnt_off + w.cnt_bytes;
+  w.bar_off = w.cnt_off + w.cnt_bytes;
+  w.gemm_off = w.bar_off + (M == 1 ? round256(kBarBytes) : 0);
   w.total = w.gemm_off + (M > 16 ? nvq::gemm_workspace_size(M, 0, km) : 0);
   return w;
 }
@@ -113,14 +124,50 @@ extern "C" nvq_status nvq_decoder_stack(const nvq_linear* linears, int64_t n_lay
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int8_t* qa[2] = {reinterpret_cast<int8_t*>(ws + lay.q_off[0]),
-                   reinterpret_cast<int8_t*>(ws + lay.q_off[1])};
-  uint16_t* da[2] = {reinterpret_cast<uint16_t*>(ws + lay.d_off[0]),
-                     reinterpret_cast<uint16_t*>(ws + lay.d_off[1])};
+  int8_t* qa[kBuffers];
+  uint16_t* da[kBuffers];
+  for (int i = 0; i < kBuffers; ++i) {
+    qa[i] = reinterpret_cast<int8_t*>(ws + lay.q_off[i]);
+    da[i] = reinterpret_cast<uint16_t*>(ws + lay.d_off[i]);
+  }
   void* gws = ws + lay.gemm_off;
   cudaError_t err = cudaSuccess;
 
-  if (M == 1) {
+  int64_t Ns[NVQ_STACK_LINEARS];
+  for (int i = 0; i < NVQ_STACK_LINEARS; ++i) Ns[i] = L0[i].N;
+  const bool persistent = M == 1 && L0[kV].N == L0[kQ].K && L0[kO].N == L0[kQ].K &&
+                          nvq::stack_m1_supported(L0[kQ].K, L0[kDown].K, Ns);
+  if (persistent) {
+    int* cnt = reinterpret_cast<int*>(ws + lay.cnt_off);
+    err = cudaMemsetAsync(cnt, 0, lay.cnt_bytes, st);
+    if (err == cudaSuccess) err = nvq::launch_quantize_q8_0(x, 1, L0[kQ].K, qa[0], da[0], st);
+    if (err == cudaSuccess) {
+      std::vector<nvq::StackLinear> lin(static_cast<size_t>(n_layers) * NVQ_STACK_LINEARS);
+      for (size_t i = 0; i < lin.size(); ++i)
+        lin[i] = {linears[i].codes, linears[i].scales, linears[i].g};
+      nvq::StackM1 sm = {};
+      sm.lin = lin.data();
+      sm.n_layers = n_layers;
+      for (int i = 0; i < NVQ_STACK_LINEARS; ++i) {
+        sm.N[i] = Ns[i];
+        sm.outs[i] = outs[i];
+      }
+      sm.K0 = L0[kQ].K;
+      sm.Kd = L0[kDown].K;
+      sm.x_q = qa[0];
+      sm.x_d = da[0];
+      for (int i = 0; i < 3; ++i)
+        for (int par = 0; par < 2; ++par) {
+          sm.b_q[i][par] = qa[1 + 2 * i + par];
+          sm.b_d[i][par] = da[1 + 2 * i + par];
+        }
+      sm.cnt[0] = cnt;
+      sm.cnt[1] = cnt + L0[kV].N / 32;
+      sm.cnt[2] = sm.cnt[1] + L0[kO].N / 32;
+      sm.bar = reinterpret_cast<unsigned int*>(ws + lay.bar_off);
+      err = nvq::launch_stack_m1(sm, st);
+    }
+  } else if (M == 1) {
     // block counters start at zero; every launch leaves them at zero
     int* cnt = reinterpret_cast<int*>(ws + lay.cnt_off);
     int* cnt_v = cnt;

@@ -109,6 +109,48 @@ def test_one_token_stack_with_grouped_requantising_launches():
     assert capi.error_flags() == 0
 
 
+def per_launch_chain(layer, xd):
+    """One layer through the single-matrix entry points (Q8_0 quantiser,
+    nvq_gemv, nvq_gemv_requant), the kernels the persistent stack launch
+    must reproduce bit for bit."""
+    (cq, sq, gq), (ck, sk, gk), (cv, sv, gv), (co, so, go), (cu, su, gu), (cg, sg, gg), \
+        (cd, sd, gd) = layer
+    cnt = lambda N: torch.zeros(N // 32, dtype=torch.int32, device="cuda")
+    qx, dx = capi.quantize_act_q8_0(xd)
+    y_q = capi.gemv(cq, sq, gq, qx, dx)
+    y_k = capi.gemv(ck, sk, gk, qx, dx)
+    y_v, qv, dv = capi.gemv_requant(cv, sv, gv, qx, dx, cnt(cv.shape[0]))
+    y_o, qo, do_ = capi.gemv_requant(co, so, go, qv, dv, cnt(co.shape[0]))
+    y_u, qu, du = capi.gemv_requant(cu, su, gu, qo, do_, cnt(cu.shape[0]))
+    y_g = capi.gemv(cg, sg, gg, qo, do_)
+    y_d = capi.gemv(cd, sd, gd, qu, du)
+    torch.cuda.synchronize()
+    return [y_q, y_k, y_v, y_o, y_u, y_g, y_d]
+
+
+def test_persistent_one_token_stack_equals_per_launch_kernels():
+    """At one token the stack runs as one persistent launch per 64 layers
+    (phases separated by grid-wide counters, weights streamed across phase
+    boundaries).  Its outputs equal, bit for bit, those of the per-matrix
+    launches of the same layer; 66 layers (two launches, the second one
+    reusing the phase counters) give the same outputs as one layer, since
+    every layer restarts from the same x."""
+    h, f = 4096, 8192
+    stack1, packed = build_stack(1, h, f, 1, "persistent")
+    layer = [(packed[n].codes, packed[n].scales, packed[n].g) for n in ORDER]
+    stack66 = capi.DecoderStack([layer] * 66, 1)
+    x = wl.activations("stack_test", "xp", 1, h, "student_t4")
+    xd = torch.from_numpy(x).cuda()
+    ref = per_launch_chain(layer, xd)
+    out1 = [t.clone() for t in stack1.forward(xd)]
+    out66 = [t.clone() for t in stack66.forward(xd)]
+    torch.cuda.synchronize()
+    for name, r, a, b in zip(ORDER, ref, out1, out66):
+        assert torch.equal(a, r), name
+        assert torch.equal(b, r), name
+    assert capi.error_flags() == 0
+
+
 def test_stack_validates_shapes_and_workspace():
     h, f = 256, 512
     stack, _ = build_stack(1, h, f, 2, "val")
