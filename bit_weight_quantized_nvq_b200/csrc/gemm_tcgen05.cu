@@ -209,8 +209,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   // lo rows of half of the 128 tokens.
   const uint32_t rank = ptx::cluster_ctarank();
   const bool leader = rank == 0;
-  const int n0 = blockIdx.x * kBN;
-  const int m0 = blockIdx.y * kBT;
+  // pairs run token tiles fastest, so the CTAs of a wave share weight tiles
+  // (each weight byte comes from DRAM about once): cluster c takes token
+  // tile c % mt and weight tiles 2 (c / mt) and 2 (c / mt) + 1
+  const int mt = M_pad / kBT;
+  const int pc = blockIdx.x >> 1;
+  const int m0 = (pc % mt) * kBT;
+  const int n0 = ((pc / mt) * 2 + static_cast<int>(rank)) * kBN;
   const int num_kb = (K + kBK - 1) / kBK;   // the last stage may hold one sub-tile
   const int num_chunks = (num_kb + kChunk - 1) / kChunk;
 
@@ -657,7 +662,9 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   // pairs of CTAs along N: an even number of 128-row tiles (an odd last
   // tile gets an all-padding partner)
   const int64_t tiles_n = (N + kBN - 1) / kBN;
-  const dim3 grid(static_cast<unsigned>((tiles_n + 1) / 2 * 2), static_cast<unsigned>(M_pad / kBT));
+  const int64_t ctas = (tiles_n + 1) / 2 * 2 * (M_pad / kBT);
+  if (ctas > INT32_MAX) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(ctas));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
