@@ -263,28 +263,46 @@ quantize_nvfp4_long_kernel(const float* __restrict__ x, int K, uint8_t* __restri
 // ---------------------------------------------------------------------------
 // NVFP4 x NVFP4 GEMM
 // ---------------------------------------------------------------------------
-constexpr int kTile = 128;                 // weight rows (MMA M) and tokens (MMA N) per CTA
+constexpr int kTile = 128;                 // weight rows per CTA (MMA M)
 constexpr int kStageK = 256;               // K per stage: 128 code bytes per row
 constexpr int kMmaK = 64;                  // K per block-scaled MMA
-constexpr int kStages = 6;
-constexpr int kChunkStages = 4;            // stages per accumulator chunk (1024 K)
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr uint32_t kCodeTile = kTile * kStageK / 2;       // 16 KB
-constexpr uint32_t kScaleTile = kTile * kStageK / 16;     // 2 KB
-constexpr uint32_t kSlot = 2 * kCodeTile + 2 * kScaleTile;   // weights | tokens | w scales | t scales
-constexpr uint32_t kAccCols = kTile;                      // one accumulator: 128 fp32 columns
-constexpr uint32_t kSfCol0 = 2 * kAccCols;                // scale factors after the accumulators
-constexpr uint32_t kSfColsPerMma = kTile / 32;                 // 4 columns per operand
-constexpr uint32_t kSfColsPerOperand = (kStageK / kMmaK) * kSfColsPerMma;   // 16 per stage
-constexpr uint32_t kSfColsPerStage = 2 * kSfColsPerOperand;    // weights | tokens
 constexpr uint32_t kTmemCols = 512;
-static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory");
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
-// barriers: full[4] sf_full[4] empty[4] acc_full[2] acc_empty[2] mma_done
-constexpr int kNumBars = 3 * kStages + 5;
-constexpr uint32_t kSmemBytes = kStages * kSlot + kNumBars * 8 + 16 + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory");
+
+// The tile shape: TN tokens per CTA (the MMA's N).  TN = 128: a 6-deep ring
+// of 36 KB stages and two 128-column accumulators promoted every 1024 K.
+// TN = 256: twice the products per byte in flight (the kernel is bound by the
+// bytes it can keep in flight per SM against the memory latency), a 4-deep
+// ring of 54 KB stages and one 256-column accumulator promoted every 4096 K
+// (at most 64 accumulations in tensor memory, a relative error below
+// 64 * 2^-23 of the sum of |terms|, inside the accuracy bound).
+template <int TN>
+struct Nvf4Cfg {
+  static constexpr int kStages = TN == 128 ? 6 : 4;
+  static constexpr int kBufs = TN == 128 ? 2 : 1;          // accumulator buffers
+  static constexpr int kChunkStages = TN == 128 ? 4 : 16;  // stages per accumulator chunk
+  static constexpr int kEpiWarps = TN / 16;                // 64 token columns per warp
+  static constexpr int kThreads = 32 * (2 + kEpiWarps);
+  static constexpr uint32_t kCodeA = kTile * kStageK / 2;  // 16 KB
+  static constexpr uint32_t kCodeB = TN * kStageK / 2;     // 16 or 32 KB
+  static constexpr uint32_t kScaleA = kTile * kStageK / 16;
+  static constexpr uint32_t kScaleB = TN * kStageK / 16;
+  static constexpr uint32_t kOffB = kCodeA;
+  static constexpr uint32_t kOffSa = kCodeA + kCodeB;
+  static constexpr uint32_t kOffSb = kOffSa + kScaleA;
+  static constexpr uint32_t kSlot = kOffSb + kScaleB;
+  static constexpr uint32_t kAccCols = TN;
+  static constexpr uint32_t kSfCol0 = kBufs * kAccCols;
+  static constexpr uint32_t kSfA = kTile / 32;             // columns per K step: weights
+  static constexpr uint32_t kSfB = TN / 32;                //                     tokens
+  static constexpr uint32_t kSfColsA = (kStageK / kMmaK) * kSfA;
+  static constexpr uint32_t kSfColsPerStage = (kStageK / kMmaK) * (kSfA + kSfB);
+  static constexpr int kNumBars = 3 * kStages + 2 * kBufs + 1;
+  static constexpr uint32_t kSmemBytes = kStages * kSlot + kNumBars * 8 + 16 + 1024;
+  static_assert(kSlot % 1024 == 0, "slots stay 1024-byte aligned for the 128-byte swizzle");
+  static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor memory");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
 
 // bit 0: a pipeline wait timed out
 __device__ unsigned int g_nvf4_error_flags = 0;
@@ -318,45 +336,72 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Scale-factor layout in tensor memory, per operand of R rows and per 64-wide
+// K step: R/32 columns; lane i, column j holds the four scales (byte b for K
+// block b) of row 32*j + i, the same in every lane quarter.  A lane writes the
+// columns of one stage (4 K steps) of an R-row operand from the stage's
+// R x 16 scale bytes in shared memory.
+template <int R>
+__device__ __forceinline__ void store_scales(uint32_t smem_scales, uint32_t taddr, int lane) {
+  constexpr int J = R / 32;
+  // 16 columns (four K steps of J = 4 row groups, or two of J = 8) at a time
+  constexpr int kSteps = 16 / J;
+#pragma unroll
+  for (int h = 0; h < 4 / kSteps; ++h) {
+    uint32_t v[16];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const uint4 w = lds128(smem_scales + 16u * (32 * j + lane));
+      const uint32_t wk[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int t = 0; t < kSteps; ++t) v[t * J + j] = wk[h * kSteps + t];
+    }
+    ptx::tmem_st_16cols(taddr + 16u * h, v);
+  }
+}
+
+template <int TN>
+__global__ void __launch_bounds__(Nvf4Cfg<TN>::kThreads, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
                  const __grid_constant__ CUtensorMap wscale_map,
                  const __grid_constant__ CUtensorMap acode_map,
                  const __grid_constant__ CUtensorMap ascale_map, int N, int K, int M,
                  float g_w, const float* __restrict__ g_a, float* __restrict__ y) {
+  using C = Nvf4Cfg<TN>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t sbase = raw + ((1024u - (raw & 1023u)) & 1023u);
   uint8_t* smem = smem_raw + (sbase - raw);
-  const uint32_t bars = sbase + kStages * kSlot;
+  const uint32_t bars = sbase + S * C::kSlot;
   auto full = [&](int s) { return bars + 8u * s; };
-  auto sf_full = [&](int s) { return bars + 8u * (kStages + s); };
-  auto empty = [&](int s) { return bars + 8u * (2 * kStages + s); };
-  auto acc_full = [&](int b) { return bars + 8u * (3 * kStages + b); };
-  auto acc_empty = [&](int b) { return bars + 8u * (3 * kStages + 2 + b); };
-  const uint32_t mma_done = bars + 8u * (kNumBars - 1);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kStages * kSlot + kNumBars * 8);
+  auto sf_full = [&](int s) { return bars + 8u * (S + s); };
+  auto empty = [&](int s) { return bars + 8u * (2 * S + s); };
+  auto acc_full = [&](int b) { return bars + 8u * (3 * S + b); };
+  auto acc_empty = [&](int b) { return bars + 8u * (3 * S + C::kBufs + b); };
+  const uint32_t mma_done = bars + 8u * (C::kNumBars - 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + S * C::kSlot + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  auto slot = [&](int s) { return sbase + s * kSlot; };
+  auto slot = [&](int s) { return sbase + s * C::kSlot; };
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // token tiles vary fastest, so the CTAs of a wave share weight tiles
-  const int m0 = blockIdx.x * kTile;          // tokens
+  const int m0 = blockIdx.x * TN;             // tokens
   const int n0 = blockIdx.y * kTile;          // weight rows
   const int num_k = K / kStageK;
-  const int num_chunks = (num_k + kChunkStages - 1) / kChunkStages;
+  const int num_chunks = (num_k + C::kChunkStages - 1) / C::kChunkStages;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       ptx::mbar_init(full(s), 1);
       ptx::mbar_init(sf_full(s), 4);
       ptx::mbar_init(empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kBufs; ++b) {
       ptx::mbar_init(acc_full(b), 1);
-      ptx::mbar_init(acc_empty(b), kEpiWarps);
+      ptx::mbar_init(acc_empty(b), C::kEpiWarps);
     }
     ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -389,60 +434,59 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
     // ------------------------------- TMA producer ------------------------------
     // the weights are never written by the kernels before this one: the first
     // slots' weight tiles are requested before waiting for the token tiles
-    const int early = min(num_k, kStages);
+    const int early = min(num_k, S);
     if (lane == 0) {
       for (int k = 0; k < early; ++k) {
-        ptx::mbar_arrive_expect_tx(full(k), kSlot);
+        ptx::mbar_arrive_expect_tx(full(k), C::kSlot);
         ptx::tma_load_2d(slot(k), &wcode_map, k * (kStageK / 2), n0, full(k));
-        ptx::tma_load_2d(slot(k) + 2 * kCodeTile, &wscale_map, k * (kStageK / 16), n0, full(k));
+        ptx::tma_load_2d(slot(k) + C::kOffSa, &wscale_map, k * (kStageK / 16), n0, full(k));
       }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (lane == 0) {
       for (int k = 0; k < early; ++k) {
-        ptx::tma_load_2d(slot(k) + kCodeTile, &acode_map, k * (kStageK / 2), m0, full(k));
-        ptx::tma_load_2d(slot(k) + 2 * kCodeTile + kScaleTile, &ascale_map, k * (kStageK / 16),
-                         m0, full(k));
+        ptx::tma_load_2d(slot(k) + C::kOffB, &acode_map, k * (kStageK / 2), m0, full(k));
+        ptx::tma_load_2d(slot(k) + C::kOffSb, &ascale_map, k * (kStageK / 16), m0, full(k));
       }
     }
     __syncwarp();
     int issued = early;
     for (int k = early; k < num_k; ++k) {
-      const int s = k % kStages;
-      if (!warp_wait(empty(s), ((k / kStages) & 1) ^ 1)) {
+      const int s = k % S;
+      if (!warp_wait(empty(s), ((k / S) & 1) ^ 1)) {
         fail();
         break;
       }
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(full(s), kSlot);
+        ptx::mbar_arrive_expect_tx(full(s), C::kSlot);
         ptx::tma_load_2d(slot(s), &wcode_map, k * (kStageK / 2), n0, full(s));
-        ptx::tma_load_2d(slot(s) + kCodeTile, &acode_map, k * (kStageK / 2), m0, full(s));
-        ptx::tma_load_2d(slot(s) + 2 * kCodeTile, &wscale_map, k * (kStageK / 16), n0, full(s));
-        ptx::tma_load_2d(slot(s) + 2 * kCodeTile + kScaleTile, &ascale_map, k * (kStageK / 16), m0,
-                         full(s));
+        ptx::tma_load_2d(slot(s) + C::kOffB, &acode_map, k * (kStageK / 2), m0, full(s));
+        ptx::tma_load_2d(slot(s) + C::kOffSa, &wscale_map, k * (kStageK / 16), n0, full(s));
+        ptx::tma_load_2d(slot(s) + C::kOffSb, &ascale_map, k * (kStageK / 16), m0, full(s));
       }
       __syncwarp();
       ++issued;
     }
     if (*abort_flag) {
-      for (int k = max(0, issued - kStages); k < issued; ++k)
-        ptx::mbar_wait_bounded(full(k % kStages), (k / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int k = max(0, issued - S); k < issued; ++k)
+        ptx::mbar_wait_bounded(full(k % S), (k / S) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // -------------------------------- MMA issuer -------------------------------
-    constexpr uint32_t idesc = idesc_nvf4(kTile, kTile);
+    constexpr uint32_t idesc = idesc_nvf4(kTile, TN);
     bool ok = true;
     for (int c = 0; c < num_chunks && ok; ++c) {
-      const int b = c & 1;
-      if (c >= 2 && !warp_wait(acc_empty(b), ((c >> 1) - 1) & 1)) {
+      const int b = c % C::kBufs;
+      // a buffer is reused once the epilogue drained its previous chunk
+      if (c >= C::kBufs && !warp_wait(acc_empty(b), ((c / C::kBufs) - 1) & 1)) {
         fail();
         break;
       }
-      const uint32_t d_tmem = tmem_base + b * kAccCols;
-      const int k_end = min(num_k, (c + 1) * kChunkStages);
-      for (int k = c * kChunkStages; k < k_end; ++k) {
-        const int s = k % kStages;
-        if (!warp_wait(sf_full(s), (k / kStages) & 1)) {
+      const uint32_t d_tmem = tmem_base + b * C::kAccCols;
+      const int k_end = min(num_k, (c + 1) * C::kChunkStages);
+      for (int k = c * C::kChunkStages; k < k_end; ++k) {
+        const int s = k % S;
+        if (!warp_wait(sf_full(s), (k / S) & 1)) {
           fail();
           ok = false;
           break;
@@ -450,14 +494,14 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
         if (lane == 0) {
           ptx::tc_fence_after();
           const uint64_t adesc0 = ptx::sw128_kmajor_desc(slot(s));
-          const uint64_t bdesc0 = ptx::sw128_kmajor_desc(slot(s) + kCodeTile);
-          const uint32_t sf = tmem_base + kSfCol0 + s * kSfColsPerStage;
+          const uint64_t bdesc0 = ptx::sw128_kmajor_desc(slot(s) + C::kOffB);
+          const uint32_t sf = tmem_base + C::kSfCol0 + s * C::kSfColsPerStage;
 #pragma unroll
           for (int j = 0; j < kStageK / kMmaK; ++j) {
             // 64 E2M1 = 32 bytes per K step inside the 128-byte swizzled rows
-            mma_nvf4(d_tmem, adesc0 + 2u * j, bdesc0 + 2u * j, idesc, sf + kSfColsPerMma * j,
-                     sf + kSfColsPerOperand + kSfColsPerMma * j,
-                     (k == c * kChunkStages && j == 0) ? 0u : 1u);
+            mma_nvf4(d_tmem, adesc0 + 2u * j, bdesc0 + 2u * j, idesc, sf + C::kSfA * j,
+                     sf + C::kSfColsA + C::kSfB * j,
+                     (k == c * C::kChunkStages && j == 0) ? 0u : 1u);
           }
           ptx::mma_commit(empty(s));
           if (k == k_end - 1) ptx::mma_commit(acc_full(b));
@@ -471,25 +515,25 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
   } else {
     // ------------- scale factors to tensor memory; then the epilogue -----------
     const int q = warp & 3;                   // lane quarter
-    const int half = (warp - 2) >> 2;         // token columns [64*half, 64*half + 64)
+    const int part = (warp - 2) >> 2;         // token columns [64*part, 64*part + 64)
     const int r = q * 32 + lane;              // weight row of the accumulator lane
     const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
-    const bool mover = half == 0;
+    const bool mover = part == 0;
     float run[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) run[i] = 0.0f;
     int drained = 0;
     auto drain = [&]() -> bool {
-      const int b = drained & 1;
-      if (!warp_wait(acc_full(b), (drained >> 1) & 1)) return false;
+      const int b = drained % C::kBufs;
+      if (!warp_wait(acc_full(b), (drained / C::kBufs) & 1)) return false;
       ptx::tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        ptx::tmem_ld_32cols(tmem_base + tlane + b * kAccCols + 64 * half + 32 * cc, v);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[16];
+        ptx::tmem_ld_16cols(tmem_base + tlane + b * C::kAccCols + 64 * part + 16 * cc, v);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) run[32 * cc + i] += __uint_as_float(v[i]);
+        for (int i = 0; i < 16; ++i) run[16 * cc + i] += __uint_as_float(v[i]);
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -499,7 +543,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
     };
     bool ok = true;
     for (int k = 0; k < num_k && ok; ++k) {
-      if (k % kChunkStages == 0 && k / kChunkStages >= 2) {
+      // before the chunk that reuses a buffer, drain the chunk that used it
+      if (k % C::kChunkStages == 0 && k / C::kChunkStages >= C::kBufs) {
         if (!drain()) {
           fail();
           ok = false;
@@ -507,26 +552,16 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
         }
       }
       if (!mover) continue;
-      const int s = k % kStages;
-      if (!warp_wait(full(s), (k / kStages) & 1)) {
+      const int s = k % S;
+      if (!warp_wait(full(s), (k / S) & 1)) {
         fail();
         ok = false;
         break;
       }
-      // this lane's column j of K step t: word t of the 16 scale bytes of
-      // row 32*j + lane (the same in every lane quarter)
-      uint32_t va[16], vb[16];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 a4 = lds128(slot(s) + 2 * kCodeTile + 16u * (32 * j + lane));
-        const uint4 b4 = lds128(slot(s) + 2 * kCodeTile + kScaleTile + 16u * (32 * j + lane));
-        va[j] = a4.x, va[4 + j] = a4.y, va[8 + j] = a4.z, va[12 + j] = a4.w;
-        vb[j] = b4.x, vb[4 + j] = b4.y, vb[8 + j] = b4.z, vb[12 + j] = b4.w;
-      }
       ptx::tc_fence_after();
-      const uint32_t sf = tmem_base + tlane + kSfCol0 + s * kSfColsPerStage;
-      ptx::tmem_st_16cols(sf, va);
-      ptx::tmem_st_16cols(sf + kSfColsPerOperand, vb);
+      const uint32_t sf = tmem_base + tlane + C::kSfCol0 + s * C::kSfColsPerStage;
+      store_scales<kTile>(slot(s) + C::kOffSa, sf, lane);
+      store_scales<TN>(slot(s) + C::kOffSb, sf + C::kSfColsA, lane);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -544,7 +579,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
       if (n < N) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const int m = m0 + 64 * half + i;
+          const int m = m0 + 64 * part + i;
           if (m < M) y[static_cast<size_t>(m) * N + n] = run[i] * (g_w * g_a[m]);
         }
       }
@@ -625,30 +660,42 @@ cudaError_t launch_quantize_nvfp4(const float* x, int64_t M, int64_t K, uint8_t*
   return cudaLaunchKernelEx(&cfg, quantize_nvfp4_kernel, x, k, codes, scales, g);
 }
 
-cudaError_t launch_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w,
-                             int64_t N, int64_t K, const uint8_t* a_codes,
-                             const uint8_t* a_scales, const float* g_a, int64_t M, float* y,
-                             cudaStream_t stream) {
+template <int TN>
+cudaError_t launch_nvf4_t(const uint8_t* w_codes, const uint8_t* w_scales, float g_w, int64_t N,
+                          int64_t K, const uint8_t* a_codes, const uint8_t* a_scales,
+                          const float* g_a, int64_t M, float* y, cudaStream_t stream) {
+  using C = Nvf4Cfg<TN>;
   CUtensorMap wc, ws, ac, as;
   if (!encode_bytes_2d(&wc, w_codes, K / 2, N, 128, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_bytes_2d(&ws, w_scales, K / 16, N, 16, kTile, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_bytes_2d(&ac, a_codes, K / 2, M, 128, kTile, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_bytes_2d(&as, a_scales, K / 16, M, 16, kTile, CU_TENSOR_MAP_SWIZZLE_NONE))
+      !encode_bytes_2d(&ac, a_codes, K / 2, M, 128, TN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_bytes_2d(&as, a_scales, K / 16, M, 16, TN, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   static SmemAttrOnce attr;
-  cudaError_t e = attr.ensure(gemm_nvf4_kernel, static_cast<int>(kSmemBytes));
+  cudaError_t e = attr.ensure(gemm_nvf4_kernel<TN>, static_cast<int>(C::kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((M + kTile - 1) / kTile),
+  cfg.gridDim = dim3(static_cast<unsigned>((M + TN - 1) / TN),
                      static_cast<unsigned>((N + kTile - 1) / kTile));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute a[1] = {pdl_attr()};
   cfg.attrs = a;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_nvf4_kernel, wc, ws, ac, as, static_cast<int>(N),
+  return cudaLaunchKernelEx(&cfg, gemm_nvf4_kernel<TN>, wc, ws, ac, as, static_cast<int>(N),
                             static_cast<int>(K), static_cast<int>(M), g_w, g_a, y);
+}
+
+cudaError_t launch_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float g_w,
+                             int64_t N, int64_t K, const uint8_t* a_codes,
+                             const uint8_t* a_scales, const float* g_a, int64_t M, float* y,
+                             cudaStream_t stream) {
+  // the 256-token tile when its grid still fills every SM at least twice
+  const int64_t tiles256 = ((M + 255) / 256) * ((N + kTile - 1) / kTile);
+  if (tiles256 >= 2 * static_cast<int64_t>(device_sm_count()))
+    return launch_nvf4_t<256>(w_codes, w_scales, g_w, N, K, a_codes, a_scales, g_a, M, y, stream);
+  return launch_nvf4_t<128>(w_codes, w_scales, g_w, N, K, a_codes, a_scales, g_a, M, y, stream);
 }
 
 cudaError_t nvf4_error_flags(bool clear, unsigned int* flags) {

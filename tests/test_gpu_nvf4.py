@@ -9,7 +9,8 @@
 * the GEMM on shapes the oracle finishes in seconds, every element compared:
   one 128-token tile and several, ragged weight rows and tokens (not a
   multiple of the 128-row tile), one K stage and K long enough to use both
-  accumulator buffers several times;
+  accumulator buffers several times; and the 256-token tiles (single
+  accumulator promoted every 4096 K) on sampled rows;
 * the prefill shapes at full size, sampled weight rows and tokens;
 * zero scales give zero, a zero token gives a zero row, repeated calls are
   bit-identical, bad shapes are refused before any launch;
@@ -96,6 +97,25 @@ def test_gemm_all_elements(M, N, K):
     torch.cuda.synchronize()
     y_ref, sa = reference(wref, aref)
     assert_within_tolerance(y.cpu().numpy(), y_ref, sa)
+    assert capi.error_flags() == 0
+
+
+# 256-token tiles (chosen when they still fill every SM twice: here 2 token
+# tiles x 149 weight tiles): a full tile and a ragged one (300 tokens), one
+# K stage and K = 4352 (two chunks of the single accumulator: 16 + 1 stages).
+@pytest.mark.parametrize("M,N,K", [(512, 19000, 256), (300, 19000, 4352)])
+def test_gemm_256_token_tiles_sampled_rows(M, N, K):
+    W = wl.weights("nvf4_test", "W256", N, K)
+    x = wl.activations("nvf4_test", "x256", M, K, "student_t4", outliers=True)
+    codes, scales, g = capi.pack_nvfp4(W)
+    rows = sample_rows(N, 96, seed=M + N + K)
+    wref = o.pack_nvfp4(W[rows], g=o.nvfp4_tensor_scale(W))
+    assert np.array_equal(codes[rows], wref[0]) and np.array_equal(scales[rows], wref[1])
+    (ac, as_, ag), aref = quantize_nvf4_both(x)
+    y = capi.gemm_nvf4(to_dev(codes), to_dev(scales), g, ac, as_, ag)
+    torch.cuda.synchronize()
+    y_ref, sa = reference(wref, aref)
+    assert_within_tolerance(y.cpu().numpy()[:, rows], y_ref, sa)
     assert capi.error_flags() == 0
 
 
