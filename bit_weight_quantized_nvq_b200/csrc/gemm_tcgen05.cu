@@ -182,7 +182,7 @@ expand_act_kernel(const int8_t* __restrict__ q, const __half* __restrict__ d, in
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restrict__ codes,
             const uint8_t* __restrict__ scales, int N, int K, int M, int M_pad, float g,
-            const float* __restrict__ tok_scale, float* __restrict__ y) {
+            const float* __restrict__ tok_scale, float* __restrict__ y, int tok_fast) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -209,13 +209,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   // lo rows of half of the 128 tokens.
   const uint32_t rank = ptx::cluster_ctarank();
   const bool leader = rank == 0;
-  // pairs run token tiles fastest, so the CTAs of a wave share weight tiles
-  // (each weight byte comes from DRAM about once): cluster c takes token
-  // tile c % mt and weight tiles 2 (c / mt) and 2 (c / mt) + 1
+  // The tile order keeps the larger operand's tiles shared by the CTAs of a
+  // wave, so that it comes from DRAM about once: with token tiles fastest
+  // (tok_fast) cluster c takes token tile c % mt and weight pair c / mt;
+  // else weight pair c % np and token tile c / np.
   const int mt = M_pad / kBT;
+  const int np = gridDim.x / (2 * mt);
   const int pc = blockIdx.x >> 1;
-  const int m0 = (pc % mt) * kBT;
-  const int n0 = ((pc / mt) * 2 + static_cast<int>(rank)) * kBN;
+  const int tt = tok_fast ? pc % mt : pc / np;
+  const int wp = tok_fast ? pc / mt : pc % np;
+  const int m0 = tt * kBT;
+  const int n0 = (wp * 2 + static_cast<int>(rank)) * kBN;
   const int num_kb = (K + kBK - 1) / kBK;   // the last stage may hold one sub-tile
   const int num_chunks = (num_kb + kChunk - 1) / kChunk;
 
@@ -677,9 +681,12 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   cluster[0].val.clusterDim.z = 1;
   cfg.attrs = cluster;
   cfg.numAttrs = 1;
+  // token tiles fastest when the packed weights are the larger operand
+  // (0.5625 B per weight against 4 B per token and K of expanded activations)
+  const int tok_fast = 9 * N >= 64 * M_pad ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, gemm_kernel, map, codes, scales, static_cast<int>(N),
                                      static_cast<int>(K), static_cast<int>(M),
-                                     static_cast<int>(M_pad), g, tok_scale, y);
+                                     static_cast<int>(M_pad), g, tok_scale, y, tok_fast);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
