@@ -26,14 +26,16 @@
 //  * warps 2..17 (four per tensor-memory lane quarter, each taking 64 of a
 //    stage's 256 K) expand the codes to fp16 w' and store them with
 //    tcgen05.st into a 3-deep ring in tensor memory (row r in lane r);
-//  * warp 1 issues tcgen05.mma.kind::f16 (M = 128, N = 2 x padded tokens:
-//    hi and lo columns side by side, K = 16) with A from tensor memory and
-//    B from shared memory, 16 per stage; the accumulator is promoted to
-//    fp32 registers every 1024 K (4 stages), alternating between two
-//    tensor-memory buffers (the tensor core's fp32 accumulation truncates,
-//    so long chains are split);
-//  * the four warps with the first K part also drain the accumulators and
-//    write y = g * tok_scale * (hi + lo).
+//  * warps 1 and 18 (on different sub-partitions: one thread issues a small
+//    MMA only every ~70 cycles, far below the tensor core's rate) issue
+//    tcgen05.mma.kind::f16 (M = 128, N = 2 x padded tokens: hi and lo
+//    columns side by side, K = 16) with A from tensor memory and B from
+//    shared memory, 8 each per stage (the K steps of one parity) into their
+//    own accumulators; these are promoted to fp32 registers every 1024 K
+//    (4 stages), alternating between two tensor-memory buffers each (the
+//    tensor core's fp32 accumulation truncates, so long chains are split);
+//  * the four warps with the first K part also drain the accumulators (the
+//    two issuers' added in a fixed order) and write y = g * tok_scale * (hi + lo).
 // Every wait is bounded (4 s); a timeout raises an error flag and the CTA
 // drains what it issued before freeing tensor memory and leaving.
 #include <algorithm>
@@ -58,7 +60,9 @@ constexpr int kSmemStages = 4;        // shared-memory ring (codes, scales, acti
 constexpr int kAStages = 3;           // tensor-memory ring of expanded weights
 constexpr int kChunkStages = 4;       // stages accumulated per TMEM buffer (1024 K)
 constexpr int kDecWarps = 16;
-constexpr int kThreads = 32 * (2 + kDecWarps);
+constexpr int kIssuers = 2;          // MMA-issuing warps (1 and kIssuer2)
+constexpr int kIssuer2 = 2 + kDecWarps;   // warp 18: another sub-partition than warp 1
+constexpr int kThreads = 32 * (3 + kDecWarps);
 constexpr uint32_t kACols = kStageK / 2;                 // 128 columns per A stage
 constexpr uint32_t kAccCol0 = kAStages * kACols;         // 384: accumulators after the A ring
 constexpr uint32_t kTmemCols = 512;
@@ -80,7 +84,7 @@ __host__ __device__ constexpr uint32_t smem_bytes(int n) {
 }
 static_assert(slot_bytes(16) % 1024 == 0 && slot_bytes(32) % 1024 == 0, "1 KB aligned slots");
 static_assert(smem_bytes(32) <= 232448, "over the opt-in shared memory of one CTA");
-static_assert(kAccCol0 + 2 * 32 <= kTmemCols, "tensor memory");
+static_assert(kAccCol0 + kIssuers * 2 * 32 <= kTmemCols, "tensor memory");
 
 // bit 0: a pipeline wait timed out
 __device__ unsigned int g_gemm_small_error_flags = 0;
@@ -167,17 +171,17 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSmemStages; ++s) {
       ptx::mbar_init(full(s), 1);
-      ptx::mbar_init(empty(s), 1);
+      ptx::mbar_init(empty(s), kIssuers);
     }
     for (int s = 0; s < kAStages; ++s) {
       ptx::mbar_init(a_full(s), kDecWarps);
-      ptx::mbar_init(a_empty(s), 1);
+      ptx::mbar_init(a_empty(s), kIssuers);
     }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(acc_full(b), 1);
+      ptx::mbar_init(acc_full(b), kIssuers);
       ptx::mbar_init(acc_empty(b), 4);
     }
-    ptx::mbar_init(mma_done, 1);
+    ptx::mbar_init(mma_done, kIssuers);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tensormap(&code_map);
@@ -273,8 +277,13 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
         ptx::mbar_wait_bounded(full(k % kSmemStages), static_cast<uint32_t>((k / kSmemStages) & 1),
                                nullptr, kWaitLimitNs);
     }
-  } else if (warp == 1) {
-    // ------------------------------- MMA issuer --------------------------------
+  } else if (warp == 1 || warp == kIssuer2) {
+    // ------------------------------ MMA issuers ---------------------------------
+    // One thread issues a small MMA only every ~70 cycles, far slower than the
+    // tensor core runs it, so two warps on different sub-partitions issue:
+    // issuer i takes the K steps of parity i of every stage into its own
+    // double-buffered accumulator (the drain adds the two).
+    const int is = warp == 1 ? 0 : 1;
     constexpr uint32_t idesc = ptx::idesc_f16_f32(kRows, NT);
     Pieces pc{u0, u1, Ks};
     int t, j0, j1;
@@ -289,7 +298,7 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
           ok = false;
           break;
         }
-        const uint32_t d_tmem = tmem_base + kAccCol0 + b * NT;
+        const uint32_t d_tmem = tmem_base + kAccCol0 + (is * 2 + b) * NT;
         const int je = min(j1, jc + kChunkStages);
         for (int j = jc; j < je; ++j, sm.advance(), ar.advance()) {
           if (!warp_wait(full(sm.slot), sm.phase) || !warp_wait(a_full(ar.slot), ar.phase)) {
@@ -304,10 +313,10 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
 #pragma unroll
             for (int sub = 0; sub < kSubs; ++sub) {
 #pragma unroll
-              for (int k = 0; k < kSubK / 16; ++k) {
+              for (int k = is; k < kSubK / 16; k += kIssuers) {
                 const uint32_t a = a_cols + sub * (kSubK / 2) + 8u * k;
                 const uint64_t bd = bdesc0 + ((sub * act_sub_bytes(NT)) >> 4) + 2u * k;
-                ptx::mma_f16_ts(d_tmem, a, bd, idesc, (j == jc && sub == 0 && k == 0) ? 0u : 1u);
+                ptx::mma_f16_ts(d_tmem, a, bd, idesc, (j == jc && sub == 0 && k == is) ? 0u : 1u);
               }
             }
             ptx::mma_commit(empty(sm.slot));
@@ -351,14 +360,18 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap code_map,
       const int b = drained & 1;
       if (!warp_wait(acc_full(b), static_cast<uint32_t>((drained >> 1) & 1))) return false;
       ptx::tc_fence_after();
-      uint32_t v[NT];
-      if constexpr (NT == 32)
-        ptx::tmem_ld_32cols(tmem_base + tlane + kAccCol0 + b * NT, v);
-      else
-        ptx::tmem_ld_16cols(tmem_base + tlane + kAccCol0 + b * NT, v);
-      ptx::tmem_wait_ld();
+      // the two issuers' accumulators of buffer b, added in a fixed order
 #pragma unroll
-      for (int n = 0; n < NT; ++n) run[n] += __uint_as_float(v[n]);
+      for (int i = 0; i < kIssuers; ++i) {
+#pragma unroll
+        for (int h = 0; h < NT / 16; ++h) {
+          uint32_t v[16];
+          ptx::tmem_ld_16cols(tmem_base + tlane + kAccCol0 + (i * 2 + b) * NT + 16 * h, v);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int n = 0; n < 16; ++n) run[16 * h + n] += __uint_as_float(v[n]);
+        }
+      }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(acc_empty(b));
