@@ -435,15 +435,40 @@ __host__ __device__ __forceinline__ int reg_block_slots(int rows, int G) {
   return (rows + G - 1) / G / 32 + 2;
 }
 
-// The next stage of a CTA's concatenated row range: at most R rows, all of
-// one matrix.
-__device__ __forceinline__ void next_stage(const RegGroup& grp, int& gr, int r_end, int R,
-                                           int& mi, int& row0, int& nrows) {
-  mi = 0;
-  while (mi + 1 < grp.count && gr >= grp.m[mi + 1].row_off) ++mi;
-  row0 = gr - grp.m[mi].row_off;
-  nrows = min(R, min(r_end - gr, grp.m[mi].N - row0));
-  gr += nrows;
+// A CTA's walk over its concatenated rows, stage by stage: the matrix of the
+// next row and that matrix's concatenated rows [off, end), held in
+// registers.  The group (launch parameters, or shared memory) is read again
+// only when the walk enters another matrix, not at every stage: a lookup
+// per stage sits on the consumers' path from one stage to the next.
+struct RowWalk {
+  int gr;        // next concatenated row
+  int mi;        // its matrix
+  int off, end;
+};
+__device__ __forceinline__ RowWalk walk_begin(const RegGroup& grp, int r_begin) {
+  RowWalk w;
+  w.gr = r_begin;
+  w.mi = 0;
+  while (w.mi + 1 < grp.count && r_begin >= grp.m[w.mi + 1].row_off) ++w.mi;
+  w.off = grp.m[w.mi].row_off;
+  w.end = w.off + grp.m[w.mi].N;
+  return w;
+}
+// The next stage (called while w.gr < r_end): at most R rows, all of one
+// matrix.  Returns true when the walk entered another matrix.
+__device__ __forceinline__ bool walk_next(const RegGroup& grp, RowWalk& w, int r_end, int R,
+                                          int& row0, int& nrows) {
+  bool entered = false;
+  while (w.gr >= w.end) {
+    ++w.mi;
+    w.off = grp.m[w.mi].row_off;
+    w.end = w.off + grp.m[w.mi].N;
+    entered = true;
+  }
+  row0 = w.gr - w.off;
+  nrows = min(R, min(r_end, w.end) - w.gr);
+  w.gr += nrows;
+  return entered;
 }
 
 template <int NPL, int WPR, bool ISUM, bool MOE>
@@ -545,8 +570,10 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
     };
     int issued = 0;
     bool ok = true;
-    int gr = r_begin;
-    for (int it = 0; gr < r_end; ++it) {
+    RowWalk wk = walk_begin(grp, r_begin);
+    const uint8_t* m_codes = grp.m[wk.mi].codes;
+    const uint8_t* m_scales = grp.m[wk.mi].scales;
+    for (int it = 0; wk.gr < r_end; ++it) {
       const int s = it % kM1Stages;
       const uint32_t ph = (it / kM1Stages) & 1;
       if (it == kM1Stages) {
@@ -560,19 +587,21 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
         break;
       }
       if (it >= kM1Stages) finalize(it - kM1Stages);
-      int mi, row0, nrows;
-      next_stage(grp, gr, r_end, R, mi, row0, nrows);
-      smi[s] = mi;
+      int row0, nrows;
+      if (walk_next(grp, wk, r_end, R, row0, nrows)) {
+        m_codes = grp.m[wk.mi].codes;
+        m_scales = grp.m[wk.mi].scales;
+      }
+      smi[s] = wk.mi;
       srow[s] = row0;
       snr[s] = nrows;
-      const RegMat& m = grp.m[mi];
       const uint32_t bar = ptx::smem_addr(full + s);
       uint8_t* st = smem + s * stage_bytes;
       ptx::mbar_arrive_expect_tx(bar, nrows * (row_code + row_scale));
-      ptx::bulk_load(ptx::smem_addr(st), m.codes + static_cast<size_t>(row0) * row_code,
+      ptx::bulk_load(ptx::smem_addr(st), m_codes + static_cast<size_t>(row0) * row_code,
                      nrows * row_code, bar);
       ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
-                     m.scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
+                     m_scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
       ++issued;
     }
     if (!waited) grid_dependency_wait();
@@ -618,12 +647,20 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
     c0[i] = -12 * s0;
     c1[i] = -12 * s1;
   }
-  int gr = r_begin;
-  for (int it = 0; gr < r_end; ++it) {
+  // the epilogue's fields of the current matrix, in registers
+  RowWalk wk = walk_begin(grp, r_begin);
+  float* m_y = grp.m[wk.mi].y;
+  float m_half_g = grp.m[wk.mi].half_g;
+  bool m_rq = grp.m[wk.mi].rq_q != nullptr;
+  for (int it = 0; wk.gr < r_end; ++it) {
     const int s = it % kM1Stages;
     const uint32_t ph = (it / kM1Stages) & 1;
-    int mi, row0, nrows;
-    next_stage(grp, gr, r_end, R, mi, row0, nrows);
+    int row0, nrows;
+    if (walk_next(grp, wk, r_end, R, row0, nrows)) {
+      m_y = grp.m[wk.mi].y;
+      m_half_g = grp.m[wk.mi].half_g;
+      m_rq = grp.m[wk.mi].rq_q != nullptr;
+    }
     if (!ptx::mbar_wait_bounded(ptx::smem_addr(full + s), ph, abort_flag, kWaitLimitNs)) {
       *abort_flag = 1;
       raise_timeout();
@@ -631,7 +668,6 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
     }
     float acc = 0.0f;
     if (rl < nrows) {
-      const RegMat& m = grp.m[mi];
       const uint8_t* st = smem + s * stage_bytes;
       const uint4* cw = reinterpret_cast<const uint4*>(st + rl * row_code) + p * (NPL * 32);
       const uint16_t* sw =
@@ -648,7 +684,8 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
         const int i0 = dev::dot16_biased(w[i].x, w[i].y, qa[i], c0[i]);
         const int i1 = dev::dot16_biased(w[i].z, w[i].w, qb[i], c1[i]);
         if constexpr (ISUM)
-          store_isum(isum, 0, m.N, row0 + rl, K, p * (NPL * 32) + lane + 32 * i, i0, i1);
+          store_isum(isum, 0, grp.m[wk.mi].N, row0 + rl, K, p * (NPL * 32) + lane + 32 * i, i0,
+                     i1);
         const float2 sf = dev::ue4m3x2_to_float2(s2[i]);
         acc = fmaf(dd[i], fmaf(sf.x, static_cast<float>(i0), sf.y * static_cast<float>(i1)), acc);
       }
@@ -656,11 +693,10 @@ gemv_m1_reg_kernel(const __grid_constant__ RegGroup grp_param, const __grid_cons
       if (WPR == 1) {
         const int row = row0 + rl;
         int how = 0;
-        if (lane == 0) {
-          m.y[row] = acc * m.half_g;
-          if (m.rq_q != nullptr) how = arrive_row(m, row, m.row_off + row, r_begin, r_end, scnt);
-        }
-        if (m.rq_q != nullptr) {
+        if (lane == 0) m_y[row] = acc * m_half_g;
+        if (m_rq) {
+          const RegMat& m = grp.m[wk.mi];
+          if (lane == 0) how = arrive_row(m, row, m.row_off + row, r_begin, r_end, scnt);
           how = __shfl_sync(0xffffffffu, how, 0);
           if (how != 0) {
             if (how == 1) __threadfence_block(); else __threadfence();
