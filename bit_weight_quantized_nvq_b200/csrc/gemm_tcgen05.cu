@@ -20,9 +20,8 @@
 //  * the tensor core's fp32 accumulation does not round to nearest (its
 //    error grows with the number of chained MMAs and is biased toward
 //    zero: about 1e-5 of sum|terms| after 1600 of them at K = 25600), so
-//    partial sums are promoted: each 512-wide K chunk accumulates in one of
-//    two TMEM buffers and the epilogue threads add it to fp32 registers
-//    (round to nearest) while the tensor core fills the other buffer.
+//    partial sums are promoted: each 2048-wide K chunk accumulates in TMEM
+//    and the epilogue threads add it to fp32 registers (round to nearest).
 //
 // Kernels:
 //  1. expand_act_kernel: Q8_0 (q, d) -> fp16 [hi rows | lo rows] in the
@@ -31,19 +30,22 @@
 //     scaled by 2^-e first and the epilogue multiplies by 2^e.
 //  2. gemm_kernel: CTA pairs (clusters of 2).  Each CTA owns 128 weight
 //     rows; the pair shares a tile of 128 tokens and the even CTA issues
-//     tcgen05.mma.cta_group::2 (M = 256, N = 128, K = 16) for both:
+//     tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16) for both:
 //       warp 0    TMA: this CTA's hi and lo rows of 64 of the tokens, for
 //                 the two 64-wide K sub-tiles of a 128-wide stage (four
 //                 64 x 64 fp16 boxes, 128-byte swizzle), into a 4-stage ring;
 //       warp 1    allocates the pair's 512 TMEM columns; in the even CTA it
-//                 waits for each stage and issues 16 pair MMAs (hi and lo of
-//                 8 K-steps into the same accumulator), with A read from
-//                 tensor memory and B from both CTAs' shared memory;
+//                 waits for each stage and issues 8 pair MMAs (M = 256,
+//                 N = 256, K = 16): each CTA's B rows are its 64 tokens' hi
+//                 rows followed by their lo rows, one 128-row operand, so a
+//                 single MMA forms the hi and the lo products of all 128
+//                 tokens in 256 accumulator columns.  A is read from tensor
+//                 memory and B from both CTAs' shared memory;
 //       warps 2-9 two threads per weight row, one per sub-tile: cp.async the
 //                 packed codes and scales, decode them to fp16 w' and
 //                 tcgen05.st them into the 4-stage A ring in tensor memory
-//                 (row m in lane m); drain finished 512-wide K chunks into
-//                 fp32 registers; store y;
+//                 (row m in lane m); drain finished 2048-wide K chunks
+//                 (hi + lo of each token) into fp32 registers; store y;
 //       warp 10   forwards "this CTA's rows of the stage landed" to the even
 //                 CTA's stage barrier.
 //     Every role runs with its whole warp converged on the waits (a wait in
@@ -66,7 +68,7 @@ namespace nvq {
 namespace {
 
 constexpr int kBN = 128;            // weight rows per CTA = TMEM lanes
-constexpr int kBT = 128;            // tokens per tile = pair MMA N (hi and lo issued separately)
+constexpr int kBT = 128;            // tokens per tile; the pair MMA's N = 256 holds their hi and lo
 constexpr int kBTc = kBT / 2;       // tokens whose hi and lo rows one CTA of the pair loads
 constexpr int kBK = 128;            // K per stage: two 64-wide sub-tiles
 constexpr int kSubK = 64;           // K per 128-byte fp16 swizzle row (TMA box, MMA tile)
@@ -82,10 +84,15 @@ constexpr int kThreads = 32 * (kFwdWarp + 1);
 constexpr int kEPT = kBK / kTPR;    // K elements one thread expands per stage (64)
 constexpr int kCPT = kEPT / 2;      // their code bytes = TMEM columns (32)
 static_assert(kTPR == kSubs && kEPT == kSubK, "thread part p expands sub-tile p");
-constexpr int kChunk = 4;           // K stages accumulated per TMEM buffer (512 K)
-constexpr uint32_t kAccCols = kBT;                  // one accumulator: 128 fp32 columns
+constexpr int kChunk = 16;          // K stages accumulated in TMEM before promotion (2048 K)
+static_assert(kChunk % (2 * kStages) == 0,
+              "a chunk is an even number of passes over the ring (stage parity = pass parity)");
+// The accumulator: 256 fp32 columns, [hi | lo of tokens 0-63 | hi | lo of
+// tokens 64-127] (each CTA's 128 B rows in turn).  There is room for one:
+// the issuer waits while the epilogue drains it, once per chunk.
+constexpr uint32_t kAccCols = 2 * kBT;
 constexpr uint32_t kACols = kBK / 2;                // one A stage: 128 fp16 = 64 columns
-constexpr uint32_t kAColBase = 2 * kAccCols;        // A ring after the two accumulators
+constexpr uint32_t kAColBase = kAccCols;            // A ring after the accumulator
 constexpr uint32_t kTmemCols = kAColBase + kStages * kACols;   // 512
 static_assert(kTmemCols == 512, "the tile uses all of tensor memory");
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
@@ -98,7 +105,7 @@ constexpr uint32_t kOffB = 0;
 constexpr uint32_t kOffCodes = kOffB + kStages * kBStageBytes;
 constexpr uint32_t kOffScales = kOffCodes + kCStages * kCodeStageBytes;
 constexpr uint32_t kOffBars = kOffScales + kCStages * kScaleStageBytes;
-// full_b, stage_full, stage_empty, acc_full[2], acc_empty[2], mma_done
+// full_b, stage_full, stage_empty, acc_full, acc_empty (two slots each, one used), mma_done
 constexpr uint32_t kNumBars = 3 * kStages + 5;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + slack to align to 1024
@@ -305,7 +312,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   } else if (warp == 1) {
     // -------------------------- pair MMA issuer (leader) ------------------------
     if (leader) {
-      constexpr uint32_t idesc = ptx::idesc_f16_f32(2 * kBN, kBT);
+      constexpr uint32_t idesc = ptx::idesc_f16_f32(2 * kBN, 2 * kBT);
       // completion of the pair MMAs is signalled to the same barrier in both CTAs
       auto commit_both = [&](uint32_t bar) {
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 0));
@@ -313,55 +320,55 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       };
       // The issuing thread is paced by the tensor core, so every instruction
       // between MMA bursts is a bubble (more so as the warp shares its
-      // scheduler with two decoding warps): a chunk is one pass over the
-      // ring, unrolled, so stage indices and flags are constants and the
-      // descriptors are plain adds, and a stage holds 16 MMAs per wait.
-      // (Issuing through a predicate from the converged warp, instead of the
-      // lane-0 branch, measured slower.)
-      static_assert(kChunk == kStages, "one chunk = one pass over the ring");
+      // scheduler with two decoding warps): one pass over the ring is
+      // unrolled, so stage indices are constants and the descriptors are
+      // plain adds.  (Issuing through a predicate from the converged warp,
+      // instead of the lane-0 branch, measured slower.)
       const uint32_t a_cols0 = tmem_base + kAColBase;
       const uint64_t bdesc0 = ptx::sw128_kmajor_desc(sbase + kOffB);
+      const uint32_t d_tmem = tmem_base;
       bool ok_mma = true;
       for (int c = 0; c < num_chunks && ok_mma; ++c) {
-        const int b = c & 1;
-        const uint32_t parity = c & 1;
-        const uint32_t d_tmem = tmem_base + b * kAccCols;
-        // a buffer is reused two chunks later, once both epilogues drained it
-        if (c >= 2 && !warp_wait(acc_empty(b), ((c >> 1) - 1) & 1)) {
+        // the accumulator is reused once the epilogue drained the last chunk
+        if (c >= 1 && !warp_wait(acc_empty(0), (c - 1) & 1)) {
           fail();
           break;
         }
+        const int nst = min(kChunk, num_kb - c * kChunk);   // stages of this chunk
+        for (int pass = 0; pass * kStages < nst && ok_mma; ++pass) {
 #pragma unroll
-        for (int j = 0; j < kStages; ++j) {
-          const int kb = c * kChunk + j;
-          if (kb >= num_kb) break;
-          if (!warp_wait(stage_full(j), parity)) {
-            fail();
-            ok_mma = false;
-            break;
-          }
-          if (lane == 0) {
-            ptx::tc_fence_after();
-            const uint32_t a_cols = a_cols0 + j * kACols;
-            const uint64_t bdesc = bdesc0 + ((j * kBStageBytes) >> 4);
-            const bool two = kb * kBK + kSubK < K;   // the last stage may hold one sub-tile
-#pragma unroll
-            for (int sub = 0; sub < kSubs; ++sub) {
-              if (sub == 1 && !two) break;
-#pragma unroll
-              for (int k = 0; k < kSubK / 16; ++k) {
-                // hi and lo products go to the same accumulator; descriptor
-                // start addresses are in 16-byte units (32 bytes = next 16 K)
-                const uint32_t a = a_cols + sub * (kSubK / 2) + 8u * k;
-                const uint64_t bhi = bdesc + ((sub * 2 * kBSubBytes) >> 4) + 2u * k;
-                ptx::mma_f16_ts_pair(d_tmem, a, bhi, idesc, (j == 0 && sub == 0 && k == 0) ? 0u : 1u);
-                ptx::mma_f16_ts_pair(d_tmem, a, bhi + (kBSubBytes >> 4), idesc, 1u);
-              }
+          for (int j = 0; j < kStages; ++j) {
+            const int kb = c * kChunk + pass * kStages + j;
+            if (pass * kStages + j >= nst) break;
+            if (!warp_wait(stage_full(j), pass & 1)) {
+              fail();
+              ok_mma = false;
+              break;
             }
-            commit_both(stage_empty(j));
-            if (j == kStages - 1 || kb == num_kb - 1) commit_both(acc_full(b));
+            if (lane == 0) {
+              ptx::tc_fence_after();
+              const uint32_t a_cols = a_cols0 + j * kACols;
+              const uint64_t bdesc = bdesc0 + ((j * kBStageBytes) >> 4);
+              const bool two = kb * kBK + kSubK < K;   // the last stage may hold one sub-tile
+              const bool first = pass == 0 && j == 0;
+#pragma unroll
+              for (int sub = 0; sub < kSubs; ++sub) {
+                if (sub == 1 && !two) break;
+#pragma unroll
+                for (int k = 0; k < kSubK / 16; ++k) {
+                  // B: this CTA's [hi | lo] rows of the sub-tile, one 128-row
+                  // operand; descriptor start addresses are in 16-byte units
+                  // (32 bytes = next 16 K)
+                  const uint32_t a = a_cols + sub * (kSubK / 2) + 8u * k;
+                  const uint64_t bk = bdesc + ((sub * 2 * kBSubBytes) >> 4) + 2u * k;
+                  ptx::mma_f16_ts_pair(d_tmem, a, bk, idesc, (first && sub == 0 && k == 0) ? 0u : 1u);
+                }
+              }
+              commit_both(stage_empty(j));
+              if (pass * kStages + j == nst - 1) commit_both(acc_full(0));
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
       }
       // no MMA may still be reading or writing tensor memory when it is released
@@ -414,27 +421,34 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     for (int j = 0; j < kCols; ++j) run[j] = 0.0f;
     int drained = 0;
     int stored = 0;   // stages whose A tile this warp stored
-    // add finished chunk c to the fp32 registers and hand its buffer back
+    // add finished chunk c to the fp32 registers (hi + lo of each of this
+    // thread's tokens: columns 2 * kCols * p + j and + kCols) and hand the
+    // accumulator back
     auto drain = [&](int c) -> bool {
-      const int b = c & 1;
-      if (!warp_wait(acc_full(b), (c >> 1) & 1)) return false;
+      if (!warp_wait(acc_full(0), c & 1)) return false;
       ptx::tc_fence_after();
-      const uint32_t base = tmem_base + tlane + b * kAccCols + kCols * p;
+      const uint32_t base = tmem_base + tlane + 2 * kCols * p;
 #pragma unroll
       for (int cc = 0; cc < kCols / 32; ++cc) {
-        uint32_t v[32];
-        ptx::tmem_ld_32cols(base + 32u * cc, v);
+        uint32_t vh[32], vl[32];
+        ptx::tmem_ld_32cols(base + 32u * cc, vh);
+        ptx::tmem_ld_32cols(base + kCols + 32u * cc, vl);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) run[cc * 32 + j] += __uint_as_float(v[j]);
+        for (int j = 0; j < 32; ++j)
+          run[cc * 32 + j] += __uint_as_float(vh[j]) + __uint_as_float(vl[j]);
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(leader_acc_empty0 + 8u * b);
+      if (lane == 0) ptx::mbar_arrive_cluster(leader_acc_empty0);
       return true;
     };
     for (int kb = 0; kb < num_kb; ++kb) {
-      if ((kb % kChunk) == 0 && kb / kChunk >= 2) {
+      // Chunk c - 1 is drained before stage c * kChunk + kStages - 1 is
+      // expanded (that stage waits for the chunk's last MMAs anyway); the
+      // issuer waits for the accumulator before chunk c, whose first stages
+      // are ready by then.
+      if (kb >= kChunk && kb % kChunk == kStages - 1) {
         if (!drain(drained++)) {
           fail();
           ok = false;
