@@ -20,7 +20,7 @@
 //  * the tensor core's fp32 accumulation does not round to nearest (its
 //    error grows with the number of chained MMAs and is biased toward
 //    zero: about 1e-5 of sum|terms| after 1600 of them at K = 25600), so
-//    partial sums are promoted: each 2048-wide K chunk accumulates in TMEM
+//    partial sums are promoted: each chunk of up to 5120 K accumulates in TMEM
 //    and the epilogue threads add it to fp32 registers (round to nearest).
 //
 // Kernels:
@@ -44,7 +44,7 @@
 //       warps 2-9 two threads per weight row, one per sub-tile: cp.async the
 //                 packed codes and scales, decode them to fp16 w' and
 //                 tcgen05.st them into the 4-stage A ring in tensor memory
-//                 (row m in lane m); drain finished 2048-wide K chunks
+//                 (row m in lane m); drain finished K chunks
 //                 (hi + lo of each token) into fp32 registers; store y;
 //       warp 10   forwards "this CTA's rows of the stage landed" to the even
 //                 CTA's stage barrier.
@@ -54,6 +54,8 @@
 //     an error flag and the CTA drains what it issued, and the pair frees
 //     TMEM together after a cluster barrier.
 #include <algorithm>
+#include <atomic>
+#include <climits>
 #include <mutex>
 
 #include <cuda.h>
@@ -84,9 +86,16 @@ constexpr int kThreads = 32 * (kFwdWarp + 1);
 constexpr int kEPT = kBK / kTPR;    // K elements one thread expands per stage (64)
 constexpr int kCPT = kEPT / 2;      // their code bytes = TMEM columns (32)
 static_assert(kTPR == kSubs && kEPT == kSubK, "thread part p expands sub-tile p");
-constexpr int kChunk = 16;          // K stages accumulated in TMEM before promotion (2048 K)
-static_assert(kChunk % (2 * kStages) == 0,
-              "a chunk is an even number of passes over the ring (stage parity = pass parity)");
+// K stages accumulated in TMEM before promotion: at most kChunk (5120 K),
+// a tile's part split into chunks of equal length.  A promotion stops the
+// issuer until the tensor core has finished every queued MMA and the
+// epilogue has read the accumulator (~1.6 us), so chunks are as long as the
+// accumulation error allows.
+constexpr int kChunk = 40;
+__host__ __device__ __forceinline__ int chunk_len(int left) {
+  const int n = (left + kChunk - 1) / kChunk;
+  return (left + n - 1) / n;
+}
 // The accumulator: 256 fp32 columns, [hi | lo of tokens 0-63 | hi | lo of
 // tokens 64-127] (each CTA's 128 B rows in turn).  There is room for one:
 // the issuer waits while the epilogue drains it, once per chunk.
@@ -105,8 +114,8 @@ constexpr uint32_t kOffB = 0;
 constexpr uint32_t kOffCodes = kOffB + kStages * kBStageBytes;
 constexpr uint32_t kOffScales = kOffCodes + kCStages * kCodeStageBytes;
 constexpr uint32_t kOffBars = kOffScales + kCStages * kScaleStageBytes;
-// full_b, stage_full, stage_empty, acc_full, acc_empty (two slots each, one used), mma_done
-constexpr uint32_t kNumBars = 3 * kStages + 5;
+// full_b, stage_full, stage_empty, acc_full, acc_empty, mma_done
+constexpr uint32_t kNumBars = 3 * kStages + 3;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;   // + slack to align to 1024
 static_assert(kOffCodes % 1024 == 0, "swizzled tiles need 1 KB alignment");
@@ -186,10 +195,95 @@ expand_act_kernel(const int8_t* __restrict__ q, const __half* __restrict__ d, in
 // ---------------------------------------------------------------------------
 // 2. the tcgen05 GEMM
 // ---------------------------------------------------------------------------
+// The work of one CTA pair.  The T tiles (128 tokens x 256 weight rows) are
+// numbered as the launcher orders them; with P pairs, the first W * P tiles
+// (W = T / P) go round-robin, whole: pair j takes tiles j, j + P, ..., so a
+// wave of pairs shares operand tiles as in a plain tiled grid.  The K stages
+// of the R = T - W * P remaining tiles are split evenly over all pairs
+// (stream-K): pair j takes the stages [R * num_kb * j / P, R * num_kb *
+// (j + 1) / P) of those tiles in order, so no pair idles in a last partial
+// wave.  A tile whose stages are split leaves each part's fp32 sums in a
+// slot of the workspace (a pair's first and last stream-K parts: slots 0
+// and 1), and gemm_fixup_kernel adds the parts in K order.  The pair's
+// stages are numbered g = 0 .. G-1 in the order it processes them.
+struct PairWork {
+  int num_kb, P, j, W, T_dp;
+  int sk_b;       // first stream-K stage of this pair (over the R last tiles)
+  int G;          // stages of this pair
+  int tile_sk0;   // tile of the pair's first stream-K stage (-1: none)
+
+  __device__ __forceinline__ void init(int T, int nkb, int pairs, int pair) {
+    num_kb = nkb;
+    P = pairs;
+    j = pair;
+    W = T / P;
+    T_dp = W * P;
+    // the launcher keeps T * num_kb within int32
+    const int64_t U_r = static_cast<int64_t>(T - T_dp) * num_kb;
+    sk_b = static_cast<int>(U_r * j / P);
+    const int sk_e = static_cast<int>(U_r * (j + 1) / P);
+    G = W * num_kb + (sk_e - sk_b);
+    tile_sk0 = sk_e > sk_b ? T_dp + static_cast<int>(sk_b / num_kb) : -1;
+  }
+  // tile (in the launcher's order) and K stage of stage g
+  __device__ __forceinline__ void stage(int g, int& tile, int& kb) const {
+    const int dp = W * num_kb;
+    if (g < dp) {
+      tile = j + (g / num_kb) * P;
+      kb = g % num_kb;
+    } else {
+      const int u = sk_b + (g - dp);
+      tile = T_dp + u / num_kb;
+      kb = u - (u / num_kb) * num_kb;
+    }
+  }
+  // stages from g (K stage kb) to the end of its tile's part
+  __device__ __forceinline__ int part_left(int g, int kb) const {
+    return min(num_kb - kb, G - g);
+  }
+};
+
+// The pair's stages one after another, without a division but where the
+// walk enters the stream-K stages.
+struct StageCursor {
+  int g, tile, kb;
+  __device__ __forceinline__ void begin(const PairWork& w) {
+    g = 0;
+    w.stage(0, tile, kb);
+  }
+  __device__ __forceinline__ void next(const PairWork& w) {
+    ++g;
+    ++kb;
+    const int dp = w.W * w.num_kb;
+    if (g == dp) {
+      if (g < w.G) w.stage(g, tile, kb);
+    } else if (kb == w.num_kb) {
+      kb = 0;
+      tile += g < dp ? w.P : 1;
+    }
+  }
+};
+
+// Tile index -> (token tile, weight pair).  With token tiles fastest
+// (tok_fast) consecutive tiles share the weight rows, else the tokens.
+__host__ __device__ __forceinline__ void tile_coords(int tile, int mt, int np, int tok_fast,
+                                                     int& tt, int& wp) {
+  tt = tok_fast ? tile % mt : tile / np;
+  wp = tok_fast ? tile / mt : tile % np;
+}
+
+// fp32 sums of one CTA's part of a tile: [p][j / 4][rt] float4, where thread
+// (rt, p) of the epilogue holds tokens 64 p + j of weight row rt
+constexpr int kPartFloats = kBN * kBT;   // 64 KB
+__device__ __forceinline__ float4* part_slot(float* parts, int cta, int slot) {
+  return reinterpret_cast<float4*>(parts + (static_cast<size_t>(cta) * 2 + slot) * kPartFloats);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restrict__ codes,
             const uint8_t* __restrict__ scales, int N, int K, int M, int M_pad, float g,
-            const float* __restrict__ tok_scale, float* __restrict__ y, int tok_fast) {
+            const float* __restrict__ tok_scale, float* __restrict__ y, int T, int np,
+            int tok_fast, float* __restrict__ parts) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
@@ -199,47 +293,41 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   // stage_full(s):  (leader) stage s complete in both CTAs: A written by all
   //                 expansion warps of the pair, both CTAs' B rows forwarded
   // stage_empty(s): the pair MMAs of stage s finished (committed to both CTAs)
+  // acc_full:       the MMAs of a chunk finished;  acc_empty: both CTAs'
+  //                 epilogues read the accumulator
   auto full_b = [&](int s) { return sbase + kOffBars + 8u * s; };
   auto stage_full = [&](int s) { return sbase + kOffBars + 8u * (kStages + s); };
   auto stage_empty = [&](int s) { return sbase + kOffBars + 8u * (2 * kStages + s); };
   constexpr uint32_t kOffAcc = 8u * (3 * kStages);
-  auto acc_full = [&](int b) { return sbase + kOffBars + kOffAcc + 8u * b; };
-  auto acc_empty = [&](int b) { return sbase + kOffBars + kOffAcc + 8u * (2 + b); };
-  const uint32_t mma_done = sbase + kOffBars + kOffAcc + 32u;
+  const uint32_t acc_full = sbase + kOffBars + kOffAcc;
+  const uint32_t acc_empty = acc_full + 8u;
+  const uint32_t mma_done = acc_full + 16u;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // The two CTAs of a cluster are a pair: CTA 0 (the leader) issues the
-  // pair MMAs for both.  Each CTA owns 128 weight rows and loads the hi and
-  // lo rows of half of the 128 tokens.
+  // pair MMAs for both.  Each CTA owns 128 weight rows of a tile and loads
+  // the hi and lo rows of half of its 128 tokens.
   const uint32_t rank = ptx::cluster_ctarank();
   const bool leader = rank == 0;
-  // The tile order keeps the larger operand's tiles shared by the CTAs of a
-  // wave, so that it comes from DRAM about once: with token tiles fastest
-  // (tok_fast) cluster c takes token tile c % mt and weight pair c / mt;
-  // else weight pair c % np and token tile c / np.
   const int mt = M_pad / kBT;
-  const int np = gridDim.x / (2 * mt);
-  const int pc = blockIdx.x >> 1;
-  const int tt = tok_fast ? pc % mt : pc / np;
-  const int wp = tok_fast ? pc / mt : pc % np;
-  const int m0 = tt * kBT;
-  const int n0 = (wp * 2 + static_cast<int>(rank)) * kBN;
   const int num_kb = (K + kBK - 1) / kBK;   // the last stage may hold one sub-tile
-  const int num_chunks = (num_kb + kChunk - 1) / kChunk;
+  // the pair's schedule lives in shared memory: its fields are read where
+  // the walks change tiles, and kept out of the registers of the loops
+  __shared__ PairWork work_s;
+  const PairWork& work = work_s;
 
   if (threadIdx.x == 0) {
+    work_s.init(T, num_kb, static_cast<int>(gridDim.x >> 1), static_cast<int>(blockIdx.x >> 1));
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(full_b(s), 1);
       ptx::mbar_init(stage_full(s), 2 * kExpWarps + 2);
       ptx::mbar_init(stage_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(acc_full(b), 1);
-      ptx::mbar_init(acc_empty(b), 2 * kExpWarps);
-    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::mbar_init(acc_empty, 2 * kExpWarps);
     ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -253,6 +341,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   ptx::cluster_sync();   // both CTAs' barriers exist before any remote arrival
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  const int G = work.G;
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -270,22 +359,32 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   if (warp == 0) {
     // ------------------------------- TMA producer ------------------------------
     int issued = 0;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % kStages;
-      const uint32_t ph = (kb / kStages) & 1;
+    StageCursor cur;
+    cur.begin(work);
+    int tok_tile = -1, tok0 = 0;   // this CTA's first token row of the current tile
+    for (int gs = 0; gs < G; ++gs, cur.next(work)) {
+      const int s = gs % kStages;
+      const uint32_t ph = (gs / kStages) & 1;
       if (!warp_wait(stage_empty(s), ph ^ 1)) {
         fail();
         break;
       }
+      if (cur.tile != tok_tile) {
+        int tt, wp;
+        tile_coords(cur.tile, mt, np, tok_fast, tt, wp);
+        tok_tile = cur.tile;
+        tok0 = tt * kBT + kBTc * static_cast<int>(rank);
+      }
       if (lane == 0) {
+        const int kb = cur.kb;
         const uint32_t dst = sbase + kOffB + s * kBStageBytes;
         const int nsub = min(kSubs, (K - kb * kBK) / kSubK);
         ptx::mbar_arrive_expect_tx(full_b(s), nsub * 2 * kBSubBytes);
         for (int sub = 0; sub < nsub; ++sub) {
           const uint32_t d0 = dst + sub * 2 * kBSubBytes;
           const int kx = kb * kBK + sub * kSubK;
-          ptx::tma_load_2d(d0, &act_map, kx, m0 + kBTc * rank, full_b(s));
-          ptx::tma_load_2d(d0 + kBSubBytes, &act_map, kx, M_pad + m0 + kBTc * rank, full_b(s));
+          ptx::tma_load_2d(d0, &act_map, kx, tok0, full_b(s));
+          ptx::tma_load_2d(d0 + kBSubBytes, &act_map, kx, M_pad + tok0, full_b(s));
         }
       }
       __syncwarp();
@@ -294,15 +393,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     if (*abort_flag) {
       // the MMAs may have stopped: wait for this CTA's copies in flight
       // before the CTA can leave
-      for (int kb = std::max(0, issued - kStages); kb < issued; ++kb)
-        ptx::mbar_wait_bounded(full_b(kb % kStages), (kb / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int gs = std::max(0, issued - kStages); gs < issued; ++gs)
+        ptx::mbar_wait_bounded(full_b(gs % kStages), (gs / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == kFwdWarp) {
     // ------------ forwarder: this CTA's activation rows have landed ---------
     const uint32_t leader_stage_full0 = ptx::mapa_shared(stage_full(0), 0);
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % kStages;
-      if (!warp_wait(full_b(s), (kb / kStages) & 1)) {
+    for (int gs = 0; gs < G; ++gs) {
+      const int s = gs % kStages;
+      if (!warp_wait(full_b(s), (gs / kStages) & 1)) {
         fail();
         break;
       }
@@ -318,56 +417,70 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 0));
         ptx::mma_commit_pair(ptx::mapa_shared(bar, 1));
       };
-      // The issuing thread is paced by the tensor core, so every instruction
-      // between MMA bursts is a bubble (more so as the warp shares its
-      // scheduler with two decoding warps): one pass over the ring is
-      // unrolled, so stage indices are constants and the descriptors are
-      // plain adds.  (Issuing through a predicate from the converged warp,
-      // instead of the lane-0 branch, measured slower.)
+      // The issuing thread is on the tensor core's critical path (it issues
+      // about as fast as the MMAs run), so the loop keeps its ring position,
+      // barrier and operand addresses in registers and advances them by
+      // constants: a few instructions per stage besides the MMAs.
       const uint32_t a_cols0 = tmem_base + kAColBase;
       const uint64_t bdesc0 = ptx::sw128_kmajor_desc(sbase + kOffB);
       const uint32_t d_tmem = tmem_base;
+      const uint32_t full0 = stage_full(0);
+      const uint32_t empty0_r0 = ptx::mapa_shared(stage_empty(0), 0);
+      const uint32_t empty0_r1 = ptx::mapa_shared(stage_empty(0), 1);
+      const uint32_t accf_r0 = ptx::mapa_shared(acc_full, 0);
+      const uint32_t accf_r1 = ptx::mapa_shared(acc_full, 1);
+      const int kb_one = K % kBK != 0 ? num_kb - 1 : -1;   // the stage with one sub-tile
+      int s = 0;            // ring slot of the next stage
+      uint32_t ph = 0;      // its phase parity
       bool ok_mma = true;
-      for (int c = 0; c < num_chunks && ok_mma; ++c) {
+      // chunks: at most kChunk stages of one tile's part; the accumulator
+      // starts from zero at each
+      int gc = 0;
+      for (int gs = 0; gs < G && ok_mma; ++gc) {
+        int tile, kb;
+        work.stage(gs, tile, kb);
+        const int n = chunk_len(work.part_left(gs, kb));
+        gs += n;
         // the accumulator is reused once the epilogue drained the last chunk
-        if (c >= 1 && !warp_wait(acc_empty(0), (c - 1) & 1)) {
+        if (gc >= 1 && !warp_wait(acc_empty, (gc - 1) & 1)) {
           fail();
           break;
         }
-        const int nst = min(kChunk, num_kb - c * kChunk);   // stages of this chunk
-        for (int pass = 0; pass * kStages < nst && ok_mma; ++pass) {
+        for (int i = 0; i < n; ++i, ++kb) {
+          if (!warp_wait(full0 + 8u * s, ph)) {
+            fail();
+            ok_mma = false;
+            break;
+          }
+          if (lane == 0) {
+            ptx::tc_fence_after();
+            const uint32_t a_cols = a_cols0 + s * kACols;
+            const uint64_t bdesc = bdesc0 + s * (kBStageBytes >> 4);
 #pragma unroll
-          for (int j = 0; j < kStages; ++j) {
-            const int kb = c * kChunk + pass * kStages + j;
-            if (pass * kStages + j >= nst) break;
-            if (!warp_wait(stage_full(j), pass & 1)) {
-              fail();
-              ok_mma = false;
-              break;
-            }
-            if (lane == 0) {
-              ptx::tc_fence_after();
-              const uint32_t a_cols = a_cols0 + j * kACols;
-              const uint64_t bdesc = bdesc0 + ((j * kBStageBytes) >> 4);
-              const bool two = kb * kBK + kSubK < K;   // the last stage may hold one sub-tile
-              const bool first = pass == 0 && j == 0;
+            for (int sub = 0; sub < kSubs; ++sub) {
+              if (sub == 1 && kb == kb_one) break;
 #pragma unroll
-              for (int sub = 0; sub < kSubs; ++sub) {
-                if (sub == 1 && !two) break;
-#pragma unroll
-                for (int k = 0; k < kSubK / 16; ++k) {
-                  // B: this CTA's [hi | lo] rows of the sub-tile, one 128-row
-                  // operand; descriptor start addresses are in 16-byte units
-                  // (32 bytes = next 16 K)
-                  const uint32_t a = a_cols + sub * (kSubK / 2) + 8u * k;
-                  const uint64_t bk = bdesc + ((sub * 2 * kBSubBytes) >> 4) + 2u * k;
-                  ptx::mma_f16_ts_pair(d_tmem, a, bk, idesc, (first && sub == 0 && k == 0) ? 0u : 1u);
-                }
+              for (int k = 0; k < kSubK / 16; ++k) {
+                // B: this CTA's [hi | lo] rows of the sub-tile, one 128-row
+                // operand; descriptor start addresses are in 16-byte units
+                // (32 bytes = next 16 K)
+                const uint32_t a = a_cols + sub * (kSubK / 2) + 8u * k;
+                const uint64_t bk = bdesc + ((sub * 2 * kBSubBytes) >> 4) + 2u * k;
+                ptx::mma_f16_ts_pair(d_tmem, a, bk, idesc,
+                                     (i == 0 && sub == 0 && k == 0) ? 0u : 1u);
               }
-              commit_both(stage_empty(j));
-              if (pass * kStages + j == nst - 1) commit_both(acc_full(0));
             }
-            __syncwarp();
+            ptx::mma_commit_pair(empty0_r0 + 8u * s);
+            ptx::mma_commit_pair(empty0_r1 + 8u * s);
+            if (i == n - 1) {
+              ptx::mma_commit_pair(accf_r0);
+              ptx::mma_commit_pair(accf_r1);
+            }
+          }
+          __syncwarp();
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
           }
         }
       }
@@ -380,30 +493,55 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     // ------------------- weight expansion, then the epilogue ------------------
     // A warp may only touch the TMEM lanes of its quarter (warp % 4), so the
     // threads of TMEM lane rt = 32 * (warp % 4) + lane expand weight row
-    // n0 + rt: warp group p = (warp - 2) / 4 takes sub-tile p of each
-    // 128-wide K stage (kEPT = 64 elements, TMEM columns kCPT * p ..).  In the
-    // epilogue the same threads split the 128 token columns.
+    // rt of the CTA's 128 rows of each tile: warp group p = (warp - 2) / 4
+    // takes sub-tile p of each 128-wide K stage (kEPT = 64 elements, TMEM
+    // columns kCPT * p ..).  In the epilogue the same threads split the 128
+    // token columns.
     const int quarter = warp & 3;
     const int p = (warp - 2) >> 2;
     const int rt = quarter * 32 + lane;
-    const int row = n0 + rt;
-    const bool valid = row < N;
-    const uint8_t* crow = codes + static_cast<size_t>(valid ? row : 0) * (K / 2) + kCPT * p;
-    const uint8_t* srow = scales + static_cast<size_t>(valid ? row : 0) * (K / 16) + 4 * p;
     const uint32_t stg_c = sbase + kOffCodes + 64u * rt + kCPT * p;
     const int t = threadIdx.x - 64;    // 0 .. kExpThreads - 1
     const uint32_t stg_s = sbase + kOffScales + 4u * t;
-    auto issue = [&](int kb) {
-      if (kb < num_kb) {
-        const uint32_t slot = kb % kCStages;
-        // this thread's sub-tile exists (K is a multiple of 64): else zero fill
-        // from an in-bounds address
-        const bool in = valid && kb * kBK + p * kSubK < K;
-        const uint8_t* c_src = in ? crow + (kBK / 2) * kb : crow;
-        const uint8_t* s_src = in ? srow + (kBK / 16) * kb : srow;
+    // weight row of this thread in tile `tile` (N: none)
+    auto tile_row = [&](int tile) {
+      int tt, wp;
+      tile_coords(tile, mt, np, tok_fast, tt, wp);
+      return (wp * 2 + static_cast<int>(rank)) * kBN + rt;
+    };
+    // Prefetch of the packed codes and scales, kCStages - 1 stages ahead of
+    // the expansion: source pointers advance by one stage's bytes, and are
+    // set again (with the divisions of the pair's schedule) only where the
+    // walk starts another tile's part.
+    const uint8_t* pf_c = codes;
+    const uint8_t* pf_s = scales;
+    int pf_kb = 0, pf_left = 0;
+    bool pf_row_ok = false;
+    auto issue = [&](int gs) {
+      if (gs < G) {
+        if (pf_left == 0) {
+          int tile;
+          work.stage(gs, tile, pf_kb);
+          pf_left = work.part_left(gs, pf_kb);
+          const int row = tile_row(tile);
+          pf_row_ok = row < N;
+          const size_t r = pf_row_ok ? static_cast<size_t>(row) : 0;
+          pf_c = codes + r * (K / 2) + kCPT * p + (kBK / 2) * static_cast<size_t>(pf_kb);
+          pf_s = scales + r * (K / 16) + 4 * p + (kBK / 16) * static_cast<size_t>(pf_kb);
+        }
+        const uint32_t slot = gs % kCStages;
+        // this thread's sub-tile exists (K is a multiple of 64): else zero
+        // fill from an in-bounds address
+        const bool in = pf_row_ok && pf_kb * kBK + p * kSubK < K;
+        const uint8_t* c_src = in ? pf_c : codes;
+        const uint8_t* s_src = in ? pf_s : scales;
         ptx::cp_async_16(stg_c + slot * kCodeStageBytes, c_src, in ? 16u : 0u);
         ptx::cp_async_16(stg_c + slot * kCodeStageBytes + 16, c_src + (in ? 16 : 0), in ? 16u : 0u);
         ptx::cp_async_4(stg_s + slot * kScaleStageBytes, s_src, in ? 4u : 0u);
+        pf_c += kBK / 2;
+        pf_s += kBK / 16;
+        ++pf_kb;
+        --pf_left;
       }
       ptx::cp_async_commit();
     };
@@ -411,72 +549,143 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
     // One arrival per warp (lane 0, after __syncwarp); arrivals go to the
     // leader's barriers.
     const uint32_t leader_stage_full0 = ptx::mapa_shared(stage_full(0), 0);
-    const uint32_t leader_acc_empty0 = ptx::mapa_shared(acc_empty(0), 0);
+    const uint32_t leader_acc_empty = ptx::mapa_shared(acc_empty, 0);
     bool ok = true;
     const uint32_t tlane = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t a_dst = tmem_base + tlane + kAColBase + kCPT * p;
     constexpr int kCols = kBT / kTPR;
-    float run[kCols];
+    // The chunk to drain next: first stage dg, dn stages, the chunk count,
+    // and about the tile's part it belongs to: whether the chunk is its
+    // first, whether the part is the whole tile, and its slot if not (0: the
+    // pair's first stream-K part, else 1).
+    int dg = 0, dn = 0, dc = 0, slot_idx = 0;
+    bool chunk_first = true, whole = true;
+    auto next_chunk = [&]() {
+      if (dg >= G) return;
+      int tile, kb;
+      work.stage(dg, tile, kb);
+      const int left = work.part_left(dg, kb);
+      dn = chunk_len(left);
+      chunk_first = kb == 0 || dg == 0 || dg == work.W * num_kb;
+      if (chunk_first) {
+        whole = kb == 0 && left == num_kb;
+        slot_idx = tile == work.tile_sk0 ? 0 : 1;
+      }
+    };
+    next_chunk();
+    // Drain the next chunk: this thread's 64 token sums (hi + lo: columns
+    // 2 * kCols * p + j and + kCols), then hand the accumulator back.  The
+    // sums go to the part's destination: y (a whole tile, scaled when the
+    // part is complete) or the part's slot.  A part of several chunks keeps
+    // its running sum there: each later chunk adds itself to it, in order.
+    auto drain = [&]() -> bool {
+      // everything but the accumulator is worked out before its wait: this
+      // chunk's destination, and the next chunk
+      int tile, kb;
+      work.stage(dg, tile, kb);
+      const bool last = dn == work.part_left(dg, kb);
+      const bool first = chunk_first, to_y = whole;
+      int tt, wp;
+      tile_coords(tile, mt, np, tok_fast, tt, wp);
+      const int nrow = tile_row(tile);
+      const int m0t = tt * kBT + kCols * p;   // this thread's first token
+      float4* slot = part_slot(parts, blockIdx.x, slot_idx);
+      const int this_dc = dc;
+      dg += dn;
+      ++dc;
+      next_chunk();
+      // the running sum of the part (every load issued before any use, and
+      // before the wait, so that they overlap it)
+      float acc[kCols];
 #pragma unroll
-    for (int j = 0; j < kCols; ++j) run[j] = 0.0f;
-    int drained = 0;
-    int stored = 0;   // stages whose A tile this warp stored
-    // add finished chunk c to the fp32 registers (hi + lo of each of this
-    // thread's tokens: columns 2 * kCols * p + j and + kCols) and hand the
-    // accumulator back
-    auto drain = [&](int c) -> bool {
-      if (!warp_wait(acc_full(0), c & 1)) return false;
+      for (int j = 0; j < kCols; ++j) acc[j] = 0.0f;
+      if (!first) {
+        if (to_y) {
+          if (nrow < N) {
+#pragma unroll
+            for (int j = 0; j < kCols; ++j)
+              if (m0t + j < M) acc[j] = __ldcg(y + static_cast<size_t>(m0t + j) * N + nrow);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kCols; j += 4) {
+            const float4 o = __ldcg(slot + (p * (kCols / 4) + j / 4) * kBN + rt);
+            acc[j] = o.x, acc[j + 1] = o.y, acc[j + 2] = o.z, acc[j + 3] = o.w;
+          }
+        }
+      }
+      if (!warp_wait(acc_full, this_dc & 1)) return false;
       ptx::tc_fence_after();
       const uint32_t base = tmem_base + tlane + 2 * kCols * p;
 #pragma unroll
-      for (int cc = 0; cc < kCols / 32; ++cc) {
-        uint32_t vh[32], vl[32];
-        ptx::tmem_ld_32cols(base + 32u * cc, vh);
-        ptx::tmem_ld_32cols(base + kCols + 32u * cc, vl);
+      for (int h = 0; h < kCols / 16; ++h) {
+        uint32_t hi[16], lo[16];
+        ptx::tmem_ld_16cols(base + 16u * h, hi);
+        ptx::tmem_ld_16cols(base + kCols + 16u * h, lo);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          run[cc * 32 + j] += __uint_as_float(vh[j]) + __uint_as_float(vl[j]);
+        for (int j = 0; j < 16; ++j)
+          acc[h * 16 + j] += __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(leader_acc_empty0);
+      if (lane == 0) ptx::mbar_arrive_cluster(leader_acc_empty);
+      if (to_y) {
+        if (nrow < N) {
+#pragma unroll
+          for (int j = 0; j < kCols; ++j) {
+            const int m = m0t + j;
+            if (m < M)
+              y[static_cast<size_t>(m) * N + nrow] = last ? acc[j] * (g * tok_scale[m]) : acc[j];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kCols; j += 4)
+          slot[(p * (kCols / 4) + j / 4) * kBN + rt] =
+              make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+      }
       return true;
     };
-    for (int kb = 0; kb < num_kb; ++kb) {
-      // Chunk c - 1 is drained before stage c * kChunk + kStages - 1 is
-      // expanded (that stage waits for the chunk's last MMAs anyway); the
-      // issuer waits for the accumulator before chunk c, whose first stages
-      // are ready by then.
-      if (kb >= kChunk && kb % kChunk == kStages - 1) {
-        if (!drain(drained++)) {
+    // A chunk is drained at the top of the iteration kStages stages after its
+    // last one: that stage waits for the chunk's last MMAs anyway, and the
+    // issuer waits for the accumulator before the next chunk, whose first
+    // stages are ready by then.  After the last stage the loop only drains
+    // (one copy of the drain in the code: the warps' loops share the
+    // instruction cache with the issuing thread).
+    int next_drain = G > 0 ? dn - 1 + kStages : INT_MAX;
+    for (int gs = 0;; ++gs) {
+      while (gs >= next_drain) {
+        if (!drain()) {
           fail();
           ok = false;
           break;
         }
+        next_drain = dg < G ? dg + dn - 1 + kStages : INT_MAX;
       }
+      if (!ok || next_drain == INT_MAX) break;
+      if (gs >= G) continue;
       ptx::cp_async_wait<kCStages - 2>();
-      const int s = kb % kStages;
-      if (!warp_wait(stage_empty(s), ((kb / kStages) & 1) ^ 1)) {
+      const int s = gs % kStages;
+      if (!warp_wait(stage_empty(s), ((gs / kStages) & 1) ^ 1)) {
         fail();
         ok = false;
         break;
       }
       ptx::tc_fence_after();
-      const int cs = kb % kCStages;
+      const int cs = gs % kCStages;
       const uint8_t* stg = smem + kOffCodes + cs * kCodeStageBytes + 64 * rt + kCPT * p;
       const uint32_t sc = *reinterpret_cast<const uint32_t*>(
           smem + kOffScales + cs * kScaleStageBytes + 4 * t);
       // The previous stage's tensor-memory store is waited for (and the
       // stage announced) only after this stage's decode, so the store's
-      // latency overlaps the decode instead of stalling the warp.
-      auto announce_prev = [&]() {
-        if (kb > 0) {
-          ptx::tmem_wait_st();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * ((kb - 1) % kStages));
-        }
+      // latency overlaps the decode instead of stalling the warp; the last
+      // stage is announced right after its store.
+      auto announce = [&](int st) {
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * (st % kStages));
       };
       {
         // sub-tile p: subblocks 0..3 of it, 8 codes per 32-bit word
@@ -494,36 +703,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
                                 e2.x, e2.y, e2.z, e2.w, e3.x, e3.y, e3.z, e3.w,
                                 e4.x, e4.y, e4.z, e4.w, e5.x, e5.y, e5.z, e5.w,
                                 e6.x, e6.y, e6.z, e6.w, e7.x, e7.y, e7.z, e7.w};
-        announce_prev();
+        if (gs > 0) announce(gs - 1);
         ptx::tmem_st_32cols(a_dst + s * kACols, v);
       }
-      issue(kb + kCStages - 1);
-      ++stored;
-    }
-    if (stored > 0) {
-      // announce the last stage this warp stored
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(leader_stage_full0 + 8u * ((stored - 1) % kStages));
+      if (gs == G - 1) announce(gs);
+      issue(gs + kCStages - 1);
     }
     ptx::cp_async_wait<0>();
-    while (ok && drained < num_chunks) {
-      if (!drain(drained++)) {
-        fail();
-        ok = false;
-      }
-    }
-    if (ok) {
-      const int nrow = n0 + rt;
-      if (nrow < N) {
-#pragma unroll
-        for (int j = 0; j < kCols; ++j) {
-          const int m = m0 + kCols * p + j;
-          if (m < M) y[static_cast<size_t>(m) * N + nrow] = run[j] * (g * tok_scale[m]);
-        }
-      }
-    }
   }
 
   // Neither CTA leaves (or frees tensor memory) while the pair's MMAs or the
@@ -534,6 +720,59 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// The tiles whose K stages were split over several pairs: y = g * tok_scale *
+// (sum of the parts in K order).  Grid (R, 2): the R stream-K tiles and the
+// two CTAs' 128-row halves; 256 threads, thread (rt, p) as in the epilogue.
+// A tile done by one pair was stored by the GEMM.
+__global__ void __launch_bounds__(kExpThreads)
+gemm_fixup_kernel(const float* __restrict__ parts, int T, int P, int num_kb, int mt, int np,
+                  int tok_fast, int N, int M, float g, const float* __restrict__ tok_scale,
+                  float* __restrict__ y) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // the GEMM's parts are written
+  const int T_dp = T / P * P;
+  const int64_t U_r = static_cast<int64_t>(T - T_dp) * num_kb;
+  const int tr = blockIdx.x;
+  const int r = blockIdx.y;
+  const int64_t ts = static_cast<int64_t>(tr) * num_kb, te = ts + num_kb;
+  auto start = [&](int i) { return U_r * i / P; };
+  // the pair whose stream-K stages include ts
+  int i0 = static_cast<int>(ts * P / U_r);
+  while (i0 + 1 < P && start(i0 + 1) <= ts) ++i0;
+  while (i0 > 0 && start(i0) > ts) --i0;
+  int parts_n = 0;
+  for (int i = i0; i < P && start(i) < te; ++i)
+    if (max(start(i), ts) < min(start(i + 1), te)) ++parts_n;
+  if (parts_n < 2) return;
+  const int t = threadIdx.x;
+  const int p = t / kBN, rt = t % kBN;
+  constexpr int kCols = kBT / kTPR;
+  float acc[kCols];
+  bool first = true;
+  for (int i = i0; i < P && start(i) < te; ++i) {
+    if (max(start(i), ts) >= min(start(i + 1), te)) continue;
+    const float4* slot = part_slot(const_cast<float*>(parts), 2 * i + r, start(i) >= ts ? 0 : 1);
+#pragma unroll
+    for (int j = 0; j < kCols; j += 4) {
+      const float4 v = __ldcg(slot + (p * (kCols / 4) + j / 4) * kBN + rt);
+      if (first) {
+        acc[j] = v.x, acc[j + 1] = v.y, acc[j + 2] = v.z, acc[j + 3] = v.w;
+      } else {
+        acc[j] += v.x, acc[j + 1] += v.y, acc[j + 2] += v.z, acc[j + 3] += v.w;
+      }
+    }
+    first = false;
+  }
+  int tt, wp;
+  tile_coords(T_dp + tr, mt, np, tok_fast, tt, wp);
+  const int nrow = (wp * 2 + r) * kBN + rt;
+  if (nrow >= N) return;
+#pragma unroll
+  for (int j = 0; j < kCols; ++j) {
+    const int m = tt * kBT + kCols * p + j;
+    if (m < M) y[static_cast<size_t>(m) * N + nrow] = acc[j] * (g * tok_scale[m]);
   }
 }
 
@@ -560,6 +799,49 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 int64_t padded_tokens(int64_t M) { return (M + kBT - 1) / kBT * kBT; }
+
+// Workspace of the prefill GEMM: the expanded activations [2 * M_pad, K]
+// fp16, the M_pad token scales, then two part slots (64 KB each) for every
+// CTA a launch may have (one per SM).
+size_t parts_offset(int64_t M, int64_t K) {
+  const int64_t mp = padded_tokens(M);
+  return static_cast<size_t>((4 * mp * K + 4 * mp + 255) / 256 * 256);
+}
+size_t parts_bytes() {
+  return static_cast<size_t>(device_sm_count()) * 2 * kPartFloats * sizeof(float);
+}
+
+// CTA pairs of the GEMM that fit on the device at once (cached per device)
+int gemm_pairs() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return device_sm_count() / 2;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int pairs = device_sm_count() / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute cluster[1];
+  cluster[0].id = cudaLaunchAttributeClusterDimension;
+  cluster[0].val.clusterDim.x = 2;
+  cluster[0].val.clusterDim.y = 1;
+  cluster[0].val.clusterDim.z = 1;
+  cfg.attrs = cluster;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel, &cfg) == cudaSuccess && n > 0)
+    pairs = std::min(pairs, n);
+  else
+    cudaGetLastError();   // leave no sticky error behind; keep the SM-count bound
+  pairs = std::max(pairs, 1);
+  if (dev >= 0 && dev < kMaxDevices) cache[dev].store(pairs, std::memory_order_relaxed);
+  return pairs;
+}
 
 // token counts that nvq_gemm hands to the decode GEMV
 constexpr int64_t kGemvTokensMax = 4;
@@ -589,8 +871,7 @@ CtxGetCurrentFn ctx_get_current() {
 
 size_t gemm_workspace_size(int64_t M, int64_t, int64_t K) {
   if (gemm_small_supported(M, K)) return gemm_small_workspace_size(M, K);
-  const int64_t mp = padded_tokens(M);
-  return static_cast<size_t>(4 * mp * K + 4 * mp);
+  return parts_offset(M, K) + parts_bytes();
 }
 
 size_t gemm_noalloc_limit() { return kNoAllocScratchBytes; }
@@ -677,14 +958,17 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   static SmemAttrOnce attr;
   cudaError_t e = attr.ensure(gemm_kernel, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  // pairs of CTAs along N: an even number of 128-row tiles (an odd last
-  // tile gets an all-padding partner)
-  const int64_t tiles_n = (N + kBN - 1) / kBN;
-  const int64_t ctas = (tiles_n + 1) / 2 * 2 * (M_pad / kBT);
-  if (ctas > INT32_MAX) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(ctas));
+  // tiles: 128 tokens x a pair of 128-row weight tiles (an odd last tile
+  // gets an all-padding partner)
+  const int64_t mt = M_pad / kBT;
+  const int64_t np = ((N + kBN - 1) / kBN + 1) / 2;
+  const int64_t T = mt * np;
+  const int64_t num_kb = (K + kBK - 1) / kBK;
+  if (T > INT32_MAX / 2 || T * num_kb > INT32_MAX) return cudaErrorInvalidValue;
+  const int P = static_cast<int>(std::min<int64_t>(gemm_pairs(), T * num_kb));
+  float* parts = reinterpret_cast<float*>(static_cast<uint8_t*>(act) + parts_offset(M, K));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * P));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
@@ -699,9 +983,28 @@ cudaError_t gemm_main(const uint8_t* codes, const uint8_t* scales, float g, int6
   // (0.5625 B per weight against 4 B per token and K of expanded activations)
   const int tok_fast = 9 * N >= 64 * M_pad ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, gemm_kernel, map, codes, scales, static_cast<int>(N),
-                                     static_cast<int>(K), static_cast<int>(M),
-                                     static_cast<int>(M_pad), g, tok_scale, y, tok_fast);
+                         static_cast<int>(K), static_cast<int>(M), static_cast<int>(M_pad), g,
+                         tok_scale, y, static_cast<int>(T), static_cast<int>(np), tok_fast,
+                         parts);
   if (e != cudaSuccess) return e;
+  // the stream-K tiles: add their parts
+  const int64_t R = T - T / P * P;
+  if (R > 0) {
+    cudaLaunchConfig_t fcfg = {};
+    fcfg.gridDim = dim3(static_cast<unsigned>(R), 2);
+    fcfg.blockDim = dim3(kExpThreads);
+    fcfg.stream = stream;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    fcfg.attrs = pdl;
+    fcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&fcfg, gemm_fixup_kernel, static_cast<const float*>(parts),
+                           static_cast<int>(T), P, static_cast<int>(num_kb),
+                           static_cast<int>(mt), static_cast<int>(np), tok_fast,
+                           static_cast<int>(N), static_cast<int>(M), g, tok_scale, y);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 
