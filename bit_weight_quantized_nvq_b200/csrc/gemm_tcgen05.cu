@@ -589,7 +589,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       tile_coords(tile, mt, np, tok_fast, tt, wp);
       const int nrow = tile_row(tile);
       const int m0t = tt * kBT + kCols * p;   // this thread's first token
-      float4* slot = part_slot(parts, blockIdx.x, slot_idx);
+      // the part's slot; a whole tile of several chunks keeps its running
+      // sum in slot 1 (free until the pair's last stream-K part, which comes
+      // after its whole tiles) and writes y only at its last chunk
+      float4* slot = part_slot(parts, blockIdx.x, to_y ? 1 : slot_idx) + p * (kCols / 4) * kBN + rt;
       const int this_dc = dc;
       dg += dn;
       ++dc;
@@ -600,18 +603,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
 #pragma unroll
       for (int j = 0; j < kCols; ++j) acc[j] = 0.0f;
       if (!first) {
-        if (to_y) {
-          if (nrow < N) {
 #pragma unroll
-            for (int j = 0; j < kCols; ++j)
-              if (m0t + j < M) acc[j] = __ldcg(y + static_cast<size_t>(m0t + j) * N + nrow);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < kCols; j += 4) {
-            const float4 o = __ldcg(slot + (p * (kCols / 4) + j / 4) * kBN + rt);
-            acc[j] = o.x, acc[j + 1] = o.y, acc[j + 2] = o.z, acc[j + 3] = o.w;
-          }
+        for (int j = 0; j < kCols; j += 4) {
+          const float4 o = __ldcg(slot + (j / 4) * kBN);
+          acc[j] = o.x, acc[j + 1] = o.y, acc[j + 2] = o.z, acc[j + 3] = o.w;
         }
       }
       if (!warp_wait(acc_full, this_dc & 1)) return false;
@@ -630,20 +625,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap act_map, const uint8_t* __restri
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(leader_acc_empty);
-      if (to_y) {
+      if (to_y && last) {
         if (nrow < N) {
 #pragma unroll
           for (int j = 0; j < kCols; ++j) {
             const int m = m0t + j;
-            if (m < M)
-              y[static_cast<size_t>(m) * N + nrow] = last ? acc[j] * (g * tok_scale[m]) : acc[j];
+            if (m < M) y[static_cast<size_t>(m) * N + nrow] = acc[j] * (g * tok_scale[m]);
           }
         }
       } else {
 #pragma unroll
         for (int j = 0; j < kCols; j += 4)
-          slot[(p * (kCols / 4) + j / 4) * kBN + rt] =
-              make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+          slot[(j / 4) * kBN] = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
       }
       return true;
     };
