@@ -497,7 +497,7 @@ class SmallGemmWorkload(GemvWorkload):
     the small-token tensor-core schedule; metric as the GEMV (weight GB/s)."""
 
     kernel = "gemm_small"
-    sources = ("gemm_small.cu", "gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+    sources = ("gemm_small.cu", "nvq_device.cuh", "tcgen05.cuh")   # the dominant kernel's code
     dtype = "nvfp4 x q8_0 (exact fp16 operands, fp32 accumulate)"
 
     def setup(self, device):
@@ -753,7 +753,7 @@ class W4A16Workload(GemvWorkload):
     shapes, one token; the activations are given in fp16 (no quantiser)."""
 
     kernel = "gemm_w4a16"
-    sources = ("gemm_small.cu", "gemm_tcgen05.cu", "nvq_device.cuh", "tcgen05.cuh")
+    sources = ("gemm_small.cu", "nvq_device.cuh", "tcgen05.cuh")   # the dominant kernel's code
     dtype = "nvfp4 x f16 (exact fp16 operands, fp32 accumulate)"
     metric = "nvfp4_f16_w4a16_weight_GBps"
 
