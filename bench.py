@@ -239,6 +239,19 @@ def profiled_traffic(kernel: str, workload: str, src_hash: str):
     return float(m_bytes.group(1))
 
 
+def gemm_launches(M: int, N: int, K: int) -> int:
+    """Kernels nvq_gemm launches after the Q8_0 expansion for M > 16 tokens:
+    the persistent tcgen05 GEMM, plus the fix-up of its stream-K tiles when
+    the tiles (128 tokens x 256 weight rows) do not divide evenly over the
+    CTA pairs (one pair per two SMs)."""
+    import torch
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    tiles = -(-M // 128) * -(-(-(-N // 128)) // 2)
+    stages = -(-K // 128)
+    P = min(pairs, tiles * stages)
+    return 1 + (1 if tiles % P else 0)
+
+
 def replay_ms(graph, stream) -> float:
     """Device time of one replay of a captured graph (CUDA events on the
     launching stream, synchronised on both sides)."""
@@ -556,7 +569,8 @@ class GemmWorkload(GemvWorkload):
         return 2.0 * self.M * N * K
 
     def launches_per_step(self):
-        return 3 * len(self.cases)       # quantise, expand, tcgen05 GEMM
+        # quantise, expand, tcgen05 GEMM (and the fix-up of its stream-K tiles)
+        return sum(2 + gemm_launches(self.M, c["N"], c["K"]) for c in self.cases)
 
     def dominant(self, c, codes, scales, stream):
         self.capi.gemm(codes, scales, c["g"], c["q"], c["d"], c["y"], c["ws"], stream=stream)
@@ -709,8 +723,13 @@ class StackWorkload:
         return float(self.M)                        # tokens
 
     def launches_per_step(self):
-        per_layer = 4 + 7 + (4 if self.M > 16 else 0)
-        return per_layer * self.n_layers
+        if self.M == 1:
+            # Q8_0 of the token, then the persistent stack kernel (64 layers a launch)
+            return 1 + -(-self.n_layers // 64)
+        if self.M <= 16:
+            return (4 + 7) * self.n_layers
+        # 4 quantisations and expansions, and the 7 GEMMs of every layer
+        return self.n_layers * (8 + sum(gemm_launches(self.M, N, K) for _, K, N in self.linears))
 
     def step(self, stream, e2e=False):
         if e2e:
