@@ -225,7 +225,9 @@ nvq_status nvq_moe_gemv(const uint8_t* codes, const uint8_t* scales, const float
 /*
  * nvq_gemm_workspace_size - bytes of device workspace nvq_gemm needs for
  * M tokens of K features (0 when M == 0).  It holds the activations
- * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q.
+ * expanded to the exact fp16 pair (hi, lo) with hi + lo = d*q and, for
+ * M > 16, two 64 KB slots of fp32 partial sums per SM of the current device
+ * (query it with the device that will run the GEMM current).
  */
 size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
@@ -244,11 +246,15 @@ size_t nvq_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *    (tokens padded to 8 or 16) takes the exact hi/lo activations (below)
  *    from shared memory; accumulators are promoted to fp32 registers every
  *    1024 K.  Results are deterministic.
- *  - otherwise: the prefill schedule on CTA pairs: weight tiles expanded in
- *    tensor memory, every 64-wide K slice multiplied by tcgen05.mma
- *    (kind::f16, cta_group::2) against hi and against lo into one fp32
- *    tensor-memory accumulator per 512-wide K chunk, whose partial sums are
- *    added in fp32 registers.
+ *  - otherwise: the prefill schedule on persistent CTA pairs (one per two
+ *    SMs): tiles of 128 tokens x 256 weight rows, the weights expanded in
+ *    tensor memory, one tcgen05.mma (kind::f16, cta_group::2, M = N = 256,
+ *    K = 16) per K-step forming the hi and the lo products in separate
+ *    accumulator columns; each chunk of up to 5120 K is added in fp32 (hi +
+ *    lo) to the tile's running sum.  Whole tiles go round-robin over the
+ *    pairs; the K stages of the last partial wave's tiles are split evenly
+ *    over all pairs, whose parts (fp32, in the workspace) a second launch
+ *    adds in K order.  Results are deterministic.
  *
  * The tensor-core schedules expand the activations once into `workspace` as
  * fp16 pairs hi = fp16(d*q), lo = fp16(d*q - hi), exact (hi + lo == d*q),
@@ -349,9 +355,10 @@ nvq_status nvq_gemm_nvf4(const uint8_t* w_codes, const uint8_t* w_scales, float 
  * Arguments, layouts, result and accuracy are those of nvq_gemm (y is the
  * same); there is no workspace argument.  Limit: the problem must fit the
  * scratch, nvq_gemm_workspace_size(M, N, K) <= 64 MiB, i.e. roughly
- * 4 * ceil(M/128)*128 * K bytes (for example M = 2048 up to K = 8160, or
- * M = 256 up to K = 65280); larger problems return NVQ_ERR_WORKSPACE and
- * should use nvq_gemm with a caller workspace.
+ * 4 * ceil(M/128)*128 * K bytes plus 128 KB per SM (on a 148-SM B200, for
+ * example M = 2048 up to K = 5760, or M = 256 up to K = 46528); larger
+ * problems return NVQ_ERR_WORKSPACE and should use nvq_gemm with a caller
+ * workspace.
  * Set-up: the first call on a device looks up the scratch's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  The address is cached per device and context;
