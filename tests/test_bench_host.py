@@ -171,3 +171,31 @@ def test_cpu_baseline_reports_one_core_and_all_cores():
     assert cb["cores"] == 1 and cb["kind"] == "oracle" and cb["value"] > 0
     assert cb["all_cores"]["cores"] == pool.cores and cb["all_cores"]["value"] > 0
     assert "64 rows" in cb["sample"]
+
+
+def test_launch_counts_follow_the_gemm_schedule(monkeypatch):
+    """The prefill GEMM adds a fix-up launch exactly when its tiles (128
+    tokens x 256 weight rows) do not divide evenly over the CTA pairs; the
+    one-token stack is one quantisation plus one persistent launch per 64
+    layers."""
+    import torch
+
+    class Props:
+        multi_processor_count = 148          # 74 CTA pairs
+
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda *a: Props())
+    # 320 and 1600 tiles over 74 pairs leave a partial wave; 74 tiles do not
+    assert bench.gemm_launches(2048, 5120, 5120) == 2
+    assert bench.gemm_launches(2048, 25600, 5120) == 2
+    assert bench.gemm_launches(256, 9472, 25600) == 1       # 2 x 37 tiles
+    assert bench.gemm_launches(128, 256, 128) == 1          # one tile, one stage
+    g = bench.GemmWorkload.__new__(bench.GemmWorkload)
+    g.M = 2048
+    g.cases = [{"K": 5120, "N": 5120}, {"K": 5120, "N": 9472}]
+    assert g.launches_per_step() == (2 + 2) + (2 + 1)          # 16 x 37 = 592 tiles: 8 whole waves
+    s = bench.StackWorkload.__new__(bench.StackWorkload)
+    s.n_layers, s.linears = 64, [("q", 5120, 5120)] * 7
+    s.M = 1
+    assert s.launches_per_step() == 2
+    s.M = 2048
+    assert s.launches_per_step() == 64 * (8 + 7 * 2)
