@@ -5,6 +5,9 @@
 * the full prefill shapes (M in {256, 2048}; (K, N) = (5120, 5120),
   (5120, 25600), (25600, 5120)): every element computed, a sample of rows and
   tokens checked against the oracle;
+* stream-K tails (the tiles of the last partial wave split over every CTA
+  pair): one tile in up to 74 parts, fewer leftover K stages than pairs,
+  a ragged last K stage; the split tiles' rows and tokens are checked;
 * tokens whose activations exceed the fp16 range (the 2^-e pre-scale);
 * fp32 outputs: |y - y_ref| <= 1e-5 * sum|terms| + 1e-6 per element.
 """
@@ -48,6 +51,33 @@ def test_prefill_full_size_sampled(M, K, N):
     q, d, q_ref, d_ref = quantize_both(x)
     y = run_gemm(P, q, d)
     toks = sample_rows(M, 192, seed=M * 7 + K)
+    y_ref, sa, _ = reference(P, q_ref[toks], d_ref[toks])
+    assert_within_tolerance(y[np.ix_(toks, rows)], y_ref, sa)
+    assert np.all(np.isfinite(y))
+
+
+# The persistent GEMM gives each of the CTA pairs (74 on a 148-SM B200) whole
+# tiles of 128 tokens x 256 weight rows round-robin and splits the K stages
+# of the tiles left over evenly.  With 300 tokens and 6400 rows there are
+# 3 x 25 = 75 tiles (token tiles run fastest here): one left over, the tile
+# of tokens 256..299 and rows 6144..6399.  At K = 25600 its 200 stages go to
+# all 74 pairs (2-3 each); at K = 1024 its 8 stages go to 8 pairs, the others
+# getting none.  With (130, 5184, 300) all 4 tiles are split, each of 41
+# stages whose last is 64 wide.
+@pytest.mark.parametrize("M,K,N,tail", [
+    (300, 25600, 6400, True), (300, 1024, 6400, True), (130, 5184, 300, False),
+])
+def test_stream_k_tails_sampled(M, K, N, tail):
+    W = wl.weights("gemm_test", "Wsk", N, K, boost_columns=True)
+    x = wl.activations("gemm_test", "xsk", M, K, "normal", outliers=True)
+    if tail:
+        rows = np.union1d(sample_rows(N, 32, seed=K), np.arange(6144, 6400, 3))
+        toks = np.union1d(sample_rows(M, 16, seed=K + 1), np.arange(256, 300))
+    else:
+        rows, toks = np.arange(N), np.arange(M)
+    P = Packed(W, rows)
+    q, d, q_ref, d_ref = quantize_both(x)
+    y = run_gemm(P, q, d)
     y_ref, sa, _ = reference(P, q_ref[toks], d_ref[toks])
     assert_within_tolerance(y[np.ix_(toks, rows)], y_ref, sa)
     assert np.all(np.isfinite(y))
