@@ -875,6 +875,7 @@ __device__ __forceinline__ bool stack_consume(const StackArgs& a, const StackCta
     const int li = l * kStackLin + m;
     const int rq = stack_rq(m);
     float* y = a.outs[m];
+    const float half_g = a.half_g[li];   // once per unit (see the producer)
     for (int row0 = r_begin; row0 < r_end; row0 += R, ++it) {
       const int nrows = min(R, r_end - row0);
       const int s = it % kM1Stages;
@@ -906,7 +907,7 @@ __device__ __forceinline__ bool stack_consume(const StackArgs& a, const StackCta
           const int row = row0 + rl;
           int how = 0;
           if (lane == 0) {
-            y[row] = acc * a.half_g[li];
+            y[row] = acc * half_g;
             if (rq >= 0) {
               // rows of this CTA per 32-row block counted in shared memory
               // (reset by the row that completes the CTA's share), the share
@@ -1022,6 +1023,10 @@ stack_m1_kernel(const __grid_constant__ StackArgs a) {
       const int r_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * N / G);
       const int r_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * N / G);
       const int li = l * kStackLin + m;
+      // the unit's matrix, read once from the launch parameters (a lookup
+      // with a dynamic index is a generic load that a store may not pass)
+      const uint8_t* const codes = a.codes[li];
+      const uint8_t* const scales = a.scales[li];
       for (int row0 = r_begin; row0 < r_end; row0 += R) {
         const int nrows = min(R, r_end - row0);
         const int s = it % kM1Stages;
@@ -1044,11 +1049,10 @@ stack_m1_kernel(const __grid_constant__ StackArgs a) {
         const uint32_t bar = ptx::smem_addr(full + s);
         uint8_t* st = smem + s * kRegStageMax;
         ptx::mbar_arrive_expect_tx(bar, nrows * (row_code + row_scale));
-        ptx::bulk_load(ptx::smem_addr(st), a.codes[li] + static_cast<size_t>(row0) * row_code,
+        ptx::bulk_load(ptx::smem_addr(st), codes + static_cast<size_t>(row0) * row_code,
                        nrows * row_code, bar);
         ptx::bulk_load(ptx::smem_addr(st + codes_bytes),
-                       a.scales[li] + static_cast<size_t>(row0) * row_scale, nrows * row_scale,
-                       bar);
+                       scales + static_cast<size_t>(row0) * row_scale, nrows * row_scale, bar);
         ++it;
       }
     }
