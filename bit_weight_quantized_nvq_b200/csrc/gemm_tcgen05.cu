@@ -11,7 +11,7 @@
 //
 //  * weights: w' = E2M1(code) * s_w is exact in fp16 (at most 6 significant
 //    bits, range 2^-10 .. 2688), so the per-16 rescale is folded into the
-//    operand, expanded in shared memory from the packed codes;
+//    operand, expanded into tensor memory from the packed codes;
 //  * activations: a = d*q has at most 18 significant bits, so it is split
 //    into the exact fp16 pair hi = fp16(a), lo = fp16(a - hi) (hi + lo == a;
 //    lo is a multiple of the ulp of d and below half an ulp of hi);
@@ -21,16 +21,20 @@
 //    error grows with the number of chained MMAs and is biased toward
 //    zero: about 1e-5 of sum|terms| after 1600 of them at K = 25600), so
 //    partial sums are promoted: each chunk of up to 5120 K accumulates in TMEM
-//    and the epilogue threads add it to fp32 registers (round to nearest).
+//    and the epilogue threads add it (hi + lo) to the tile's running sum in
+//    fp32 (round to nearest).
 //
 // Kernels:
 //  1. expand_act_kernel: Q8_0 (q, d) -> fp16 [hi rows | lo rows] in the
 //     caller's workspace, once per call (tokens padded to 128 with zeros).
 //     A token whose largest |d*q| would overflow fp16 (|x| > 65504) is
 //     scaled by 2^-e first and the epilogue multiplies by 2^e.
-//  2. gemm_kernel: CTA pairs (clusters of 2).  Each CTA owns 128 weight
-//     rows; the pair shares a tile of 128 tokens and the even CTA issues
-//     tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16) for both:
+//  2. gemm_kernel: persistent CTA pairs (clusters of 2, one per two SMs).
+//     A tile is 128 tokens x 256 weight rows; each CTA owns 128 of the rows
+//     and the even CTA issues tcgen05.mma.cta_group::2 (M = 256, N = 256,
+//     K = 16) for both.  Whole tiles go round-robin over the pairs; the K
+//     stages of the last partial wave's tiles are split evenly over all
+//     pairs (PairWork).  Roles:
 //       warp 0    TMA: this CTA's hi and lo rows of 64 of the tokens, for
 //                 the two 64-wide K sub-tiles of a 128-wide stage (four
 //                 64 x 64 fp16 boxes, 128-byte swizzle), into a 4-stage ring;
@@ -44,15 +48,19 @@
 //       warps 2-9 two threads per weight row, one per sub-tile: cp.async the
 //                 packed codes and scales, decode them to fp16 w' and
 //                 tcgen05.st them into the 4-stage A ring in tensor memory
-//                 (row m in lane m); drain finished K chunks
-//                 (hi + lo of each token) into fp32 registers; store y;
+//                 (row m in lane m); drain each finished K chunk (hi + lo
+//                 of each token) into y (a whole tile's last chunk, scaled)
+//                 or the fp32 part slot of the workspace;
 //       warp 10   forwards "this CTA's rows of the stage landed" to the even
 //                 CTA's stage barrier.
 //     Every role runs with its whole warp converged on the waits (a wait in
 //     a diverged lane stalls the issuing loop by ~150-200 cycles a stage)
 //     and one lane issuing.  Every wait is bounded (4 s); a timeout raises
 //     an error flag and the CTA drains what it issued, and the pair frees
-//     TMEM together after a cluster barrier.
+//     TMEM together after a cluster barrier.  No CTA waits for another
+//     pair.
+//  3. gemm_fixup_kernel: y of the tiles whose stages were split, the parts
+//     added in K order (results do not depend on timing).
 #include <algorithm>
 #include <atomic>
 #include <climits>
