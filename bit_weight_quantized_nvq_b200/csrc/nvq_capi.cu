@@ -83,11 +83,24 @@ nvq_status check_dot_args(const void* codes, const void* scales, int64_t N,
 namespace nvq {
 void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = e; }
 
+// SMs of the current device: cached on first use (the workspace sizes that
+// depend on it are queried before any launch), 148 without a device.
 int device_sm_count() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return 148;
   int sms = g_device_sms[dev].load(std::memory_order_relaxed);
-  return sms > 0 ? sms : 148;
+  if (sms > 0) return sms;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  g_device_sms[dev].store(sms, std::memory_order_relaxed);
+  return sms;
 }
 }  // namespace nvq
 
