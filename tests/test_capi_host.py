@@ -166,3 +166,81 @@ def test_host_packer_matches_oracle_bit_exactly(case):
     assert np.float32(g) == go
     assert np.array_equal(s, so)
     assert np.array_equal(c, co)
+
+
+def test_host_validation_of_the_other_entry_points():
+    """MoE, W4A16, NVFP4 x NVFP4, the allocation-free GEMM and the decoder
+    stack refuse bad arguments on the host, before any device call."""
+    lib = capi.lib()
+    keep = []
+
+    def p(nbytes=4096, off=0):
+        b, a = _dev_like(nbytes, off)
+        keep.append(b)
+        return a
+
+    codes, scales, q, d, y, ids, gs = p(), p(), p(), p(), p(), p(), p()
+    moe = lib.nvq_moe_gemv        # codes, scales, g[E], E, N, K, ids, T, top_k, q, d, y, stream
+    assert moe(codes, scales, gs, 4, 64, 96, ids, 2, 2, q, d, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert moe(codes, scales, gs, 4, 64, 2048, ids, 2, 9, q, d, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert moe(codes, scales, gs, 0, 64, 2048, ids, 2, 2, q, d, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert moe(codes, scales, gs, 4, 64, 2048, None, 2, 2, q, d, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert moe(codes, scales, gs, 4, 64, 2048, p(off=4), 2, 2, q, d, y, None) == capi.NVQ_ERR_MISALIGNED
+    assert moe(codes, scales, gs, 4, 64, 2048, ids, 0, 2, q, d, y, None) == capi.NVQ_OK
+
+    w4 = lib.nvq_gemm_w4a16       # codes, scales, g, N, K, x, M, y, ws, ws_bytes, stream
+    assert lib.nvq_gemm_w4a16_workspace_size(17, 8, 256) == 0
+    assert lib.nvq_gemm_w4a16_workspace_size(1, 8, 192) == 0
+    need = lib.nvq_gemm_w4a16_workspace_size(4, 8, 256)
+    assert need > 0
+    ws = p(need)
+    assert w4(codes, scales, 1.0, 8, 192, q, 4, y, ws, need, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert w4(codes, scales, 1.0, 8, 256, q, 17, y, ws, need, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert w4(codes, scales, float("nan"), 8, 256, q, 4, y, ws, need, None) == capi.NVQ_ERR_INVALID_ARG
+    assert w4(codes, scales, 1.0, 8, 256, q, 4, y, None, need, None) == capi.NVQ_ERR_WORKSPACE
+    assert w4(codes, scales, 1.0, 8, 256, q, 4, y, ws, need - 1, None) == capi.NVQ_ERR_WORKSPACE
+    assert w4(codes, scales, 1.0, 8, 256, q, 0, y, None, 0, None) == capi.NVQ_OK
+
+    qn = lib.nvq_quantize_act_nvfp4   # x, M, K, codes, scales, g, stream
+    assert qn(p(), 2, 24, codes, scales, gs, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert qn(None, 2, 32, codes, scales, gs, None) == capi.NVQ_ERR_INVALID_ARG
+    assert qn(p(off=4), 2, 32, codes, scales, gs, None) == capi.NVQ_ERR_MISALIGNED
+    assert qn(None, 0, 32, None, None, None, None) == capi.NVQ_OK
+
+    nf = lib.nvq_gemm_nvf4        # w_codes, w_scales, g_w, N, K, a_codes, a_scales, a_g, M, y, stream
+    assert nf(codes, scales, 1.0, 8, 128, q, d, gs, 4, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert nf(codes, scales, 1.0, 65535 * 128 + 1, 256, q, d, gs, 4, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert nf(codes, scales, float("nan"), 8, 256, q, d, gs, 4, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert nf(codes, scales, 1.0, 8, 256, q, d, None, 4, y, None) == capi.NVQ_ERR_INVALID_ARG
+    assert nf(codes, scales, 1.0, 8, 256, q, d, gs, 4, p(off=8), None) == capi.NVQ_ERR_MISALIGNED
+    assert nf(codes, scales, 1.0, 0, 256, q, d, gs, 4, y, None) == capi.NVQ_OK
+
+    na = lib.nvq_gemm_noalloc     # codes, scales, g, N, K, q, d, M, y, stream
+    assert na(codes, scales, 1.0, 8, 96, q, d, 4, y, None) == capi.NVQ_ERR_BAD_SHAPE
+    # 2048 tokens of K = 25600 need ~200 MiB of expanded activations
+    assert na(codes, scales, 1.0, 128, 25600, q, d, 2048, y, None) == capi.NVQ_ERR_WORKSPACE
+    assert na(codes, scales, 1.0, 0, 64, q, d, 4, y, None) == capi.NVQ_OK
+
+    # decoder stack: hidden 64, MLP 128; q k v o up gate down
+    shapes = [(64, 64), (64, 64), (64, 64), (64, 64), (128, 64), (128, 64), (64, 128)]
+
+    def layers(n, g=1.0, bad_n=None, off=0):
+        arr = (capi.Linear * (7 * n))()
+        for l in range(n):
+            for i, (N, K) in enumerate(shapes):
+                arr[7 * l + i] = capi.Linear(p(off=off), p(), g, N if bad_n != (l, i) else N + 1, K)
+        return arr
+
+    outs = (ctypes.c_void_p * 7)(*[p(16384) for _ in range(7)])
+    x = p()
+    st = lib.nvq_decoder_stack    # linears, n_layers, x, M, outs, ws, ws_bytes, stream
+    good = layers(2)
+    need = lib.nvq_decoder_stack_workspace_size(good, 1)
+    assert need > 0
+    ws = p(need)
+    assert st(good, 0, x, 1, outs, ws, need, None) == capi.NVQ_OK
+    assert st(layers(2, bad_n=(1, 4)), 2, x, 1, outs, ws, need, None) == capi.NVQ_ERR_BAD_SHAPE
+    assert st(layers(2, g=float("nan")), 2, x, 1, outs, ws, need, None) == capi.NVQ_ERR_INVALID_ARG
+    assert st(layers(2, off=4), 2, x, 1, outs, ws, need, None) == capi.NVQ_ERR_MISALIGNED
+    assert st(good, 2, x, 1, outs, ws, need - 1, None) == capi.NVQ_ERR_WORKSPACE
+    assert st(good, 2, x, 1, None, ws, need, None) == capi.NVQ_ERR_INVALID_ARG
